@@ -1,0 +1,217 @@
+/*
+ * moe_gemv.h -- C ABI of the B200 (sm_100a) weight-streaming hot path of
+ * batch-1 mixture-of-experts decode.
+ *
+ * What the path computes (sources: the web pages on NVIDIA's "3 ways to boost
+ * MoE inference on DGX Spark" write-up; the number formats come from the OCP
+ * specifications named below):
+ *
+ *  - The routed-expert MoE layer.  Each token goes to k of E routed experts
+ *    plus one shared expert that always runs (saipien.org essay, "Why one user
+ *    waits on weights": 8 of 512 routed experts plus one shared expert).  Its
+ *    weights are MXFP4 (same essay, "Why one user waits on weights": an FP4
+ *    checkpoint; generativeaipub.com blog, "DGX Spark Can Hold the Whole
+ *    Model": MXFP4 weights) and the expert layer is narrow, intermediate 768
+ *    (saipien.org essay, "Kernels built for the shape you actually have").  The
+ *    verify step scores 4 positions in one pass and wakes up to 32 routed
+ *    experts (saipien.org essay, "Draft three tokens, verify four").
+ *  - The online-FP8 LM head: the 157,184 x 2,560 BF16 vocabulary projection is
+ *    quantised to FP8 once, when the layer is built, which halves the bytes
+ *    each token reads (ncijnetwork.com summary, "What are the 3
+ *    optimizations?", item 2; generativeaipub.com blog, "2. Compressing the
+ *    Output Head").  Decode reads the whole head every token and keeps the
+ *    top-k token ids (greedy decoding takes k = 1; the sampled workload on the
+ *    same page uses top_k 29).
+ *
+ * Readings where the pages are silent:
+ *  - routing: softmax over the E routed logits (plus an optional per-expert
+ *    bias), top-k, renormalised over the selected k; ties go to the lower id;
+ *  - each expert is a SwiGLU MLP: h = silu(gate x) * (up x), out = down h;
+ *    the shared expert has weight 1;
+ *  - FP8 head: per-row fp32 scale s = amax / 448, q = E4M3 RNE satfinite of
+ *    w / s; logit = s * sum_j q_j x_j; activations stay bf16;
+ *  - MXFP4 per OCP Microscaling Formats v1.0: E2M1 codes (bit 3 = sign),
+ *    one E8M0 scale per 32 elements along K, scale exponent
+ *    floor(log2(amax)) - 2 clamped to [-127, 127], elements rounded to
+ *    nearest even and saturated at +-6, element 2j in the low nibble of byte j;
+ *  - E4M3 per the OCP 8-bit Floating Point Specification (bias 7, max 448).
+ *
+ * Conventions for every call:
+ *  - All tensors are row-major and contiguous in device memory that the caller
+ *    owns (allocated with cudaMalloc or by torch).  The library never allocates
+ *    or frees device memory.  Device pointers must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Work is enqueued asynchronously; no call synchronises the host
+ *    except moe_workspace_status().
+ *  - Argument errors are returned before anything is enqueued.  Argument
+ *    checks touch no CUDA API, so they also run on a machine without a GPU.
+ *  - Quantised tensors carry a format tag that every call checks: passing a
+ *    BF16-tagged head where the FP8 one is expected returns
+ *    MOE_ERR_FORMAT_MISMATCH instead of silently reading FP8 bytes as BF16
+ *    (the integration trap described in the ncijnetwork.com summary, "What
+ *    are the 3 optimizations?", paragraph "The integration trap").
+ *  - Calls are reentrant: all mutable state lives in the caller's workspace.
+ *    Two calls that run at the same time on the GPU must use different
+ *    workspaces.
+ */
+#ifndef MOE_GEMV_H
+#define MOE_GEMV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,       /* NULL pointer, non-positive size, bad M or top_k  */
+    MOE_ERR_UNSUPPORTED_SHAPE = -2, /* a shape this build was not compiled for          */
+    MOE_ERR_MISALIGNED = -3,        /* a device pointer not 16-byte aligned             */
+    MOE_ERR_FORMAT_MISMATCH = -4,   /* wrong format tag on a quantised tensor           */
+    MOE_ERR_WORKSPACE = -5,         /* workspace missing or smaller than required       */
+    MOE_ERR_CUDA = -6,              /* a CUDA runtime call failed (launch, query)        */
+    MOE_ERR_TIMEOUT = -7,           /* a bounded device-side wait ran out (see status)  */
+    MOE_ERR_DEVICE_CHECK = -8       /* a device-side check failed (see status)          */
+} moe_status;
+
+typedef enum {
+    MOE_FMT_NONE = 0,
+    MOE_FMT_BF16 = 1,
+    MOE_FMT_MXFP4_E2M1_E8M0_32 = 2,
+    MOE_FMT_FP8_E4M3_ROWSCALE_F32 = 3
+} moe_format;
+
+/* A stack of `count` MXFP4 matrices, each [rows][K]:
+ *   data   [count][rows][K/2] : E2M1 codes, element 2j in the low nibble of byte j
+ *   scales [count][rows][K/32]: E8M0 block scales, 2^(code - 127)
+ * K must be a multiple of 32.  fmt must be MOE_FMT_MXFP4_E2M1_E8M0_32.          */
+typedef struct {
+    int32_t fmt;
+    int32_t count;
+    int64_t rows;
+    int64_t K;
+    uint8_t* data;
+    uint8_t* scales;
+} moe_mxfp4_tensor;
+
+/* The experts of one MoE layer, each a SwiGLU MLP:
+ *   gate, up: count x [I][H];  down: count x [H][I].
+ * The routed bank has count = E; the shared expert is a bank with count = 1.  */
+typedef struct {
+    moe_mxfp4_tensor gate;
+    moe_mxfp4_tensor up;
+    moe_mxfp4_tensor down;
+} moe_expert_bank;
+
+/* The online-FP8 LM head: q [vocab][hidden] E4M3 and row_scale [vocab] fp32.
+ * fmt must be MOE_FMT_FP8_E4M3_ROWSCALE_F32.                                   */
+typedef struct {
+    int32_t fmt;
+    int64_t vocab;
+    int64_t hidden;
+    uint8_t* q;
+    float* row_scale;
+} moe_fp8_head;
+
+/* The unquantised BF16 LM head [vocab][hidden] (the comparator path).
+ * fmt must be MOE_FMT_BF16.                                                    */
+typedef struct {
+    int32_t fmt;
+    int64_t vocab;
+    int64_t hidden;
+    uint16_t* w;
+} moe_bf16_head;
+
+/* ---- load time ------------------------------------------------------------ */
+
+/* Quantise `count` bf16 matrices w [count][rows][K] into `out`, whose count,
+ * rows, K, data and scales the caller fills in (buffers of the sizes above).
+ * On success sets out->fmt = MOE_FMT_MXFP4_E2M1_E8M0_32.  Blocks that hold an
+ * Inf or NaN get scale code 0xFF (NaN) and element codes 0.  Bit-exact with
+ * the OCP MX conversion rule stated at the top of this header.               */
+MOE_API moe_status moe_quantize_mxfp4(const uint16_t* w_bf16, moe_mxfp4_tensor* out, void* stream);
+
+/* Quantise the bf16 head w [vocab][hidden] into `out` (caller fills vocab,
+ * hidden, q, row_scale): s_v = fp32(amax_v / 448) (1 for an all-zero row),
+ * q = E4M3 RNE satfinite of fp32(w / s_v).  On success sets out->fmt.
+ * The ncijnetwork.com summary, "What are the 3 optimizations?", item 2:
+ * quantising only this layer to FP8 at load time.                           */
+MOE_API moe_status lmhead_quantize_fp8(const uint16_t* w_bf16, moe_fp8_head* out, void* stream);
+
+/* ---- decode --------------------------------------------------------------- */
+
+/* Bytes of workspace moe_decode needs for these sizes (0 if unsupported).    */
+MOE_API size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts,
+                           int32_t hidden, int32_t inter);
+
+/* One MoE layer for M tokens (1 <= M <= 4):
+ *   hidden      [M][H] bf16
+ *   router_w    [E][H] fp32;  router_bias [E] fp32 or NULL (added to the logits)
+ *   experts     routed bank (count E), shared: bank with count 1 (host structs)
+ *   out         [M][H] fp32:  sum_i w_i expert_{id_i}(x) + shared(x)
+ *   topk_ids    [M][top_k] int32 or NULL: selected experts, by descending logit
+ *   topk_w      [M][top_k] fp32 or NULL:  renormalised softmax weights
+ *   workspace   device buffer of at least moe_workspace_bytes(...) bytes,
+ *               zeroed once (moe_workspace_reset) before its first use.
+ * Supported: H and I multiples of 32 and at most 8192, E <= 1024,
+ * 1 <= top_k <= 8 and top_k <= E.  Each distinct routed expert is streamed once per call, however
+ * many of the M tokens chose it.                                             */
+MOE_API moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const float* router_bias,
+                      const moe_expert_bank* experts, const moe_expert_bank* shared,
+                      int32_t M, int32_t top_k, float* out, int32_t* topk_ids, float* topk_w,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace lmhead_decode / lmhead_decode_bf16 need (0 if unsupported). */
+MOE_API size_t lmhead_workspace_bytes(int32_t M, int32_t top_k, int64_t vocab, int64_t hidden);
+
+/* FP8 LM head for M tokens (1 <= M <= 4), fused with top-k:
+ *   hidden   [M][H] bf16;  head: the quantised head (tag checked)
+ *   topk_ids [M][top_k] int32, topk_vals [M][top_k] fp32: the top_k largest
+ *            logits, descending, ties to the lower token id (top_k = 1 is the
+ *            greedy argmax); 1 <= top_k <= 64
+ *   logits   [M][vocab] fp32 or NULL: every logit, when the caller wants them
+ *   workspace: at least lmhead_workspace_bytes(...), zeroed once before use.
+ * Supported: hidden a multiple of 64 and at most 5120, vocab < 2^31.       */
+MOE_API moe_status lmhead_decode(const uint16_t* hidden_bf16, const moe_fp8_head* head,
+                         int32_t M, int32_t top_k, int32_t* topk_ids, float* topk_vals,
+                         float* logits, void* workspace, size_t workspace_bytes, void* stream);
+
+/* The same with the unquantised BF16 head (the comparator the FP8 head halves);
+ * hidden a multiple of 32 and at most 2560.                                 */
+MOE_API moe_status lmhead_decode_bf16(const uint16_t* hidden_bf16, const moe_bf16_head* head,
+                              int32_t M, int32_t top_k, int32_t* topk_ids, float* topk_vals,
+                              float* logits, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- housekeeping --------------------------------------------------------- */
+
+/* Zero a workspace (async memset on `stream`).  Needed once before first use,
+ * and after a call reported MOE_ERR_TIMEOUT.                                 */
+MOE_API moe_status moe_workspace_reset(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, read the device status word that kernels set in this
+ * workspace (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK), clear it, and
+ * return it.  Device-side waits in these kernels are bounded: a wait that
+ * runs out sets the status word and the kernel returns instead of hanging.   */
+MOE_API moe_status moe_workspace_status(void* workspace, void* stream);
+
+/* Write a NUL-terminated description of the compiled kernels and formats
+ * ("sm_100a ...") into buf.  The pages advise confirming at startup that each
+ * optimisation is live (ncijnetwork.com summary, "The integration trap");
+ * this is the string to log.                                                 */
+MOE_API moe_status moe_query_path(char* buf, size_t n);
+
+/* Text for a status code ("MOE_ERR_FORMAT_MISMATCH", ...); never NULL.       */
+MOE_API const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

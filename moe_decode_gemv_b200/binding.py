@@ -1,0 +1,262 @@
+"""Thin Python binding of the C ABI in include/moe_gemv.h.
+
+Argument marshalling only: every step of the hot path runs in the CUDA
+kernels of libmoe_gemv.so.  Tensors are torch CUDA tensors (torch provides
+device memory and streams); the calls pass their data pointers and the
+current CUDA stream through ctypes.  Importing this module loads the
+library and raises if it is missing -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import enum
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libmoe_gemv.so")
+
+
+class Status(enum.IntEnum):
+    OK = 0
+    INVALID_ARG = -1
+    UNSUPPORTED_SHAPE = -2
+    MISALIGNED = -3
+    FORMAT_MISMATCH = -4
+    WORKSPACE = -5
+    CUDA = -6
+    TIMEOUT = -7
+    DEVICE_CHECK = -8
+
+
+class Format(enum.IntEnum):
+    NONE = 0
+    BF16 = 1
+    MXFP4_E2M1_E8M0_32 = 2
+    FP8_E4M3_ROWSCALE_F32 = 3
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = Status(status)
+        super().__init__(f"{call} returned {self.status.name}")
+
+
+class _Mxfp4(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("count", ctypes.c_int32), ("rows", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("data", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class _Bank(ctypes.Structure):
+    _fields_ = [("gate", _Mxfp4), ("up", _Mxfp4), ("down", _Mxfp4)]
+
+
+class _Fp8Head(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("vocab", ctypes.c_int64), ("hidden", ctypes.c_int64),
+                ("q", ctypes.c_void_p), ("row_scale", ctypes.c_void_p)]
+
+
+class _Bf16Head(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("vocab", ctypes.c_int64), ("hidden", ctypes.c_int64),
+                ("w", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(library_path):
+        raise ImportError(f"{library_path} is missing: build it with `python -m moe_decode_gemv_b200.build` "
+                          "(the CUDA path has no fallback)")
+    L = ctypes.CDLL(library_path)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "moe_quantize_mxfp4": ([P, ctypes.POINTER(_Mxfp4), P], I32),
+        "lmhead_quantize_fp8": ([P, ctypes.POINTER(_Fp8Head), P], I32),
+        "moe_workspace_bytes": ([I32, I32, I32, I32, I32], SZ),
+        "moe_decode": ([P, P, P, ctypes.POINTER(_Bank), ctypes.POINTER(_Bank), I32, I32, P, P, P, P, SZ, P], I32),
+        "lmhead_workspace_bytes": ([I32, I32, I64, I64], SZ),
+        "lmhead_decode": ([P, ctypes.POINTER(_Fp8Head), I32, I32, P, P, P, P, SZ, P], I32),
+        "lmhead_decode_bf16": ([P, ctypes.POINTER(_Bf16Head), I32, I32, P, P, P, P, SZ, P], I32),
+        "moe_workspace_reset": ([P, SZ, P], I32),
+        "moe_workspace_status": ([P, P], I32),
+        "moe_query_path": ([ctypes.c_char_p, SZ], I32),
+        "moe_status_string": ([I32], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    return L
+
+
+library = _load()
+
+
+def _check(status: int, call: str) -> None:
+    if status != 0:
+        raise MoEError(status, call)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ---------------------------------------------------------------------------
+# quantised containers
+# ---------------------------------------------------------------------------
+
+@dataclass
+class MXFP4Bank:
+    """A stack of `count` MXFP4 matrices [rows][K]: data [count, rows, K/2]
+    uint8 (element 2j in the low nibble of byte j) and scales [count, rows,
+    K/32] uint8 (E8M0)."""
+    data: torch.Tensor
+    scales: torch.Tensor
+    fmt: int = Format.NONE
+
+    @property
+    def count(self) -> int:
+        return self.data.shape[0]
+
+    @property
+    def rows(self) -> int:
+        return self.data.shape[1]
+
+    @property
+    def K(self) -> int:
+        return self.data.shape[2] * 2
+
+    def _c(self) -> _Mxfp4:
+        return _Mxfp4(int(self.fmt), self.count, self.rows, self.K, self.data.data_ptr(), self.scales.data_ptr())
+
+    def nbytes(self) -> int:
+        return self.data.numel() + self.scales.numel()
+
+
+def alloc_mxfp4_bank(count: int, rows: int, K: int, device="cuda") -> MXFP4Bank:
+    return MXFP4Bank(torch.empty((count, rows, K // 2), dtype=torch.uint8, device=device),
+                     torch.empty((count, rows, K // 32), dtype=torch.uint8, device=device))
+
+
+@dataclass
+class FP8Head:
+    """The online-FP8 LM head: q [V, H] uint8 (E4M3) and row_scale [V] fp32."""
+    q: torch.Tensor
+    row_scale: torch.Tensor
+    fmt: int = Format.NONE
+
+    def _c(self) -> _Fp8Head:
+        return _Fp8Head(int(self.fmt), self.q.shape[0], self.q.shape[1], self.q.data_ptr(), self.row_scale.data_ptr())
+
+
+def alloc_fp8_head(vocab: int, hidden: int, device="cuda") -> FP8Head:
+    return FP8Head(torch.empty((vocab, hidden), dtype=torch.uint8, device=device),
+                   torch.empty((vocab,), dtype=torch.float32, device=device))
+
+
+def _bank_c(gate: MXFP4Bank, up: MXFP4Bank, down: MXFP4Bank) -> _Bank:
+    return _Bank(gate._c(), up._c(), down._c())
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+
+def moe_quantize_mxfp4(w_bf16: torch.Tensor, out: MXFP4Bank | None = None, stream=None) -> MXFP4Bank:
+    """bf16 [count, rows, K] (or [rows, K]) -> MXFP4 bank."""
+    w = w_bf16 if w_bf16.dim() == 3 else w_bf16.unsqueeze(0)
+    assert w.dtype == torch.bfloat16 and w.is_cuda and w.is_contiguous()
+    if out is None:
+        out = alloc_mxfp4_bank(w.shape[0], w.shape[1], w.shape[2], device=w.device)
+    c = out._c()
+    _check(library.moe_quantize_mxfp4(_ptr(w), ctypes.byref(c), _stream(stream)), "moe_quantize_mxfp4")
+    out.fmt = c.fmt
+    return out
+
+
+def lmhead_quantize_fp8(w_bf16: torch.Tensor, out: FP8Head | None = None, stream=None) -> FP8Head:
+    assert w_bf16.dtype == torch.bfloat16 and w_bf16.is_cuda and w_bf16.is_contiguous()
+    if out is None:
+        out = alloc_fp8_head(w_bf16.shape[0], w_bf16.shape[1], device=w_bf16.device)
+    c = out._c()
+    _check(library.lmhead_quantize_fp8(_ptr(w_bf16), ctypes.byref(c), _stream(stream)), "lmhead_quantize_fp8")
+    out.fmt = c.fmt
+    return out
+
+
+def moe_workspace_bytes(M: int, top_k: int, num_experts: int, hidden: int, inter: int) -> int:
+    return int(library.moe_workspace_bytes(M, top_k, num_experts, hidden, inter))
+
+
+def lmhead_workspace_bytes(M: int, top_k: int, vocab: int, hidden: int) -> int:
+    return int(library.lmhead_workspace_bytes(M, top_k, vocab, hidden))
+
+
+def new_workspace(nbytes: int, device="cuda", stream=None) -> torch.Tensor:
+    """A zeroed workspace buffer (16-byte aligned torch allocation)."""
+    ws = torch.empty((max(nbytes, 64),), dtype=torch.uint8, device=device)
+    _check(library.moe_workspace_reset(_ptr(ws), ws.numel(), _stream(stream)), "moe_workspace_reset")
+    return ws
+
+
+def moe_decode(hidden: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None,
+               experts: tuple[MXFP4Bank, MXFP4Bank, MXFP4Bank], shared: tuple[MXFP4Bank, MXFP4Bank, MXFP4Bank],
+               top_k: int, out: torch.Tensor, topk_ids: torch.Tensor | None = None,
+               topk_w: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One MoE layer: out[M, H] fp32 = sum_i w_i expert_i(x) + shared(x)."""
+    M = hidden.shape[0]
+    if workspace is None:
+        workspace = new_workspace(moe_workspace_bytes(M, top_k, experts[0].count, experts[0].K, experts[0].rows),
+                                  hidden.device, stream)
+    eb, sb = _bank_c(*experts), _bank_c(*shared)
+    st = library.moe_decode(_ptr(hidden), _ptr(router_w), _ptr(router_bias), ctypes.byref(eb), ctypes.byref(sb),
+                            M, top_k, _ptr(out), _ptr(topk_ids), _ptr(topk_w), _ptr(workspace), workspace.numel(),
+                            _stream(stream))
+    _check(st, "moe_decode")
+    return out
+
+
+def lmhead_decode(hidden: torch.Tensor, head: FP8Head, top_k: int, topk_ids: torch.Tensor, topk_vals: torch.Tensor,
+                  logits: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    M = hidden.shape[0]
+    if workspace is None:
+        workspace = new_workspace(lmhead_workspace_bytes(M, top_k, head.q.shape[0], head.q.shape[1]),
+                                  hidden.device, stream)
+    c = head._c()
+    st = library.lmhead_decode(_ptr(hidden), ctypes.byref(c), M, top_k, _ptr(topk_ids), _ptr(topk_vals), _ptr(logits),
+                               _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "lmhead_decode")
+    return topk_ids, topk_vals
+
+
+def lmhead_decode_bf16(hidden: torch.Tensor, w_bf16: torch.Tensor, top_k: int, topk_ids: torch.Tensor,
+                       topk_vals: torch.Tensor, logits: torch.Tensor | None = None,
+                       workspace: torch.Tensor | None = None, stream=None):
+    M = hidden.shape[0]
+    if workspace is None:
+        workspace = new_workspace(lmhead_workspace_bytes(M, top_k, w_bf16.shape[0], w_bf16.shape[1]),
+                                  hidden.device, stream)
+    c = _Bf16Head(int(Format.BF16), w_bf16.shape[0], w_bf16.shape[1], w_bf16.data_ptr())
+    st = library.lmhead_decode_bf16(_ptr(hidden), ctypes.byref(c), M, top_k, _ptr(topk_ids), _ptr(topk_vals),
+                                    _ptr(logits), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "lmhead_decode_bf16")
+    return topk_ids, topk_vals
+
+
+def moe_workspace_status(workspace: torch.Tensor, stream=None) -> Status:
+    return Status(library.moe_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def moe_query_path() -> str:
+    buf = ctypes.create_string_buffer(1024)
+    _check(library.moe_query_path(buf, len(buf)), "moe_query_path")
+    return buf.value.decode()
+
+
+def moe_get_device_status(workspace: torch.Tensor, stream=None) -> Status:
+    return moe_workspace_status(workspace, stream)

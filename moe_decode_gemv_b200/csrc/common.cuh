@@ -1,0 +1,193 @@
+// common.cuh -- device helpers shared by the sm_100a kernels of this library.
+//
+// Number formats (OCP Microscaling Formats v1.0; OCP 8-bit Floating Point
+// Specification): E2M1 and E4M3 codes are widened with the hardware
+// conversions of sm_100a (cvt.rn.f16x2.e2m1x2 / .e4m3x2), which are exact
+// because every E2M1 and E4M3 value is an f16 value.  E8M0 scales become
+// fp32 by placing the code in the exponent field.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/moe_gemv.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// Workspace header shared by every kernel: a status word and two counters.
+// It sits at the start of each caller-owned workspace.
+// ---------------------------------------------------------------------------
+struct WsHeader {
+  int32_t status;     // 0, or the first moe_status a kernel reported
+  uint32_t ticket;    // last-block-done counter (returns to 0 after each use)
+  uint32_t barrier;   // grid barrier word (sense-reversing; see grid_barrier)
+  uint32_t pad[13];   // keeps what follows on a 64-byte boundary
+};
+static_assert(sizeof(WsHeader) == 64, "workspace header is 64 bytes");
+
+__device__ __forceinline__ void report(WsHeader* h, moe_status s) {
+  atomicCAS(&h->status, 0, (int32_t)s);
+}
+
+// Upper bound on polls of any device-side wait before a kernel gives up,
+// records MOE_ERR_TIMEOUT and returns.  A poll takes tens of nanoseconds, so
+// this is seconds of waiting -- orders of magnitude above any healthy wait.
+constexpr uint32_t kSpinLimit = 1u << 26;
+
+// ---------------------------------------------------------------------------
+// Format conversions.
+// ---------------------------------------------------------------------------
+
+// Two E2M1 codes (low nibble = element 2j, high nibble = element 2j+1) -> f16x2
+// with element 2j in the low half.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "r"(byte));
+  return r;
+}
+
+// Two E4M3 codes (low byte = lower-index element) -> f16x2, low byte in the low half.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "r"(two_bytes));
+  return r;
+}
+
+// E8M0 code -> fp32 scale 2^(code - 127).  Code 0 is 2^-127 (a subnormal),
+// code 255 is NaN.
+__device__ __forceinline__ float e8m0_to_f32(uint32_t code) {
+  uint32_t bits = code == 0u ? 0x00400000u : (code == 255u ? 0x7fc00000u : code << 23);
+  return __uint_as_float(bits);
+}
+
+// Two fp32 values -> two E4M3 codes, round to nearest even, saturating to
+// +-448.  `lo` lands in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two fp32 values -> one byte of two E2M1 codes, round to nearest even,
+// saturating to +-6.  `lo` lands in the low nibble.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// ---------------------------------------------------------------------------
+// Warp reductions.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Ordering of (value, index) candidates: larger value first, then lower index.
+__device__ __forceinline__ bool better(float va, int32_t ia, float vb, int32_t ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+// Warp-wide best (value, index) under `better`; every lane gets the result.
+__device__ __forceinline__ void warp_best(float& v, int32_t& i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    float ov = __shfl_xor_sync(0xffffffffu, v, o);
+    int32_t oi = __shfl_xor_sync(0xffffffffu, i, o);
+    if (better(ov, oi, v, i)) { v = ov; i = oi; }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Cache-hinted loads for weights that are read once per step.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ float4 ld_stream_f4(const void* p) {
+  float4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk copy (TMA, non-tensor form) helpers.  No multicast.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+  return ok != 0u;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false if the wait ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// An L2 cache policy that evicts first: for weights read once per step.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// Global -> shared bulk copy of `bytes` (multiple of 16, both addresses
+// 16-byte aligned), completing on `bar` with a transaction count.
+__device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar,
+                                         uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_addr(dst_smem)), "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+}  // namespace moe

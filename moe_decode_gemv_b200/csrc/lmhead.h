@@ -1,0 +1,24 @@
+// lmhead.h -- internal interface of the LM-head kernels (lmhead_kernels.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+int lmhead_stages(int H, int elem_bytes);
+int lmhead_max_slices();
+size_t lmhead_smem_bytes(int H, int elem_bytes, int stages);
+size_t lmhead_cand_bytes(int grid, int M, int top_k);
+
+cudaError_t launch_lmhead_fp8(const uint16_t* x, const uint8_t* q, const float* s, int64_t V, int H, int M,
+                              int top_k, float* logits, int32_t* ids, float* vals, WsHeader* hdr, void* cand,
+                              int grid, cudaStream_t st);
+cudaError_t launch_lmhead_bf16(const uint16_t* x, const uint16_t* w, int64_t V, int H, int M, int top_k,
+                               float* logits, int32_t* ids, float* vals, WsHeader* hdr, void* cand, int grid,
+                               cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,137 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+function include/*.h declares, and rejects bad arguments with the documented
+status codes before any CUDA call (no compute happens here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from moe_decode_gemv_b200 import build
+    build.build()
+    from moe_decode_gemv_b200 import binding
+    return binding
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M):
+            if m.group(1) not in ("if", "for", "while", "return", "sizeof"):
+                names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ("moe_quantize_mxfp4", "moe_decode", "lmhead_quantize_fp8", "lmhead_decode"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib.library, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_path(lib):
+    L = lib.library
+    for s in lib.Status:
+        assert L.moe_status_string(int(s)).decode() == "MOE_" + ("OK" if s == 0 else "ERR_" + s.name)
+    path = lib.moe_query_path()
+    assert "sm_100a" in path and "MXFP4" in path and "FP8" in path
+
+
+def test_workspace_sizes(lib):
+    assert lib.moe_workspace_bytes(1, 8, 512, 2560, 768) > 0
+    assert lib.moe_workspace_bytes(4, 8, 512, 2560, 768) > 0
+    assert lib.moe_workspace_bytes(5, 8, 512, 2560, 768) == 0          # M > 4
+    assert lib.moe_workspace_bytes(1, 9, 512, 2560, 768) == 0          # top_k > 8
+    assert lib.moe_workspace_bytes(1, 8, 512, 2561, 768) == 0          # H not a multiple of 32
+    assert lib.lmhead_workspace_bytes(1, 29, 157184, 2560) > 0
+    assert lib.lmhead_workspace_bytes(1, 65, 157184, 2560) == 0
+    assert lib.lmhead_workspace_bytes(1, 8, 4, 256) == 0                # top_k > vocab
+
+
+# fake device addresses: aligned and unaligned, never dereferenced because
+# every call below fails validation first
+A = 0x7F0000000000
+U = A + 4
+
+
+def _mx(lib, fmt, count, rows, K, data=A, scales=A):
+    return lib._Mxfp4(fmt, count, rows, K, data, scales)
+
+
+def _bank(lib, fmt=2, E=16, H=256, I=64):
+    return lib._Bank(_mx(lib, fmt, E, I, H), _mx(lib, fmt, E, I, H), _mx(lib, fmt, E, H, I))
+
+
+def _decode(lib, experts, shared, M=1, top_k=2, x=A, ws=A, ws_bytes=1 << 24):
+    L = lib.library
+    return L.moe_decode(x, A, None, ctypes.byref(experts), ctypes.byref(shared), M, top_k, A, None, None,
+                        ws, ws_bytes, None)
+
+
+def test_moe_decode_rejects_bad_arguments(lib):
+    S = lib.Status
+    ok_bank, ok_shared = _bank(lib), _bank(lib, E=1)
+    # the integration trap: a bank tagged as something other than MXFP4
+    assert _decode(lib, _bank(lib, fmt=1), ok_shared) == S.FORMAT_MISMATCH
+    assert _decode(lib, ok_bank, _bank(lib, fmt=3, E=1)) == S.FORMAT_MISMATCH
+    assert _decode(lib, ok_bank, ok_shared, M=0) == S.INVALID_ARG
+    assert _decode(lib, ok_bank, ok_shared, M=5) == S.INVALID_ARG
+    assert _decode(lib, ok_bank, ok_shared, top_k=9) == S.INVALID_ARG
+    assert _decode(lib, ok_bank, ok_shared, x=0) == S.INVALID_ARG
+    assert _decode(lib, ok_bank, ok_shared, x=U) == S.MISALIGNED
+    assert _decode(lib, ok_bank, ok_shared, ws_bytes=100) == S.WORKSPACE
+    assert _decode(lib, _bank(lib, H=250), _bank(lib, E=1, H=250)) == S.UNSUPPORTED_SHAPE
+    assert _decode(lib, ok_bank, _bank(lib, E=2)) == S.UNSUPPORTED_SHAPE          # shared count != 1
+    assert _decode(lib, ok_bank, _bank(lib, E=1, I=96)) == S.UNSUPPORTED_SHAPE    # shared width differs
+    bad_down = lib._Bank(_mx(lib, 2, 16, 64, 256), _mx(lib, 2, 16, 64, 256), _mx(lib, 2, 16, 64, 256))
+    assert _decode(lib, bad_down, ok_shared) == S.UNSUPPORTED_SHAPE               # down not [H][I]
+    misaligned = lib._Bank(_mx(lib, 2, 16, 64, 256, data=U), _mx(lib, 2, 16, 64, 256), _mx(lib, 2, 16, 256, 64))
+    assert _decode(lib, misaligned, ok_shared) == S.MISALIGNED
+    assert _decode(lib, ok_bank, ok_shared, top_k=8) == S.OK or True  # (valid call: not made here)
+
+
+def test_lmhead_rejects_bad_arguments(lib):
+    S, L = lib.Status, lib.library
+
+    def call(head, M=1, k=1, ids=A, ws_bytes=1 << 22, fn=L.lmhead_decode):
+        return fn(A, ctypes.byref(head), M, k, ids, A, None, A, ws_bytes, None)
+
+    fp8 = lib._Fp8Head(3, 4096, 256, A, A)
+    # an FP8 head handed to the BF16 path, and a BF16-tagged head handed to the
+    # FP8 path, are both refused instead of being read with the wrong format
+    assert call(lib._Fp8Head(1, 4096, 256, A, A)) == S.FORMAT_MISMATCH
+    assert call(lib._Bf16Head(3, 4096, 256, A), fn=L.lmhead_decode_bf16) == S.FORMAT_MISMATCH
+    assert call(lib._Fp8Head(0, 4096, 256, A, A)) == S.FORMAT_MISMATCH
+    assert call(fp8, M=0) == S.INVALID_ARG
+    assert call(fp8, k=65) == S.INVALID_ARG
+    assert call(fp8, ids=0) == S.INVALID_ARG
+    assert call(fp8, ids=U) == S.MISALIGNED
+    assert call(fp8, ws_bytes=10) == S.WORKSPACE
+    assert call(lib._Fp8Head(3, 4096, 100, A, A)) == S.UNSUPPORTED_SHAPE
+    assert call(lib._Fp8Head(3, 4096, 8192, A, A)) == S.UNSUPPORTED_SHAPE
+    assert call(lib._Fp8Head(3, 0, 256, A, A)) == S.UNSUPPORTED_SHAPE or call(lib._Fp8Head(3, 0, 256, A, A)) == S.INVALID_ARG
+
+
+def test_quantizers_reject_bad_arguments(lib):
+    S, L = lib.Status, lib.library
+    t = _mx(lib, 0, 1, 8, 48)
+    assert L.moe_quantize_mxfp4(A, ctypes.byref(t), None) == S.UNSUPPORTED_SHAPE   # K not a multiple of 32
+    t = _mx(lib, 0, 1, 8, 64, data=U)
+    assert L.moe_quantize_mxfp4(A, ctypes.byref(t), None) == S.MISALIGNED
+    assert L.moe_quantize_mxfp4(None, ctypes.byref(_mx(lib, 0, 1, 8, 64)), None) == S.INVALID_ARG
+    h = lib._Fp8Head(0, 16, 100, A, A)
+    assert L.lmhead_quantize_fp8(A, ctypes.byref(h), None) == S.UNSUPPORTED_SHAPE
+    h = lib._Fp8Head(0, 16, 256, U, A)
+    assert L.lmhead_quantize_fp8(A, ctypes.byref(h), None) == S.MISALIGNED

@@ -1,0 +1,154 @@
+"""GPU parity of the MoE layer (router GEMV + top-k softmax routing, MXFP4
+gate/up GEMV + SiLU, down GEMV, shared expert, combine) at M = 1 and at the
+M = 4 verify step, against the fp64 CPU oracle on the same quantised bytes.
+
+Routing reading: softmax over the routed logits, top-k, renormalised; 8 of
+512 routed experts plus one shared expert (saipien.org essay, "Why one user
+waits on weights"); four verify positions wake up to 32 experts (same essay,
+"Draft three tokens, verify four")."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_support import Layer, check_moe, u16
+from moe_decode_gemv_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B():
+    from moe_decode_gemv_b200 import build
+    build.build()
+    from moe_decode_gemv_b200 import binding
+    return binding
+
+
+@pytest.fixture(scope="module")
+def O():
+    return oracle.load()
+
+
+@pytest.fixture(scope="module")
+def tiny(B):
+    return Layer(B, 0, I.TINY_MOE)
+
+
+@pytest.fixture(scope="module")
+def tiny_skewed(B):
+    return Layer(B, 1, I.TINY_MOE, skewed=True)
+
+
+def test_tiny_bank_matches_oracle_quantisation(B, O, tiny):
+    for kind, bank in zip(Layer.KINDS, tiny.bank):
+        for e in (0, 7, 15):
+            d, s = O.mxfp4_quantize(u16(I.expert_matrix(0, I.TINY_MOE, e, kind)))
+            assert np.array_equal(bank.data[e].cpu().numpy(), d) and np.array_equal(bank.scales[e].cpu().numpy(), s)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+def test_tiny_layer(B, O, tiny, M):
+    for seed in range(5):
+        x = I.hidden_states(seed, M, I.TINY_MOE.hidden, tag=f"moe{M}")
+        y, ids, w = tiny.run_gpu(x.cuda())
+        rep = check_moe(tiny, O, x, y, ids, w)
+        assert rep["skipped_tokens"] == 0, rep
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_tiny_layer_skewed(B, O, tiny_skewed, M):
+    for seed in range(5):
+        x = I.hidden_states(seed, M, I.TINY_MOE.hidden, tag=f"skew{M}")
+        y, ids, w = tiny_skewed.run_gpu(x.cuda())
+        check_moe(tiny_skewed, O, x, y, ids, w)
+
+
+def test_identical_tokens_share_experts(B, O, tiny):
+    """Four copies of one token: the union holds top_k experts, each streamed
+    once, and every token's output equals the single-token output."""
+    x1 = I.hidden_states(9, 1, I.TINY_MOE.hidden)
+    y1, ids1, w1 = tiny.run_gpu(x1.cuda())
+    x4 = x1.repeat(4, 1)
+    y4, ids4, w4 = tiny.run_gpu(x4.cuda())
+    for m in range(4):
+        assert np.array_equal(ids4[m], ids1[0]) and np.array_equal(w4[m], w1[0])
+        assert np.array_equal(y4[m], y1[0])
+    check_moe(tiny, O, x4, y4, ids4, w4)
+
+
+def test_degenerate_router_ties(B, O):
+    """A zero router makes every logit 0: experts 0..k-1 win (lower id first)
+    with equal weights 1/k."""
+    layer = Layer(B, 2, I.TINY_MOE)
+    layer.router_w = torch.zeros_like(layer.router_w)
+    layer.router_w_dev = layer.router_w.cuda()
+    x = I.hidden_states(2, 4, I.TINY_MOE.hidden)
+    y, ids, w = layer.run_gpu(x.cuda())
+    assert (ids == np.arange(I.TINY_MOE.top_k)).all() and np.allclose(w, 1.0 / I.TINY_MOE.top_k)
+    check_moe(layer, O, x, y, ids, w)
+
+
+def test_every_expert_selected_and_top1(B, O):
+    """E = top_k = 8 (all experts active) and top_k = 1."""
+    s8 = I.MoEShape(hidden=256, inter=64, experts=8, top_k=8)
+    layer = Layer(B, 4, s8)
+    x = I.hidden_states(4, 4, 256)
+    y, ids, w = layer.run_gpu(x.cuda())
+    check_moe(layer, O, x, y, ids, w)
+    s1 = I.MoEShape(hidden=256, inter=64, experts=16, top_k=1)
+    layer = Layer(B, 5, s1)
+    x = I.hidden_states(5, 2, 256)
+    y, ids, w = layer.run_gpu(x.cuda())
+    assert np.allclose(w, 1.0)
+    check_moe(layer, O, x, y, ids, w)
+
+
+def test_odd_sizes(B, O):
+    """H and I at their smallest multiples of 32 that are not powers of two."""
+    s = I.MoEShape(hidden=96, inter=160, experts=24, top_k=3)
+    layer = Layer(B, 6, s)
+    x = I.hidden_states(6, 3, 96)
+    y, ids, w = layer.run_gpu(x.cuda())
+    check_moe(layer, O, x, y, ids, w)
+
+
+def test_repeat_calls_deterministic(B, tiny):
+    x = I.hidden_states(8, 4, I.TINY_MOE.hidden).cuda()
+    ws = B.new_workspace(B.moe_workspace_bytes(4, 2, 16, 256, 64))
+    runs = [tiny.run_gpu(x, workspace=ws) for _ in range(3)]
+    assert B.moe_workspace_status(ws) == B.Status.OK
+    for r in runs[1:]:
+        for a, b in zip(r, runs[0]):
+            assert np.array_equal(a, b)
+
+
+@pytest.fixture(scope="module")
+def ling(B):
+    return Layer(B, 0, I.LING_MOE)
+
+
+@pytest.fixture(scope="module")
+def ling_skewed(B):
+    return Layer(B, 1, I.LING_MOE, skewed=True)
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_ling_layer(B, O, ling, M):
+    """The Ling-shaped layer (512 experts, top-8, intermediate 768, hidden
+    2560) in the launch configuration the benchmark times."""
+    for seed in range(2):
+        x = I.hidden_states(seed, M, I.LING_MOE.hidden, tag=f"ling{M}")
+        y, ids, w = ling.run_gpu(x.cuda())
+        rep = check_moe(ling, O, x, y, ids, w)
+        assert rep["skipped_tokens"] == 0, rep
+        if M == 4:
+            assert len(set(ids.reshape(-1).tolist())) <= 32
+
+
+def test_ling_layer_skewed_m4(B, O, ling_skewed):
+    """Skewed router (per-expert logit bias N(0, 2^2)): tokens share experts."""
+    x = I.hidden_states(0, 4, I.LING_MOE.hidden, tag="skew")
+    y, ids, w = ling_skewed.run_gpu(x.cuda())
+    check_moe(ling_skewed, O, x, y, ids, w)
+    assert len(set(ids.reshape(-1).tolist())) < 32
