@@ -161,8 +161,9 @@ MOE_API size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts
  *   topk_w      [M][top_k] fp32 or NULL:  renormalised softmax weights
  *   workspace   device buffer of at least moe_workspace_bytes(...) bytes,
  *               zeroed once (moe_workspace_reset) before its first use.
- * Supported: H and I multiples of 32 and at most 8192, E <= 1024,
- * 1 <= top_k <= 8 and top_k <= E.  Each distinct routed expert is streamed once per call, however
+ * Supported: H and I multiples of 64, H <= 4096, I <= 1024, E <= 1024,
+ * 1 <= top_k <= 8 and top_k <= E.  The call is one cooperative launch
+ * (one CTA per SM, all resident).  Each distinct routed expert is streamed once per call, however
  * many of the M tokens chose it.                                             */
 MOE_API moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const float* router_bias,
                       const moe_expert_bank* experts, const moe_expert_bank* shared,
@@ -189,6 +190,22 @@ MOE_API moe_status lmhead_decode(const uint16_t* hidden_bf16, const moe_fp8_head
 MOE_API moe_status lmhead_decode_bf16(const uint16_t* hidden_bf16, const moe_bf16_head* head,
                               int32_t M, int32_t top_k, int32_t* topk_ids, float* topk_vals,
                               float* logits, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- between the layers of a decode step ---------------------------------- */
+
+/* The next layer's input from a layer's output, for a stack of MoE layers
+ * each re-routed from the previous layer's RMS-normalised output (the decode
+ * stream of the workload): out[m][j] = bf16_RNE(y[m][j] / sqrt(mean_j y[m][j]^2
+ * + eps)), gain 1.  y [M][H] fp32, out [M][H] bf16; H a multiple of 8.       */
+MOE_API moe_status moe_rmsnorm_bf16(const float* y, int32_t M, int32_t H, float eps, uint16_t* out,
+                                    void* stream);
+
+/* Greedy feedback: out[m] = table[ids[m * ids_stride]] for the next step
+ * (table [V][H] bf16; ids device int32, e.g. the column 0 of lmhead_decode's
+ * topk_ids with ids_stride = top_k).  An id outside [0, V) gives a zero row.
+ * H a multiple of 8.                                                         */
+MOE_API moe_status moe_embed_gather(const uint16_t* table, int64_t V, int64_t H, const int32_t* ids,
+                                    int32_t ids_stride, int32_t M, uint16_t* out, void* stream);
 
 /* ---- housekeeping --------------------------------------------------------- */
 

@@ -77,6 +77,8 @@ def _load() -> ctypes.CDLL:
         "lmhead_workspace_bytes": ([I32, I32, I64, I64], SZ),
         "lmhead_decode": ([P, ctypes.POINTER(_Fp8Head), I32, I32, P, P, P, P, SZ, P], I32),
         "lmhead_decode_bf16": ([P, ctypes.POINTER(_Bf16Head), I32, I32, P, P, P, P, SZ, P], I32),
+        "moe_rmsnorm_bf16": ([P, I32, I32, ctypes.c_float, P, P], I32),
+        "moe_embed_gather": ([P, I64, I64, P, I32, I32, P, P], I32),
         "moe_workspace_reset": ([P, SZ, P], I32),
         "moe_workspace_status": ([P, P], I32),
         "moe_query_path": ([ctypes.c_char_p, SZ], I32),
@@ -246,6 +248,22 @@ def lmhead_decode_bf16(hidden: torch.Tensor, w_bf16: torch.Tensor, top_k: int, t
                                     _ptr(logits), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "lmhead_decode_bf16")
     return topk_ids, topk_vals
+
+
+def moe_rmsnorm_bf16(y: torch.Tensor, out: torch.Tensor, eps: float = 1e-6, stream=None) -> torch.Tensor:
+    """bf16 [M, H] = RMSNorm (gain 1) of fp32 [M, H]: the next layer's input."""
+    M, H = y.shape
+    _check(library.moe_rmsnorm_bf16(_ptr(y), M, H, float(eps), _ptr(out), _stream(stream)), "moe_rmsnorm_bf16")
+    return out
+
+
+def moe_embed_gather(table: torch.Tensor, ids: torch.Tensor, out: torch.Tensor, ids_stride: int = 1,
+                     stream=None) -> torch.Tensor:
+    """out[m] = table[ids[m * ids_stride]] (bf16 rows)."""
+    V, H = table.shape
+    st = library.moe_embed_gather(_ptr(table), V, H, _ptr(ids), ids_stride, out.shape[0], _ptr(out), _stream(stream))
+    _check(st, "moe_embed_gather")
+    return out
 
 
 def moe_workspace_status(workspace: torch.Tensor, stream=None) -> Status:

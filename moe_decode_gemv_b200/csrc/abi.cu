@@ -13,6 +13,7 @@
 #include "lmhead.h"
 #include "moe.h"
 #include "quantize.h"
+#include "stack.h"
 
 namespace {
 
@@ -109,7 +110,7 @@ moe_status lmhead_quantize_fp8(const uint16_t* w_bf16, moe_fp8_head* out, void* 
 
 size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts, int32_t hidden, int32_t inter) {
   if (M < 1 || M > 4 || top_k < 1 || top_k > 8 || num_experts < 1 || num_experts > 1024) return 0;
-  if (hidden < 32 || hidden % 32 != 0 || hidden > 8192 || inter < 32 || inter % 32 != 0 || inter > 8192) return 0;
+  if (hidden < 64 || inter < 64 || !moe::moe_fused_supported(hidden, inter)) return 0;
   return moe::moe_ws_bytes(M, top_k, num_experts, hidden, inter);
 }
 
@@ -125,7 +126,7 @@ moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const 
     if (t->fmt != MOE_FMT_MXFP4_E2M1_E8M0_32) return MOE_ERR_FORMAT_MISMATCH;
   const int64_t E = experts->gate.count, H = experts->gate.K, I = experts->gate.rows;
   if (E < 1 || E > 1024 || top_k > E) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (H < 32 || H % 32 != 0 || H > 8192 || I < 32 || I % 32 != 0 || I > 8192) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (H < 64 || I < 64 || !moe::moe_fused_supported((int)H, (int)I)) return MOE_ERR_UNSUPPORTED_SHAPE;
   moe_status s;
   if ((s = check_bank(experts, E, H, I)) != MOE_OK) return s;
   if ((s = check_bank(shared, 1, H, I)) != MOE_OK) return s;
@@ -144,7 +145,7 @@ moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const 
   a.M = M; a.top_k = top_k; a.E = (int)E; a.H = (int)H; a.I = (int)I;
   a.out = out; a.ids_out = topk_ids; a.w_out = topk_w;
   a.ws = moe::MoeWs::carve(workspace, (int)E, (int)H, (int)I);
-  return cuda_status(moe::launch_moe(a, static_cast<cudaStream_t>(stream)));
+  return cuda_status(moe::launch_moe_fused(a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t lmhead_workspace_bytes(int32_t M, int32_t top_k, int64_t vocab, int64_t hidden) {
@@ -173,6 +174,20 @@ moe_status lmhead_decode_bf16(const uint16_t* hidden_bf16, const moe_bf16_head* 
                             topk_vals, logits, workspace, workspace_bytes, stream);
 }
 
+moe_status moe_rmsnorm_bf16(const float* y, int32_t M, int32_t H, float eps, uint16_t* out, void* stream) {
+  if (!y || !out || M < 1 || H < 8 || H % 8 != 0 || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(out)) return MOE_ERR_MISALIGNED;
+  return cuda_status(moe::launch_rmsnorm_bf16(y, M, H, eps, out, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_embed_gather(const uint16_t* table, int64_t V, int64_t H, const int32_t* ids, int32_t ids_stride,
+                            int32_t M, uint16_t* out, void* stream) {
+  if (!table || !ids || !out || V < 1 || H < 8 || H % 8 != 0 || M < 1 || ids_stride < 1) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(table) || !aligned16(out) || (reinterpret_cast<uintptr_t>(ids) & 3u)) return MOE_ERR_MISALIGNED;
+  return cuda_status(moe::launch_embed_gather(table, V, (int)H, ids, ids_stride, M, out,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_workspace_reset(void* workspace, size_t workspace_bytes, void* stream) {
   if (!workspace || workspace_bytes < sizeof(moe::WsHeader)) return MOE_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)));
@@ -194,9 +209,9 @@ moe_status moe_workspace_status(void* workspace, void* stream) {
 moe_status moe_query_path(char* buf, size_t n) {
   if (!buf || n == 0) return MOE_ERR_INVALID_ARG;
   const char* desc =
-      "sm_100a; moe: router fp32 GEMV + warp top-k, MXFP4 (E2M1/E8M0-32) gate/up GEMV + SiLU, down GEMV, "
-      "ordered combine; lm-head: FP8 E4M3 per-row-scale GEMV (bulk-copy ring, mma.sync f16) fused top-k; "
-      "comparator: BF16 head GEMV";
+      "sm_100a; moe: one persistent kernel (router fp32 GEMV + top-k, MXFP4 E2M1/E8M0-32 gate/up + SiLU, "
+      "down, ordered combine; bulk-copy ring, mma.sync f16); lm-head: FP8 E4M3 per-row-scale GEMV "
+      "(bulk-copy ring, mma.sync f16) fused top-k; comparator: BF16 head GEMV";
   std::snprintf(buf, n, "%s", desc);
   return std::strlen(desc) < n ? MOE_OK : MOE_ERR_INVALID_ARG;
 }

@@ -31,10 +31,29 @@ __device__ __forceinline__ void report(WsHeader* h, moe_status s) {
   atomicCAS(&h->status, 0, (int32_t)s);
 }
 
-// Upper bound on polls of any device-side wait before a kernel gives up,
-// records MOE_ERR_TIMEOUT and returns.  A poll takes tens of nanoseconds, so
-// this is seconds of waiting -- orders of magnitude above any healthy wait.
-constexpr uint32_t kSpinLimit = 1u << 26;
+// Every device-side wait in this library is bounded in time: after
+// kWaitLimitNs of waiting a kernel records MOE_ERR_TIMEOUT and returns instead
+// of hanging.  A healthy wait here lasts microseconds.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Polls `ready()` until it returns true or kWaitLimitNs have passed, sleeping
+// `backoff_ns` between polls so that a waiting warp leaves the issue slots to
+// the warps doing the work.  Returns false on timeout.
+template <typename F>
+__device__ __forceinline__ bool bounded_spin(F ready, uint32_t backoff_ns = 64) {
+  const uint64_t start = global_ns();
+  for (;;) {
+    if (ready()) return true;
+    if (global_ns() - start > kWaitLimitNs) return false;
+    if (backoff_ns) __nanosleep(backoff_ns);
+  }
+}
 
 // ---------------------------------------------------------------------------
 // Format conversions.
@@ -114,16 +133,18 @@ __device__ __forceinline__ void warp_best(float& v, int32_t& i) {
 // ---------------------------------------------------------------------------
 // Cache-hinted loads for weights that are read once per step.
 // ---------------------------------------------------------------------------
+// (not volatile: the compiler may batch and reorder these reads of data that
+// no kernel writes while they are in flight)
 __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
   uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
 
 __device__ __forceinline__ float4 ld_stream_f4(const void* p) {
   float4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+  asm("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
                : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
   return r;
 }
@@ -152,19 +173,19 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended (up to the hint, here 0.1 ms) instead of spinning.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(100000u) : "memory");
   return ok != 0u;
 }
 
 // Bounded wait on an mbarrier phase.  Returns false if the wait ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+  return bounded_spin([&] { return mbar_try_wait(bar, parity); }, 0);
 }
 
 // An L2 cache policy that evicts first: for weights read once per step.

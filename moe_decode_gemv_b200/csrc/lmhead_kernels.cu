@@ -14,17 +14,18 @@
 //    mbarriers; rows are copied one by one into a padded stride so that the
 //    consumers' 16-byte shared loads are free of bank conflicts.
 //  * Eight consumer warps split K.  Each computes 16 rows x 8 token columns
-//    with mma.sync m16n8k16 (f16 x f16 -> fp32): the A fragments are built in
-//    registers straight from the E4M3 bytes (one cvt per pair; every E4M3
-//    value is an f16 value, so this is exact) and the B fragments hold the
-//    token activations, resident in registers for the whole kernel.  This is
-//    a GEMV: the tensor-core instruction is used because it retires 2,048
-//    multiply-adds per issue, which keeps the instruction count per weight
-//    byte far below what the HBM stream allows at M = 4.
-//  * bf16 activations become f16 exactly after a per-token power-of-two
-//    scale 2^sigma_m that puts max|x_m| in [2^14, 2^15); the logit is
-//    acc * s_v * 2^-sigma_m.  Only elements more than 2^28 below the token's
-//    largest fall into the f16 subnormal range.
+//    with mma.sync m16n8k32 (E4M3 x E4M3 -> fp32): the weight bytes from
+//    shared memory ARE the A fragments -- no conversion instruction per
+//    weight -- and the B fragments hold the token activations, resident in
+//    registers for the whole kernel.  This is a GEMV: the tensor-core
+//    instruction is used because it retires 4,096 multiply-adds per issue and
+//    needs no per-weight decode, which keeps the instruction count per weight
+//    byte far below what the HBM stream allows, at M = 1 and M = 4 alike.
+//  * Activations: each bf16 token is scaled by 2^sigma_m (max |x| into
+//    [2^7, 2^8)) and split into two E4M3 parts hi + lo, which represent the
+//    bf16 value exactly (8 significand bits = 4 + 4) for every element above
+//    E4M3's subnormal range; the two parts take two MMAs.  The logit is
+//    acc * s_v * 2^-sigma_m.
 //  * Epilogue per tile: the consumers' partial sums meet in shared memory;
 //    one warp per token applies the row scale, writes logits when asked and
 //    merges the 16 candidates into the CTA's running top-k list (sorted, ties
@@ -41,14 +42,15 @@ namespace {
 
 constexpr int kTileRows = 16;
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kThreads = (kConsumerWarps + 2) * 32;  // consumers + producer + epilogue
 constexpr int kMaxSlicesPerWarp = 10;  // row bytes <= 10 * 8 * 64 = 5120: H <= 5120 (fp8), 2560 (bf16)
 constexpr size_t kMaxSmem = 232448;    // 227 KB of dynamic shared memory per CTA
 
 template <typename W>
 struct HeadTraits;
 
-// FP8 E4M3 weights: a 64-byte K slice is 64 elements; 4 MMAs of k16 each.
+// FP8 E4M3 weights: a 64-byte K slice is 64 elements = 2 MMAs of k32, each
+// run twice (hi and lo parts of the activations): 4 MMAs per slice.
 template <>
 struct HeadTraits<uint8_t> {
   static constexpr int kElemBytes = 1;
@@ -67,6 +69,15 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -89,6 +100,49 @@ struct Cand {
   int32_t id;
 };
 
+constexpr int kCandBuf = 128;     // per-token candidate buffer of the epilogue warp
+constexpr int kSurvivors = 2048;  // entries kept by the final merge's lower bound
+
+// Warp-cooperative: move the best min(k, n) of buf[0..n) to buf[0..) in order
+// (value descending, ties to the lower id), padding with empty candidates up
+// to k.  Returns min(k, n).  Selection by repeated warp argmax: O(n k / 32).
+__device__ int select_top(Cand* buf, int n, int k, int lane) {
+  constexpr int kPer = kCandBuf / 32;
+  Cand c[kPer];
+  bool taken[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int j = lane + 32 * i;
+    c[i] = j < n ? buf[j] : Cand{-FLT_MAX, INT32_MAX};
+    taken[i] = j >= n;
+  }
+  __syncwarp();
+  const int keep = n < k ? n : k;
+  for (int r = 0; r < k; ++r) {
+    float bv = -FLT_MAX;
+    int32_t bi = INT32_MAX;
+    int bslot = -1;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      if (!taken[i] && (bslot < 0 || better(c[i].v, c[i].id, bv, bi))) { bv = c[i].v; bi = c[i].id; bslot = i; }
+    float wv = bv;
+    int32_t wi = bi;
+    warp_best(wv, wi);
+    // the owner of the winner marks it taken (ids are unique among real candidates)
+    if (r < keep && bslot >= 0 && bi == wi && bv == wv) taken[bslot] = true;
+    if (lane == 0) buf[r] = r < keep ? Cand{wv, wi} : Cand{-FLT_MAX, INT32_MAX};
+  }
+  __syncwarp();
+  return keep;
+}
+
+// Warp roles: warp 0..7 consumers (K split), warp 8 producer (bulk copies),
+// warp 9 epilogue (cross-warp sum, row scale, logits, top-k).  Consumers hand
+// each tile's partial sums to the epilogue warp through kRed buffers guarded
+// by mbarriers, so no CTA-wide barrier sits in the streaming loop.
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kRed = 4;
+
 template <typename W, int kSlices>
 __global__ void __launch_bounds__(kThreads, 1)
 lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
@@ -107,13 +161,16 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
   const int stride = padded_stride(row_bytes);
   const int tile_bytes = kTileRows * stride;
 
-  // shared-memory carve-up: [ring][reduce 2x][top-k lists][barriers]
+  // shared-memory carve-up: [ring][reduce buffers][top-k lists][barriers][scalars]
   uint8_t* ring = smem;
-  float* red = reinterpret_cast<float*>(ring + (size_t)stages * tile_bytes);      // [2][W][16][4]
-  Cand* lists = reinterpret_cast<Cand*>(red + 2 * kConsumerWarps * kTileRows * 4);  // [M][top_k]
-  uint64_t* full = reinterpret_cast<uint64_t*>(lists + 4 * 64);
+  float* red = reinterpret_cast<float*>(ring + (size_t)stages * tile_bytes);       // [kRed][8][16][4]
+  Cand* lists = reinterpret_cast<Cand*>(red + kRed * kConsumerWarps * kTileRows * 4);  // [M][top_k]
+  Cand* cbuf = lists + 4 * 64;                                                       // [M][kCandBuf]
+  uint64_t* full = reinterpret_cast<uint64_t*>(cbuf + 4 * kCandBuf);
   uint64_t* empty = full + stages;
-  int* s_sigma = reinterpret_cast<int*>(empty + stages);  // [4]
+  uint64_t* red_full = empty + stages;
+  uint64_t* red_empty = red_full + kRed;
+  int* s_sigma = reinterpret_cast<int*>(red_empty + kRed);  // [4]
   int* s_poison = s_sigma + 4;  // set once any bounded wait ran out
   int* s_last = s_sigma + 5;
 
@@ -126,6 +183,10 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
+    }
+    for (int r = 0; r < kRed; ++r) {
+      mbar_init(&red_full[r], kConsumerWarps);
+      mbar_init(&red_empty[r], 1);
     }
     fence_mbar_init();
     *s_poison = 0;
@@ -140,7 +201,7 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
       if (sizeof(W) == 1 && amax > 0.f) {
         int e = (int)((__float_as_uint(amax) >> 23) & 0xff);
         int fl = e ? e - 127 : (31 - __clz(__float_as_uint(amax) & 0x7fffff)) - 149;
-        sigma = 14 - fl;
+        sigma = 7 - fl;  // max |x * 2^sigma| in [2^7, 2^8): inside E4M3's normal range
         sigma = sigma > 126 ? 126 : (sigma < -126 ? -126 : sigma);
       }
       s_sigma[warp] = sigma;
@@ -149,39 +210,50 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
   for (int i = threadIdx.x; i < M * top_k; i += blockDim.x) lists[i] = Cand{-FLT_MAX, INT32_MAX};
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
+  // bounded wait shared by all roles: lane 0 polls, the warp agrees on the result
+  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+    bool ok = !*(volatile int*)s_poison;
+    if (ok && lane == 0) ok = mbar_wait(bar, parity);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok && lane == 0 && !*(volatile int*)s_poison) {
+      report(hdr, MOE_ERR_TIMEOUT);
+      atomicExch(s_poison, 1);
+    }
+    return ok;
+  };
+
+  if (warp == kProducerWarp) {
     // ------------------------------ producer ------------------------------
     const uint64_t policy = l2_evict_first_policy();
     int64_t it = 0, issued = 0;
     for (int64_t t = t_begin; t < t_end; ++t, ++it) {
       const int s = (int)(it % stages);
       const uint32_t ph = (uint32_t)((it / stages) & 1);
-      bool ok = !*(volatile int*)s_poison;
-      if (ok && it >= stages && lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        // after a timeout nothing more is issued; the consumers run on without waiting
-        if (lane == 0 && !*(volatile int*)s_poison) { report(hdr, MOE_ERR_TIMEOUT); atomicExch(s_poison, 1); }
-        continue;
-      }
+      if (it >= stages && !wait_all(&empty[s], ph ^ 1u)) continue;  // after a timeout: issue nothing more
+      if (*(volatile int*)s_poison) continue;
       const int64_t r0 = t * kTileRows;
       const int nrows = (int)(V - r0 < kTileRows ? V - r0 : kTileRows);
       if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(nrows * row_bytes));
       __syncwarp();
       if (lane < nrows)
         bulk_g2s(ring + (size_t)s * tile_bytes + (size_t)lane * stride,
-                 reinterpret_cast<const uint8_t*>(w) + (size_t)(r0 + lane) * row_bytes, (uint32_t)row_bytes, &full[s], policy);
+                 reinterpret_cast<const uint8_t*>(w) + (size_t)(r0 + lane) * row_bytes, (uint32_t)row_bytes,
+                 &full[s], policy);
       issued = it + 1;
     }
-    // drain: every issued copy must land before this CTA may exit
+    // every issued copy must land before this CTA may exit
     if (lane == 0) {
       const int64_t first = issued > stages ? issued - stages : 0;
       for (int64_t j = first; j < issued; ++j) mbar_wait(&full[j % stages], (uint32_t)((j / stages) & 1));
     }
-  } else {
+  } else if (warp < kConsumerWarps) {
     // ------------------------------ consumers -----------------------------
     const int g = lane >> 2, tq = lane & 3;
-    // B fragments: token n = g, this warp's K slices
+    // B fragments: token n = g, this warp's K slices, resident for the whole kernel.
+    // FP8 head: the token, scaled by 2^sigma, is split into two E4M3 parts,
+    // x' = hi + lo, exact for every element whose magnitude is above E4M3's
+    // subnormal range (more than 2^-14 of the token's largest).  Each part
+    // takes its own MMA; the weights enter the MMA as raw E4M3 bytes.
     uint32_t bfrag[kSlices][T::kMmasPerSlice][2];
     {
       const bool live = g < M;
@@ -189,23 +261,35 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
 #pragma unroll
       for (int si = 0; si < kSlices; ++si) {
         const int slice = warp + si * kConsumerWarps;
-        const int e0 = slice * (64 / T::kElemBytes) + tq * (16 / T::kElemBytes);  // first element of the lane chunk
+        const bool in = live && slice * 64 < row_bytes;
+        if constexpr (sizeof(W) == 1) {
+          const int e0 = slice * 64 + tq * 16;
 #pragma unroll
-        for (int j = 0; j < T::kMmasPerSlice; ++j) {
-#pragma unroll
-          for (int p = 0; p < 2; ++p) {
-            const int k0 = e0 + 4 * j + 2 * p;
-            uint32_t v = 0u;
-            if (live && slice * 64 < row_bytes) {
-              const uint32_t pair = *reinterpret_cast<const uint32_t*>(x + (size_t)g * H + k0);
-              if constexpr (sizeof(W) == 1) {
-                __half2 h2 = __floats2half2_rn(bf16_bits_to_f32(pair & 0xffffu) * scl, bf16_bits_to_f32(pair >> 16) * scl);
-                v = *reinterpret_cast<uint32_t*>(&h2);
-              } else {
-                v = pair;  // bf16 pair as is
-              }
+          for (int q = 0; q < 4; ++q) {  // four groups of 4 elements: mma (q / 2), register (q % 2)
+            uint32_t hw = 0u, lw = 0u;
+            if (in) {
+              const uint2 p = *reinterpret_cast<const uint2*>(x + (size_t)g * H + e0 + 4 * q);
+              const float v0 = bf16_bits_to_f32(p.x & 0xffffu) * scl, v1 = bf16_bits_to_f32(p.x >> 16) * scl;
+              const float v2 = bf16_bits_to_f32(p.y & 0xffffu) * scl, v3 = bf16_bits_to_f32(p.y >> 16) * scl;
+              const uint32_t h01 = f32x2_to_e4m3x2(v0, v1), h23 = f32x2_to_e4m3x2(v2, v3);
+              const uint32_t f01 = e4m3x2_to_f16x2(h01), f23 = e4m3x2_to_f16x2(h23);
+              const float2 r01 = __half22float2(*reinterpret_cast<const __half2*>(&f01));
+              const float2 r23 = __half22float2(*reinterpret_cast<const __half2*>(&f23));
+              hw = h01 | (h23 << 16);
+              lw = f32x2_to_e4m3x2(v0 - r01.x, v1 - r01.y) | (f32x2_to_e4m3x2(v2 - r23.x, v3 - r23.y) << 16);
             }
-            bfrag[si][j][p] = v;
+            bfrag[si][2 * (q / 2)][q % 2] = hw;      // j = 0 (mma 0, hi), 2 (mma 1, hi)
+            bfrag[si][2 * (q / 2) + 1][q % 2] = lw;  // j = 1 (mma 0, lo), 3 (mma 1, lo)
+          }
+        } else {
+          const int e0 = slice * 32 + tq * 8;
+#pragma unroll
+          for (int j = 0; j < T::kMmasPerSlice; ++j) {
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+              const int k0 = e0 + 4 * j + 2 * p;
+              bfrag[si][j][p] = in ? *reinterpret_cast<const uint32_t*>(x + (size_t)g * H + k0) : 0u;
+            }
           }
         }
       }
@@ -214,97 +298,116 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
     int64_t it = 0;
     for (int64_t t = t_begin; t < t_end; ++t, ++it) {
       const int s = (int)(it % stages);
-      const uint32_t ph = (uint32_t)((it / stages) & 1);
-      bool ok = !*(volatile int*)s_poison;
-      if (ok && lane == 0) ok = mbar_wait(&full[s], ph);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok && lane == 0 && !*(volatile int*)s_poison) { report(hdr, MOE_ERR_TIMEOUT); atomicExch(s_poison, 1); }
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      const bool ok = wait_all(&full[s], (uint32_t)((it / stages) & 1));
+      // one accumulator per MMA index: four independent chains instead of one
+      float acc[T::kMmasPerSlice][4];
+#pragma unroll
+      for (int j = 0; j < T::kMmasPerSlice; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
       if (ok) {
         const uint8_t* tile = ring + (size_t)s * tile_bytes;
+        uint4 ra[kSlices], rb[kSlices];
+#pragma unroll
+        for (int si = 0; si < kSlices; ++si) {  // all shared loads of the tile first
+          const int slice = warp + si * kConsumerWarps;
+          if (slice * 64 < row_bytes) {
+            ra[si] = *reinterpret_cast<const uint4*>(tile + (size_t)g * stride + slice * 64 + tq * 16);
+            rb[si] = *reinterpret_cast<const uint4*>(tile + (size_t)(g + 8) * stride + slice * 64 + tq * 16);
+          }
+        }
 #pragma unroll
         for (int si = 0; si < kSlices; ++si) {
           const int slice = warp + si * kConsumerWarps;
           if (slice * 64 < row_bytes) {
-            const uint4 ra = *reinterpret_cast<const uint4*>(tile + (size_t)g * stride + slice * 64 + tq * 16);
-            const uint4 rb = *reinterpret_cast<const uint4*>(tile + (size_t)(g + 8) * stride + slice * 64 + tq * 16);
-            const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w}, wb[4] = {rb.x, rb.y, rb.z, rb.w};
+            const uint32_t wa[4] = {ra[si].x, ra[si].y, ra[si].z, ra[si].w};
+            const uint32_t wb[4] = {rb[si].x, rb[si].y, rb[si].z, rb[si].w};
             if constexpr (sizeof(W) == 1) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint32_t a[4] = {e4m3x2_to_f16x2(wa[j] & 0xffffu), e4m3x2_to_f16x2(wb[j] & 0xffffu),
-                                       e4m3x2_to_f16x2(wa[j] >> 16), e4m3x2_to_f16x2(wb[j] >> 16)};
-                mma_f16(d, a, bfrag[si][j][0], bfrag[si][j][1]);
-              }
+              // rows g and g+8, 16 bytes each: words 0,1 feed MMA 0 and words 2,3 MMA 1
+              mma_e4m3(acc[0], wa[0], wb[0], wa[1], wb[1], bfrag[si][0][0], bfrag[si][0][1]);
+              mma_e4m3(acc[1], wa[0], wb[0], wa[1], wb[1], bfrag[si][1][0], bfrag[si][1][1]);
+              mma_e4m3(acc[2], wa[2], wb[2], wa[3], wb[3], bfrag[si][2][0], bfrag[si][2][1]);
+              mma_e4m3(acc[3], wa[2], wb[2], wa[3], wb[3], bfrag[si][3][0], bfrag[si][3][1]);
             } else {
 #pragma unroll
               for (int j = 0; j < 2; ++j) {
                 const uint32_t a[4] = {wa[2 * j], wb[2 * j], wa[2 * j + 1], wb[2 * j + 1]};
-                mma_bf16(d, a, bfrag[si][j][0], bfrag[si][j][1]);
+                mma_bf16(acc[j], a, bfrag[si][j][0], bfrag[si][j][1]);
               }
             }
           }
         }
       }
+      float d[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        d[q] = acc[0][q];
+#pragma unroll
+        for (int j = 1; j < T::kMmasPerSlice; ++j) d[q] += acc[j][q];
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
 
-      // partial sums -> shared; tokens 2tq and 2tq+1 live in lanes with tq < 2
-      float* rb = red + (size_t)(it & 1) * kConsumerWarps * kTileRows * 4;
-      if (tq < 2) {
+      // hand the partial sums to the epilogue warp
+      const int r = (int)(it % kRed);
+      if (it >= kRed) wait_all(&red_empty[r], (uint32_t)(((it / kRed) & 1) ^ 1));
+      float* rb = red + (size_t)r * kConsumerWarps * kTileRows * 4;
+      if (tq < 2) {  // tokens 2tq, 2tq+1 (M <= 4)
         rb[(warp * kTileRows + g) * 4 + 2 * tq] = d[0];
         rb[(warp * kTileRows + g) * 4 + 2 * tq + 1] = d[1];
         rb[(warp * kTileRows + g + 8) * 4 + 2 * tq] = d[2];
         rb[(warp * kTileRows + g + 8) * 4 + 2 * tq + 1] = d[3];
       }
-      asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32));
-
-      if (warp < M) {
-        // one warp per token: lanes 0..15 own one row of the tile each
-        const int m = warp;
-        const int64_t row = t * kTileRows + lane;
-        const bool valid = lane < kTileRows && row < V;
-        float v = -FLT_MAX;
-        if (valid) {
-          float acc = 0.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&red_full[r]);
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    int cnt[4] = {0, 0, 0, 0};
+    Cand thr[4] = {{-FLT_MAX, INT32_MAX}, {-FLT_MAX, INT32_MAX}, {-FLT_MAX, INT32_MAX}, {-FLT_MAX, INT32_MAX}};
+    // Per token: a buffer of candidates better than the current threshold (the
+    // k-th best kept so far).  Appends are one ballot; when the buffer could
+    // overflow, a selection pass keeps the best k and raises the threshold.
+    int64_t it = 0;
+    for (int64_t t = t_begin; t < t_end; ++t, ++it) {
+      const int r = (int)(it % kRed);
+      const int64_t row = t * kTileRows + lane;
+      const bool valid = lane < kTileRows && row < V;
+      const float rs = (valid && row_scale) ? __ldg(row_scale + row) : 1.0f;
+      const bool ok = wait_all(&red_full[r], (uint32_t)((it / kRed) & 1));
+      const float* rb = red + (size_t)r * kConsumerWarps * kTileRows * 4;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      if (valid && ok) {
 #pragma unroll
-          for (int ww = 0; ww < kConsumerWarps; ++ww) acc += rb[(ww * kTileRows + lane) * 4 + m];
-          const float rs = row_scale ? row_scale[row] : 1.0f;
-          v = acc * rs * __uint_as_float((uint32_t)(127 - s_sigma[m]) << 23);
-          if (logits) logits[(size_t)m * V + row] = v;
-        }
-        // merge into the sorted list: candidates arrive in increasing id order
-        Cand* L = lists + m * top_k;
-        const Cand worst = L[top_k - 1];
-        uint32_t pend = __ballot_sync(0xffffffffu, valid && better(v, (int32_t)row, worst.v, worst.id));
-        while (pend) {
-          const int src = __ffs(pend) - 1;
-          pend &= pend - 1;
-          const float cv = __shfl_sync(0xffffffffu, v, src);
-          const int32_t cid = (int32_t)(t * kTileRows + src);
-          // position = number of entries better than the candidate
-          int pos = 0;
-          for (int base = 0; base < top_k; base += 32) {
-            const int j = base + lane;
-            const bool b = j < top_k && better(L[j].v, L[j].id, cv, cid);
-            pos += __popc(__ballot_sync(0xffffffffu, b));
-          }
-          if (pos < top_k) {
-            for (int base = ((top_k - 1) / 32) * 32; base >= 0; base -= 32) {
-              const int j = base + lane;
-              Cand c{};
-              const bool mv = j >= pos && j < top_k - 1;
-              if (mv) c = L[j];
-              __syncwarp();
-              if (mv) L[j + 1] = c;
-              __syncwarp();
-            }
-            if (lane == 0) L[pos] = Cand{cv, cid};
-            __syncwarp();
-          }
+        for (int ww = 0; ww < kConsumerWarps; ++ww) {
+          const float4 p = *reinterpret_cast<const float4*>(rb + (ww * kTileRows + lane) * 4);
+          acc[0] += p.x; acc[1] += p.y; acc[2] += p.z; acc[3] += p.w;
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&red_empty[r]);
+      for (int m = 0; m < M; ++m) {
+        float v = -FLT_MAX;
+        if (valid) {
+          v = acc[m] * rs * __uint_as_float((uint32_t)(127 - s_sigma[m]) << 23);
+          if (logits) logits[(size_t)m * V + row] = v;
+        }
+        Cand* buf = cbuf + m * kCandBuf;
+        if (cnt[m] + kTileRows > kCandBuf) {
+          cnt[m] = select_top(buf, cnt[m], top_k, lane);
+          if (cnt[m] >= top_k) thr[m] = buf[top_k - 1];
+        }
+        const bool pass = valid && better(v, (int32_t)row, thr[m].v, thr[m].id);
+        const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+        if (pass) buf[cnt[m] + __popc(bal & ((1u << lane) - 1u))] = Cand{v, (int32_t)row};
+        cnt[m] += __popc(bal);
+        __syncwarp();
+      }
     }
+    for (int m = 0; m < M; ++m) {
+      Cand* buf = cbuf + m * kCandBuf;
+      select_top(buf, cnt[m], top_k, lane);
+      for (int i = lane; i < top_k; i += 32) lists[m * top_k + i] = buf[i];
+    }
+    __syncwarp();
   }
 
   // ------------------------- CTA lists -> global ---------------------------
@@ -318,47 +421,68 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
     *s_last = (tk == gridDim.x - 1);
   }
   __syncthreads();
-  if (!*s_last) return;
+  const bool last = *s_last;
+  __syncthreads();  // every thread holds the flag before the merge reuses shared memory
+  if (!last) return;
   __threadfence();
 
   // ------------------------ last CTA: merge the lists ------------------------
-  // One warp per token; each list is sorted, so repeatedly take the best head.
-  uint8_t* heads = ring;  // [M][gridDim] list positions (top_k <= 64); the ring is free now
-  for (int i = threadIdx.x; i < M * (int)gridDim.x; i += blockDim.x) heads[i] = 0;
-  __syncthreads();
-  if (warp < M) {
-    const int m = warp;
-    uint8_t* hm = heads + m * gridDim.x;
-    for (int r = 0; r < top_k; ++r) {
-      float bv = -FLT_MAX;
-      int32_t bid = INT32_MAX;
-      int32_t bc = -1;
-      for (int c = lane; c < (int)gridDim.x; c += 32) {
-        const int hh = hm[c];
-        if (hh < top_k) {
-          const Cand* cc = cand + ((size_t)c * M + m) * top_k + hh;
-          const float cv = __ldcg(&cc->v);
-          const int32_t ci = __ldcg(&cc->id);
-          if (bc < 0 || better(cv, ci, bv, bid)) { bv = cv; bid = ci; bc = c; }
-        }
-      }
-      // warp-wide best, carrying the list index
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int32_t oi = __shfl_xor_sync(0xffffffffu, bid, o);
-        const int32_t oc = __shfl_xor_sync(0xffffffffu, bc, o);
-        if (oc >= 0 && (bc < 0 || better(ov, oi, bv, bid))) { bv = ov; bid = oi; bc = oc; }
-      }
-      if (lane == 0) {
-        out_ids[m * top_k + r] = bid;
-        out_vals[m * top_k + r] = bv;
-        if (bc >= 0) hm[bc] = (uint8_t)(hm[bc] + 1);
-      }
+  // Per token: stage every CTA's sorted list in shared memory.  The k best of
+  // the lists' first entries are k real candidates, so the k-th best of them,
+  // L, is a lower bound on the global k-th best: only entries not worse than
+  // L can be in the top k.  Keep those (typically a few dozen) and select the
+  // top k of them with one warp.
+  Cand* stage = reinterpret_cast<Cand*>(smem);                 // [G * top_k]  (the ring is free now)
+  Cand* surv = stage + (size_t)gridDim.x * top_k;              // [kSurvivors]
+  Cand* wbuf = surv + kSurvivors;                              // [kCandBuf] selection buffer of warp 0
+  int* s_cnt = reinterpret_cast<int*>(wbuf + kCandBuf);
+  Cand* s_bound = reinterpret_cast<Cand*>(s_cnt + 4);
+  const int nl = (int)gridDim.x * top_k;
+  // warp 0's chunked selection: the best top_k of src[0..n) into wbuf[0..top_k)
+  auto select_from = [&](const Cand* src, int n, int stride) {
+    int cnt = 0, pos = 0;
+    do {
+      const int take = min(kCandBuf - cnt, n - pos);
+      for (int i = lane; i < take; i += 32) wbuf[cnt + i] = src[(size_t)(pos + i) * stride];
       __syncwarp();
+      pos += take;
+      cnt = select_top(wbuf, cnt + take, top_k, lane);
+    } while (pos < n);
+  };
+  for (int m = 0; m < M; ++m) {
+    for (int i = threadIdx.x; i < nl; i += blockDim.x) {
+      const int cc = i / top_k, j = i - cc * top_k;
+      const Cand* src = cand + ((size_t)cc * M + m) * top_k + j;
+      stage[i] = Cand{__ldcg(&src->v), __ldcg(&src->id)};
     }
+    if (threadIdx.x == 0) *s_cnt = 0;
+    __syncthreads();
+    if (warp == 0) {
+      select_from(stage, (int)gridDim.x, top_k);  // the lists' first entries
+      if (lane == 0) *s_bound = wbuf[top_k - 1];  // an empty slot (worst) when fewer than top_k lists
+    }
+    __syncthreads();
+    const Cand L = *s_bound;
+    for (int i = threadIdx.x; i < nl; i += blockDim.x) {
+      const Cand e = stage[i];
+      if (!better(L.v, L.id, e.v, e.id)) {  // e is L or better
+        const int pos = atomicAdd(s_cnt, 1);
+        if (pos < kSurvivors) surv[pos] = e;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const int n = *s_cnt;
+      // more survivors than the buffer holds (heavy ties): select from all staged entries instead
+      if (n <= kSurvivors) select_from(surv, n, 1);
+      else select_from(stage, nl, 1);
+      for (int i = lane; i < top_k; i += 32) {
+        out_ids[m * top_k + i] = wbuf[i].id;
+        out_vals[m * top_k + i] = wbuf[i].v;
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
   if (threadIdx.x == 0) hdr->ticket = 0u;
 }
 
@@ -376,12 +500,16 @@ int lmhead_stages(int H, int elem_bytes) {
   return stages;
 }
 
+size_t lmhead_merge_smem_bytes(int grid, int top_k) {
+  return ((size_t)grid * top_k + kSurvivors + kCandBuf) * sizeof(Cand) + 4 * sizeof(int) + sizeof(Cand);
+}
+
 size_t lmhead_smem_bytes(int H, int elem_bytes, int stages) {
   const int stride = padded_stride(H * elem_bytes);
   size_t bytes = (size_t)stages * kTileRows * stride;
-  bytes += 2 * kConsumerWarps * kTileRows * 4 * sizeof(float);
-  bytes += 4 * 64 * sizeof(Cand);
-  bytes += 2 * stages * sizeof(uint64_t) + 8 * sizeof(int);
+  bytes += 4 * kConsumerWarps * kTileRows * 4 * sizeof(float);  // kRed reduce buffers
+  bytes += 4 * 64 * sizeof(Cand) + 4 * kCandBuf * sizeof(Cand);
+  bytes += (2 * stages + 2 * 4) * sizeof(uint64_t) + 8 * sizeof(int);
   return bytes;
 }
 
@@ -392,7 +520,10 @@ static cudaError_t launch_head_t(const uint16_t* x, const W* w, const float* s, 
                                  float* logits, int32_t* ids, float* vals, WsHeader* hdr, void* cand, int grid,
                                  cudaStream_t st) {
   const int stages = lmhead_stages(H, (int)sizeof(W));
-  const size_t smem = lmhead_smem_bytes(H, (int)sizeof(W), stages);
+  size_t smem = lmhead_smem_bytes(H, (int)sizeof(W), stages);
+  const size_t merge = lmhead_merge_smem_bytes(grid, top_k);
+  if (merge > smem) smem = merge;  // the final merge reuses the whole dynamic buffer
+  if (smem > kMaxSmem) return cudaErrorInvalidConfiguration;
   auto kern = lmhead_topk_kernel<W, kSlices>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

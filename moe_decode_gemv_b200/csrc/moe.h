@@ -31,6 +31,9 @@ struct MoeWs {
   float* slot_w;        // [kMaxSlots][4]: combine weight of the slot for token m
   float* h;             // [kMaxSlots][4][I]
   float* ypart;         // [kMaxSlots][4][H]
+  uint32_t* slot_ready; // [kMaxSlots]: rows of h written (reset by the kernel's last CTA)
+  uint32_t* hmax;       // [kMaxSlots][4]: max |h| as fp32 bits (reset likewise)
+  uint32_t* tile_ticket;// [H/32]: slots finished per 32-row output tile (self-resetting)
 
   static size_t align(size_t v) { return (v + 255) & ~size_t(255); }
   static size_t bytes(int M, int top_k, int E, int H, int I) {
@@ -43,6 +46,9 @@ struct MoeWs {
     b += align((size_t)kMaxSlots * 4 * sizeof(float));
     b += align((size_t)kMaxSlots * 4 * I * sizeof(float));
     b += align((size_t)kMaxSlots * 4 * H * sizeof(float));
+    b += align(kMaxSlots * sizeof(uint32_t));
+    b += align((size_t)kMaxSlots * 4 * sizeof(uint32_t));
+    b += align((size_t)(H / 32 + 1) * sizeof(uint32_t));
     return b;
   }
   static MoeWs carve(void* base, int E, int H, int I) {
@@ -55,7 +61,10 @@ struct MoeWs {
     w.slot_mask = reinterpret_cast<uint32_t*>(p); p += align(kMaxSlots * sizeof(uint32_t));
     w.slot_w = reinterpret_cast<float*>(p); p += align((size_t)kMaxSlots * 4 * sizeof(float));
     w.h = reinterpret_cast<float*>(p); p += align((size_t)kMaxSlots * 4 * I * sizeof(float));
-    w.ypart = reinterpret_cast<float*>(p);
+    w.ypart = reinterpret_cast<float*>(p); p += align((size_t)kMaxSlots * 4 * H * sizeof(float));
+    w.slot_ready = reinterpret_cast<uint32_t*>(p); p += align(kMaxSlots * sizeof(uint32_t));
+    w.hmax = reinterpret_cast<uint32_t*>(p); p += align((size_t)kMaxSlots * 4 * sizeof(uint32_t));
+    w.tile_ticket = reinterpret_cast<uint32_t*>(p);
     return w;
   }
 };
@@ -73,7 +82,9 @@ struct MoeArgs {
   MoeWs ws;
 };
 
-size_t moe_ws_bytes(int M, int top_k, int E, int H, int I);
-cudaError_t launch_moe(const MoeArgs& a, cudaStream_t st);
+inline size_t moe_ws_bytes(int M, int top_k, int E, int H, int I) { return MoeWs::bytes(M, top_k, E, H, I); }
+size_t moe_fused_smem_bytes(int H, int I);
+bool moe_fused_supported(int H, int I);
+cudaError_t launch_moe_fused(const MoeArgs& a, cudaStream_t st);
 
 }  // namespace moe

@@ -1,0 +1,63 @@
+// stack_kernels.cu -- the two small steps between the weight streams of a
+// decode step through a stack of MoE layers:
+//  * RMSNorm of a layer's fp32 output into the next layer's bf16 input
+//    (gain 1): out = bf16_RNE(y / sqrt(mean(y^2) + eps));
+//  * the embedding row of each position's greedy token for the next step.
+// Both move kilobytes; they exist so that a whole step (embedding, layers,
+// norms, LM head) can run on the device and be captured in one CUDA graph.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "stack.h"
+
+namespace moe {
+namespace {
+
+// One CTA per row.
+__global__ void rmsnorm_bf16_kernel(const float* __restrict__ y, int H, float eps, uint16_t* __restrict__ out) {
+  const float* row = y + (size_t)blockIdx.x * H;
+  float ss = 0.f;
+  for (int j = threadIdx.x; j < H; j += blockDim.x) ss = fmaf(row[j], row[j], ss);
+  ss = warp_sum(ss);
+  __shared__ float part[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) part[warp] = ss;
+  __syncthreads();
+  if (warp == 0) {
+    float v = lane < (int)(blockDim.x >> 5) ? part[lane] : 0.f;
+    v = warp_sum(v);
+    if (lane == 0) part[0] = sqrtf(__fdiv_rn(v, (float)H) + eps);
+  }
+  __syncthreads();
+  const float rms = part[0];
+  for (int j = threadIdx.x; j < H; j += blockDim.x) {
+    const __nv_bfloat16 b = __float2bfloat16_rn(__fdiv_rn(row[j], rms));
+    out[(size_t)blockIdx.x * H + j] = *reinterpret_cast<const uint16_t*>(&b);
+  }
+}
+
+// One CTA per position; 16-byte copies.  An id outside [0, V) yields a zero
+// row (no out-of-bounds read).
+__global__ void embed_gather_kernel(const uint16_t* __restrict__ table, int64_t V, int H,
+                                    const int32_t* __restrict__ ids, int ids_stride, uint16_t* __restrict__ out) {
+  const int32_t id = ids[(size_t)blockIdx.x * ids_stride];
+  const bool ok = id >= 0 && id < V;
+  const uint4* src = reinterpret_cast<const uint4*>(table + (size_t)(ok ? id : 0) * H);
+  uint4* dst = reinterpret_cast<uint4*>(out + (size_t)blockIdx.x * H);
+  for (int j = threadIdx.x; j < H / 8; j += blockDim.x) dst[j] = ok ? src[j] : make_uint4(0, 0, 0, 0);
+}
+
+}  // namespace
+
+cudaError_t launch_rmsnorm_bf16(const float* y, int M, int H, float eps, uint16_t* out, cudaStream_t st) {
+  rmsnorm_bf16_kernel<<<M, 256, 0, st>>>(y, H, eps, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_embed_gather(const uint16_t* table, int64_t V, int H, const int32_t* ids, int ids_stride, int M,
+                                uint16_t* out, cudaStream_t st) {
+  embed_gather_kernel<<<M, 128, 0, st>>>(table, V, H, ids, ids_stride, out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

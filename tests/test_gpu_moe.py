@@ -105,10 +105,11 @@ def test_every_expert_selected_and_top1(B, O):
 
 
 def test_odd_sizes(B, O):
-    """H and I at their smallest multiples of 32 that are not powers of two."""
-    s = I.MoEShape(hidden=96, inter=160, experts=24, top_k=3)
+    """H and I multiples of 64 that are not powers of two, E not a multiple of
+    the CTA count, top_k = 3."""
+    s = I.MoEShape(hidden=192, inter=192, experts=24, top_k=3)
     layer = Layer(B, 6, s)
-    x = I.hidden_states(6, 3, 96)
+    x = I.hidden_states(6, 3, 192)
     y, ids, w = layer.run_gpu(x.cuda())
     check_moe(layer, O, x, y, ids, w)
 
