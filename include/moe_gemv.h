@@ -191,6 +191,24 @@ MOE_API moe_status lmhead_decode_bf16(const uint16_t* hidden_bf16, const moe_bf1
                               int32_t M, int32_t top_k, int32_t* topk_ids, float* topk_vals,
                               float* logits, void* workspace, size_t workspace_bytes, void* stream);
 
+/* lmhead_decode for callers that cannot provide a workspace: hosts that own
+ * every device allocation and give a plugin only its inputs and outputs, or
+ * loops that must not call cudaMalloc (it can synchronise the device).  No
+ * counterpart on the pages: this is an interface convenience.  The scratch is
+ * one fixed device array of MOE_LMHEAD_NOALLOC_SCRATCH_BYTES, held by every
+ * GPU that loads the library until the process exits.  It must fit a 64-byte
+ * header plus (SM count) x M x top_k x 8 bytes of candidate lists, e.g.
+ * M x top_k <= 221 on a 148-SM B200; larger requests return
+ * MOE_ERR_WORKSPACE.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) and should come before any stream capture.
+ * Each call clears the array's header on `stream` before its kernel.  All
+ * calls share the array, so calls that overlap on the GPU (different
+ * streams, or different threads) race: serialise them.  Allocates nothing.  */
+#define MOE_LMHEAD_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+MOE_API moe_status lmhead_decode_noalloc(const uint16_t* hidden_bf16, const moe_fp8_head* head,
+                                         int32_t M, int32_t top_k, int32_t* topk_ids, float* topk_vals,
+                                         float* logits, void* stream);
+
 /* ---- between the layers of a decode step ---------------------------------- */
 
 /* The next layer's input from a layer's output, for a stack of MoE layers

@@ -77,6 +77,7 @@ def _load() -> ctypes.CDLL:
         "lmhead_workspace_bytes": ([I32, I32, I64, I64], SZ),
         "lmhead_decode": ([P, ctypes.POINTER(_Fp8Head), I32, I32, P, P, P, P, SZ, P], I32),
         "lmhead_decode_bf16": ([P, ctypes.POINTER(_Bf16Head), I32, I32, P, P, P, P, SZ, P], I32),
+        "lmhead_decode_noalloc": ([P, ctypes.POINTER(_Fp8Head), I32, I32, P, P, P, P], I32),
         "moe_rmsnorm_bf16": ([P, I32, I32, ctypes.c_float, P, P], I32),
         "moe_embed_gather": ([P, I64, I64, P, I32, I32, P, P], I32),
         "moe_workspace_reset": ([P, SZ, P], I32),
@@ -247,6 +248,18 @@ def lmhead_decode_bf16(hidden: torch.Tensor, w_bf16: torch.Tensor, top_k: int, t
     st = library.lmhead_decode_bf16(_ptr(hidden), ctypes.byref(c), M, top_k, _ptr(topk_ids), _ptr(topk_vals),
                                     _ptr(logits), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "lmhead_decode_bf16")
+    return topk_ids, topk_vals
+
+
+def lmhead_decode_noalloc(hidden: torch.Tensor, head: FP8Head, top_k: int, topk_ids: torch.Tensor,
+                          topk_vals: torch.Tensor, logits: torch.Tensor | None = None, stream=None):
+    """lmhead_decode without a workspace: for callers that cannot allocate
+    device memory; the library's fixed scratch array is used instead (calls
+    that overlap on the GPU race on it)."""
+    c = head._c()
+    st = library.lmhead_decode_noalloc(_ptr(hidden), ctypes.byref(c), hidden.shape[0], top_k, _ptr(topk_ids),
+                                       _ptr(topk_vals), _ptr(logits), _stream(stream))
+    _check(st, "lmhead_decode_noalloc")
     return topk_ids, topk_vals
 
 

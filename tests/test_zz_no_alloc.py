@@ -1,0 +1,65 @@
+"""The workspace-free LM-head entry point, for callers that cannot allocate
+device memory (a host that owns every allocation and hands a plugin only its
+inputs and outputs, or a loop where cudaMalloc is not allowed).
+
+It must agree with lmhead_decode, which takes a caller workspace, on two calls
+in a row (the second reuses the scratch the first left behind), and refuse a
+request too large for its fixed scratch.  Collected last on purpose."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_support import MAX_ABS_TOL, REL_L2_TOL, rel_l2
+from moe_decode_gemv_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B():
+    from moe_decode_gemv_b200 import build
+    build.build()
+    from moe_decode_gemv_b200 import binding
+    return binding
+
+
+def _outputs(M, k, V, dev="cuda"):
+    return (torch.empty((M, k), dtype=torch.int32, device=dev), torch.empty((M, k), dtype=torch.float32, device=dev),
+            torch.empty((M, V), dtype=torch.float32, device=dev))
+
+
+@pytest.mark.parametrize("shape,M,k", [(I.TINY_HEAD, 1, 1), (I.TINY_HEAD, 4, 29), (I.LING_HEAD, 1, 29),
+                                       (I.LING_HEAD, 4, 29)])
+def test_matches_workspace_entry_point_twice(B, shape, M, k):
+    head = B.lmhead_quantize_fp8(I.lmhead_weight(0, shape).cuda())
+    ref_ids, ref_vals, ref_logits = _outputs(M, k, shape.vocab)
+    for call in range(2):
+        x = I.hidden_states(call, M, shape.hidden, tag="noalloc").cuda()
+        B.lmhead_decode(x, head, k, ref_ids, ref_vals, ref_logits)
+        ids, vals, logits = _outputs(M, k, shape.vocab)
+        B.lmhead_decode_noalloc(x, head, k, ids, vals, logits)
+        torch.cuda.synchronize()
+        assert torch.equal(ids, ref_ids), f"call {call}: ids differ"
+        v, rv = vals.cpu().numpy(), ref_vals.cpu().numpy()
+        assert np.abs(v - rv).max() <= MAX_ABS_TOL
+        lg, rlg = logits.cpu().numpy(), ref_logits.cpu().numpy()
+        assert rel_l2(lg, rlg) <= REL_L2_TOL and np.abs(lg - rlg).max() <= MAX_ABS_TOL
+
+
+def test_refuses_requests_beyond_its_scratch(B):
+    """M x top_k candidate lists for every SM must fit the fixed scratch."""
+    head = B.lmhead_quantize_fp8(I.lmhead_weight(0, I.TINY_HEAD).cuda())
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    limit = B.library.lmhead_decode_noalloc  # raw C call: expect a status, not an exception
+    M, k = 4, 64
+    need = 64 + min(sms, I.TINY_HEAD.vocab // 16) * M * k * 8
+    x = I.hidden_states(0, M, I.TINY_HEAD.hidden).cuda()
+    ids, vals, _ = _outputs(M, k, I.TINY_HEAD.vocab)
+    c = head._c()
+    st = limit(ctypes.c_void_p(x.data_ptr()), ctypes.byref(c), M, k, ctypes.c_void_p(ids.data_ptr()),
+               ctypes.c_void_p(vals.data_ptr()), None, None)
+    expected = B.Status.WORKSPACE if need > 256 * 1024 else B.Status.OK
+    assert st == expected, (st, need)
+    torch.cuda.synchronize()
