@@ -53,6 +53,8 @@ def parse():
     p.add_argument("--only", choices=["all", "head", "moe"], default="all",
                    help="profiling aid: time only one half of the step (small device footprint)")
     p.add_argument("--layers", type=int, default=N_LAYERS, help="layer copies that rotate (profiling aid)")
+    p.add_argument("--no-stream", action="store_true", help="skip the 16-layer decode-stream leg")
+    p.add_argument("--stream-steps", type=int, default=200)
     return p.parse_args()
 
 
@@ -292,6 +294,102 @@ def time_bf16_head(wl, M, steps):
 
 
 # ---------------------------------------------------------------------------
+# the decode-step stream: 16 layers + LM head, greedy feedback
+# ---------------------------------------------------------------------------
+
+STREAM_LAYERS = 16
+
+
+class Stream:
+    """A stack of 16 Ling-shaped layers (each re-routed from the previous
+    layer's RMS-normalised output), the FP8 LM head and a bf16 embedding table;
+    one step embeds the previous greedy tokens, runs the stack and the head."""
+
+    def __init__(self, B, I, seed, device, M, head, x_table=None):
+        import torch
+        self.B, self.torch, self.M = B, torch, M
+        s, h = I.LING_MOE, I.LING_HEAD
+        self.s, self.h = s, h
+        self.layers = []
+        for l in range(STREAM_LAYERS):
+            router = I.router_weight(seed, s.experts, s.hidden, layer=100 + l, device=device)
+            banks, shared = [], []
+            for kind in ("gate", "up", "down"):
+                rows, cols = (s.inter, s.hidden) if kind != "down" else (s.hidden, s.inter)
+                st = I.normal(seed, f"S{l}/bank/{kind}", (s.experts, rows, cols), I.WEIGHT_STD, device=device)
+                banks.append(B.moe_quantize_mxfp4(st))
+                del st
+                shared.append(B.moe_quantize_mxfp4(I.expert_matrix(seed, s, "shared", kind, layer=100 + l,
+                                                                    device=device)))
+            self.layers.append((router, tuple(banks), tuple(shared)))
+        self.head = head
+        self.table = I.normal(seed, "embed", (h.vocab, h.hidden), 1.0, device=device)
+        self.ids = torch.arange(M, dtype=torch.int32, device=device).view(M, 1).repeat(1, 1) * 7 + 3
+        self.x = torch.empty((M, s.hidden), dtype=torch.bfloat16, device=device)
+        self.y = torch.empty((M, s.hidden), dtype=torch.float32, device=device)
+        self.tv = torch.empty((M, 1), dtype=torch.float32, device=device)
+        self.moe_ws = B.new_workspace(B.moe_workspace_bytes(M, s.top_k, s.experts, s.hidden, s.inter), device)
+        self.head_ws = B.new_workspace(B.lmhead_workspace_bytes(M, 1, h.vocab, h.hidden), device)
+        torch.cuda.synchronize()
+
+    def step(self):
+        B = self.B
+        B.moe_embed_gather(self.table, self.ids, self.x, ids_stride=1)
+        for router, banks, shared in self.layers:
+            B.moe_decode(self.x, router, None, banks, shared, self.s.top_k, self.y, workspace=self.moe_ws)
+            B.moe_rmsnorm_bf16(self.y, self.x, 1e-6)
+        B.lmhead_decode(self.x, self.head, 1, self.ids, self.tv, None, workspace=self.head_ws)
+
+    def run(self, steps, warmup=3):
+        """Device time per step; the step is captured as one CUDA graph when
+        capture works, else launched directly."""
+        torch = self.torch
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        graph = None
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.step()
+            graph = g
+        except Exception as exc:  # capture unsupported: direct launches
+            graph = None
+            capture_error = str(exc).splitlines()[0]
+        run = graph.replay if graph is not None else self.step
+        for _ in range(warmup):
+            run()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(steps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / steps
+        out = {"steps": steps, "us_per_step": us, "cuda_graph": graph is not None}
+        if graph is None:
+            out["capture_error"] = capture_error
+        return out
+
+
+def stream_leg(wl, B, I, A, seed, device, steps):
+    res = {}
+    for M in (1, 4):
+        st = Stream(B, I, seed, device, M, wl.head)
+        r = st.run(steps if M == 1 else max(steps // 4, 1))
+        if M == 1:
+            nbytes = STREAM_LAYERS * A.moe_layer_bytes(I.LING_MOE, I.LING_MOE.top_k) + A.lmhead_fp8_bytes(I.LING_HEAD)
+            r["algorithmic_bytes_per_step"] = nbytes
+            r["achieved_gbs"] = nbytes / (r["us_per_step"] * 1e-6) / 1e9
+        res[f"m{M}"] = r
+        del st
+        import torch
+        torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle (baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 
@@ -521,6 +619,11 @@ def main():
     if m4 is not None:
         line["m4"] = {"us_per_step": m4["per_step_us"], "moe_us_mean": m4["moe_us_mean"],
                       "head_us_mean": m4["head_us_mean"], "steps": max(args.steps // 2, 1)}
+    if not args.no_stream:
+        try:
+            line["stream_16_layers"] = stream_leg(wl, B, I, A, args.seed + rank, device, args.stream_steps)
+        except Exception as exc:  # the headline numbers above stand without this leg
+            line["stream_16_layers"] = {"error": f"{type(exc).__name__}: {str(exc).splitlines()[0][:200]}"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.seed)
     if dist is not None:

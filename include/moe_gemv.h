@@ -180,7 +180,11 @@ MOE_API size_t lmhead_workspace_bytes(int32_t M, int32_t top_k, int64_t vocab, i
  *            greedy argmax); 1 <= top_k <= 64
  *   logits   [M][vocab] fp32 or NULL: every logit, when the caller wants them
  *   workspace: at least lmhead_workspace_bytes(...), zeroed once before use.
- * Supported: hidden a multiple of 64 and at most 5120, vocab < 2^31.       */
+ * Supported: hidden a multiple of 64 and at most 5120, vocab < 2^31, and a
+ * vocabulary whose logits fit in shared memory across the GPU's SMs while the
+ * head streams (each CTA keeps its rows' M logits: on a 148-SM B200 about
+ * 1.2 M rows at M = 4 and H = 2560); larger returns
+ * MOE_ERR_UNSUPPORTED_SHAPE.                                                */
 MOE_API moe_status lmhead_decode(const uint16_t* hidden_bf16, const moe_fp8_head* head,
                          int32_t M, int32_t top_k, int32_t* topk_ids, float* topk_vals,
                          float* logits, void* workspace, size_t workspace_bytes, void* stream);
@@ -242,6 +246,18 @@ MOE_API moe_status moe_workspace_status(void* workspace, void* stream);
  * optimisation is live (ncijnetwork.com summary, "The integration trap");
  * this is the string to log.                                                 */
 MOE_API moe_status moe_query_path(char* buf, size_t n);
+
+/* Self-test of the bounded device waits; the pages have no counterpart.
+ * Enqueues one small kernel that waits on a word of the workspace header that
+ * no kernel ever writes, using the same bounded wait as the decode kernels but
+ * with a limit of `limit_us` microseconds (1 .. 1,000,000).  When the limit
+ * runs out the kernel records MOE_ERR_TIMEOUT in the workspace's status word
+ * and returns; read it with moe_workspace_status.  The decode kernels' own
+ * limit is 1 s.  Any workspace of at least 64 bytes serves; calls that
+ * overlap on the GPU must not share one.  Returns MOE_ERR_WORKSPACE,
+ * MOE_ERR_MISALIGNED or MOE_ERR_INVALID_ARG for bad arguments.             */
+MOE_API moe_status moe_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint32_t limit_us,
+                                             void* stream);
 
 /* Text for a status code ("MOE_ERR_FORMAT_MISMATCH", ...); never NULL.       */
 MOE_API const char* moe_status_string(moe_status s);

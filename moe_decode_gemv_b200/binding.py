@@ -84,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "moe_workspace_status": ([P, P], I32),
         "moe_query_path": ([ctypes.c_char_p, SZ], I32),
         "moe_status_string": ([I32], ctypes.c_char_p),
+        "moe_selftest_wait_timeout": ([P, SZ, ctypes.c_uint32, P], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -281,6 +282,13 @@ def moe_embed_gather(table: torch.Tensor, ids: torch.Tensor, out: torch.Tensor, 
 
 def moe_workspace_status(workspace: torch.Tensor, stream=None) -> Status:
     return Status(library.moe_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def moe_selftest_wait_timeout(workspace: torch.Tensor, limit_us: int, stream=None) -> None:
+    """Enqueue a bounded wait on a flag that nothing sets (limit in
+    microseconds); the kernel records TIMEOUT in the workspace status word."""
+    _check(library.moe_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(limit_us), _stream(stream)),
+           "moe_selftest_wait_timeout")
 
 
 def moe_query_path() -> str:

@@ -10,6 +10,7 @@
 
 #include "../../include/moe_gemv.h"
 #include "common.cuh"
+#include "device_cache.h"
 #include "lmhead.h"
 #include "moe.h"
 #include "quantize.h"
@@ -65,11 +66,13 @@ moe_status launch_head_common(const uint16_t* hidden, const void* w, const float
   if (ws_bytes < head_ws_bytes(M, top_k)) return MOE_ERR_WORKSPACE;
 
   int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::current_device_sms(&dev, &sms) != cudaSuccess) return MOE_ERR_CUDA;
   const int64_t ntiles = (V + 15) / 16;
   int grid = sms < kHeadMaxGrid ? sms : kHeadMaxGrid;
   if (grid > ntiles) grid = (int)ntiles;
+  int stages = 0;
+  size_t smem = 0;  // each CTA keeps its rows' logits in shared memory: a limit on vocab / SMs
+  if (!moe::lmhead_plan((int)H, fp8 ? 1 : 2, M, top_k, V, grid, &stages, &smem)) return MOE_ERR_UNSUPPORTED_SHAPE;
   auto* hdr = static_cast<moe::WsHeader*>(ws);
   void* cand = static_cast<uint8_t*>(ws) + sizeof(moe::WsHeader);
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -42,17 +42,23 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-// Polls `ready()` until it returns true or kWaitLimitNs have passed, sleeping
+// Polls `ready()` until it returns true or `limit_ns` have passed, sleeping
 // `backoff_ns` between polls so that a waiting warp leaves the issue slots to
 // the warps doing the work.  Returns false on timeout.
 template <typename F>
-__device__ __forceinline__ bool bounded_spin(F ready, uint32_t backoff_ns = 64) {
+__device__ __forceinline__ bool bounded_spin_for(F ready, uint64_t limit_ns, uint32_t backoff_ns = 64) {
   const uint64_t start = global_ns();
   for (;;) {
     if (ready()) return true;
-    if (global_ns() - start > kWaitLimitNs) return false;
+    if (global_ns() - start > limit_ns) return false;
     if (backoff_ns) __nanosleep(backoff_ns);
   }
+}
+
+// The same with the library's limit, kWaitLimitNs.
+template <typename F>
+__device__ __forceinline__ bool bounded_spin(F ready, uint32_t backoff_ns = 64) {
+  return bounded_spin_for(ready, kWaitLimitNs, backoff_ns);
 }
 
 // ---------------------------------------------------------------------------
@@ -99,6 +105,48 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Eight E2M1 codes (one word, element i in nibble i) -> eight E4M3 codes by
+// moving bits only: E2M1 s|e1 e0|m becomes E4M3 s|0 0 e1 e0|m 0 0, whose
+// value is the E2M1 value times 2^-6 for every code (the E2M1 subnormal 0.5
+// becomes the E4M3 subnormal 2^-7).  `even` gets elements 0, 2, 4, 6 in bytes
+// 0..3 and `odd` elements 1, 3, 5, 7; a caller pairs them with activations
+// permuted the same way.
+__device__ __forceinline__ uint32_t e2m1x8_even_to_e4m3x4(uint32_t w) {
+  return ((w << 2) & 0x1c1c1c1cu) | ((w << 4) & 0x80808080u);
+}
+__device__ __forceinline__ uint32_t e2m1x8_odd_to_e4m3x4(uint32_t w) {
+  return ((w >> 2) & 0x1c1c1c1cu) | (w & 0x80808080u);
+}
+
+// E4M3 x E4M3 -> fp32 tensor-core MMA, m16n8k32 (A row-major 16x32, B 32x8).
+__device__ __forceinline__ void mma_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four fp32 values -> E4M3 parts (byte j of each part belongs to value j):
+// p[0] = rne(v), p[1] = rne(v - p[0]), p[2] = rne(v - p[0] - p[1]), ...
+// Each part takes the next four significant bits of v as long as the
+// remainder stays in E4M3's normal range; the residues are exact in fp32.
+template <int kParts>
+__device__ __forceinline__ void split_e4m3x4(float a, float b, float c, float d, uint32_t (&p)[kParts]) {
+#pragma unroll
+  for (int q = 0; q < kParts; ++q) {
+    const uint32_t ab = f32x2_to_e4m3x2(a, b), cd = f32x2_to_e4m3x2(c, d);
+    p[q] = ab | (cd << 16);
+    if (q + 1 < kParts) {
+      const uint32_t fab = e4m3x2_to_f16x2(ab), fcd = e4m3x2_to_f16x2(cd);
+      const float2 rab = __half22float2(*reinterpret_cast<const __half2*>(&fab));
+      const float2 rcd = __half22float2(*reinterpret_cast<const __half2*>(&fcd));
+      a -= rab.x; b -= rab.y; c -= rcd.x; d -= rcd.y;
+    }
+  }
+}
 
 // ---------------------------------------------------------------------------
 // Warp reductions.

@@ -9,9 +9,10 @@
 
 namespace moe {
 
-int lmhead_stages(int H, int elem_bytes);
 int lmhead_max_slices();
-size_t lmhead_smem_bytes(int H, int elem_bytes, int stages);
+// Ring depth and shared memory of one launch; false if the shape does not fit
+// in one CTA's shared memory (the CTA keeps its rows' logits there).
+bool lmhead_plan(int H, int elem_bytes, int M, int top_k, int64_t V, int grid, int* stages, size_t* smem);
 size_t lmhead_cand_bytes(int grid, int M, int top_k);
 
 cudaError_t launch_lmhead_fp8(const uint16_t* x, const uint8_t* q, const float* s, int64_t V, int H, int M,

@@ -26,15 +26,19 @@
 //    bf16 value exactly (8 significand bits = 4 + 4) for every element above
 //    E4M3's subnormal range; the two parts take two MMAs.  The logit is
 //    acc * s_v * 2^-sigma_m.
-//  * Epilogue per tile: the consumers' partial sums meet in shared memory;
-//    one warp per token applies the row scale, writes logits when asked and
-//    merges the 16 candidates into the CTA's running top-k list (sorted, ties
-//    to the lower id).  The last CTA to finish merges all CTAs' lists.
+//  * Epilogue: two warps take alternate tiles.  A tile's 16 row scales ride
+//    in its ring stage (one more bulk copy) and reach the epilogue with the
+//    consumers' partial sums, so no global load sits on the epilogue's path.
+//    The epilogue sums the partials, applies the row scale and 2^-sigma_m,
+//    writes logits when asked, and offers the 16 values to a per-token sorted
+//    top-k list held in its registers (ties to the lower id).  The last CTA to
+//    finish merges all CTAs' lists.
 #include <cuda_runtime.h>
 
 #include <cfloat>
 
 #include "common.cuh"
+#include "device_cache.h"
 #include "lmhead.h"
 
 namespace moe {
@@ -42,9 +46,10 @@ namespace {
 
 constexpr int kTileRows = 16;
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 2) * 32;  // consumers + producer + epilogue
+constexpr int kEpilogueWarps = 2;  // alternate tiles
+constexpr int kThreads = (kConsumerWarps + 1 + kEpilogueWarps) * 32;  // consumers + producer + epilogue
 constexpr int kMaxSlicesPerWarp = 10;  // row bytes <= 10 * 8 * 64 = 5120: H <= 5120 (fp8), 2560 (bf16)
-constexpr size_t kMaxSmem = 232448;    // 227 KB of dynamic shared memory per CTA
+constexpr size_t kMaxSmem = kMaxDynamicSmem;
 
 template <typename W>
 struct HeadTraits;
@@ -63,23 +68,6 @@ struct HeadTraits<uint16_t> {
   static constexpr int kMmasPerSlice = 2;
 };
 
-__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void mma_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -95,45 +83,153 @@ __host__ __device__ constexpr int padded_stride(int row_bytes) {
   return (row_bytes % 128 == 0) ? row_bytes + 64 : row_bytes;
 }
 
+// One ring stage: 16 rows at the padded stride, then the 16 rows' fp32 scales
+// (64 B), rounded up to 128 B.
+__host__ __device__ constexpr int stage_bytes(int row_bytes) {
+  return (kTileRows * padded_stride(row_bytes) + 64 + 127) / 128 * 128;
+}
+
 struct Cand {
   float v;
   int32_t id;
 };
 
-constexpr int kCandBuf = 128;     // per-token candidate buffer of the epilogue warp
-constexpr int kSurvivors = 2048;  // entries kept by the final merge's lower bound
+constexpr uint32_t kFull = 0xffffffffu;
 
-// Warp-cooperative: move the best min(k, n) of buf[0..n) to buf[0..) in order
-// (value descending, ties to the lower id), padding with empty candidates up
-// to k.  Returns min(k, n).  Selection by repeated warp argmax: O(n k / 32).
-__device__ int select_top(Cand* buf, int n, int k, int lane) {
-  constexpr int kPer = kCandBuf / 32;
-  Cand c[kPer];
-  bool taken[kPer];
+// A sorted top-k list (k <= 64) held in one warp's registers: rank r < 32 sits
+// in lane r of row 0, rank 32 + r in lane r of row 1.  Ranks >= k are unused.
+// Empty entries are (-FLT_MAX, INT32_MAX), below every admissible candidate.
+// (tv, ti), replicated in every lane, is the entry at rank k - 1: a candidate
+// enters only if it is better than that one.
+struct WarpList {
+  float v0, v1;
+  int32_t i0, i1;
+  float tv;
+  int32_t ti;
+};
+
+__device__ __forceinline__ void list_init(WarpList& L) {
+  L.v0 = L.v1 = L.tv = -FLT_MAX;
+  L.i0 = L.i1 = L.ti = INT32_MAX;
+}
+
+// Insert (cv, ci), known to be better than the threshold (warp-uniform call).
+// Its rank p is the number of kept entries better than it; entries at ranks
+// >= p move down one place and the one at rank k - 1 drops out.
+__device__ __forceinline__ void list_insert(WarpList& L, float cv, int32_t ci, int k, int lane) {
+  const uint32_t m0 = k >= 32 ? kFull : ((1u << k) - 1u);
+  int p = __popc(__ballot_sync(kFull, better(L.v0, L.i0, cv, ci)) & m0);
+  if (k > 32) {
+    const uint32_t m1 = k >= 64 ? kFull : ((1u << (k - 32)) - 1u);
+    p += __popc(__ballot_sync(kFull, better(L.v1, L.i1, cv, ci)) & m1);
+    float u = __shfl_up_sync(kFull, L.v1, 1);
+    int32_t j = __shfl_up_sync(kFull, L.i1, 1);
+    const float carry_v = __shfl_sync(kFull, L.v0, 31);  // rank 31 moves to rank 32
+    const int32_t carry_i = __shfl_sync(kFull, L.i0, 31);
+    if (lane == 0) { u = carry_v; j = carry_i; }
+    if (32 + lane > p) { L.v1 = u; L.i1 = j; }
+    else if (32 + lane == p) { L.v1 = cv; L.i1 = ci; }
+  }
+  const float u = __shfl_up_sync(kFull, L.v0, 1);
+  const int32_t j = __shfl_up_sync(kFull, L.i0, 1);
+  if (lane > p) { L.v0 = u; L.i0 = j; }
+  else if (lane == p) { L.v0 = cv; L.i0 = ci; }
+  const int t = k - 1;
+  L.tv = __shfl_sync(kFull, t < 32 ? L.v0 : L.v1, t & 31);
+  L.ti = __shfl_sync(kFull, t < 32 ? L.i0 : L.i1, t & 31);
+}
+
+// Offer one candidate per lane (ignored where !valid).  Candidates that beat
+// the threshold are inserted one at a time, lowest lane first, re-testing the
+// rest against the raised threshold after each insertion.
+__device__ __forceinline__ void list_offer(WarpList& L, float v, int32_t id, bool valid, int k, int lane) {
+  uint32_t bal = __ballot_sync(kFull, valid && better(v, id, L.tv, L.ti));
+  while (bal) {
+    const int src = __ffs(bal) - 1;
+    const float cv = __shfl_sync(kFull, v, src);
+    const int32_t ci = __shfl_sync(kFull, id, src);
+    list_insert(L, cv, ci, k, lane);
+    bal &= (bal - 1u) & __ballot_sync(kFull, valid && better(v, id, L.tv, L.ti));
+  }
+}
+
+constexpr int kCandCap = 256;  // candidates a warp ranks by counting (more: the list path)
+
+// The best k (<= 64) of vals[0..n) under `better`, entry i carrying the id
+// row0 + i, by one warp; writes the sorted list (padded with empty entries
+// when fewer than k are admissible) to out[0..k).  NaN and -inf values are
+// not admissible.  The values fall into 64 groups (i mod 64); the k-th best
+// of the group maxima, L, is a lower bound on the k-th best value (those are
+// k real entries), so only values not worse than L can be selected -- a few
+// dozen -- and they are ranked by counting.  `scratch` holds kCandCap entries.
+__device__ void warp_topk_rows(const float* vals, int n, int64_t row0, int k, int lane, Cand* scratch, Cand* out) {
+  float m0 = -FLT_MAX, m1 = -FLT_MAX;
+  int32_t j0 = INT32_MAX, j1 = INT32_MAX;
+  for (int i = lane; i < n; i += 32) {
+    const float v = vals[i];
+    const int32_t id = (int32_t)(row0 + i);
+    if (((i >> 5) & 1) == 0) {
+      if (better(v, id, m0, j0)) { m0 = v; j0 = id; }
+    } else if (better(v, id, m1, j1)) {
+      m1 = v; j1 = id;
+    }
+  }
+  int r0 = 0, r1 = 0;
+  for (int j = 0; j < 32; ++j) {
+    const float a = __shfl_sync(kFull, m0, j), b = __shfl_sync(kFull, m1, j);
+    const int32_t ai = __shfl_sync(kFull, j0, j), bi = __shfl_sync(kFull, j1, j);
+    r0 += better(a, ai, m0, j0) + better(b, bi, m0, j0);
+    r1 += better(a, ai, m1, j1) + better(b, bi, m1, j1);
+  }
+  // real maxima have distinct ids, so at most one has rank k - 1; none when
+  // fewer than k groups hold an admissible value (then there is no bound)
+  const uint32_t s0 = __ballot_sync(kFull, r0 == k - 1 && j0 != INT32_MAX);
+  const uint32_t s1 = __ballot_sync(kFull, r1 == k - 1 && j1 != INT32_MAX);
+  float Lv = -FLT_MAX;
+  int32_t Li = INT32_MAX;
+  if (s0) {
+    Lv = __shfl_sync(kFull, m0, __ffs(s0) - 1);
+    Li = __shfl_sync(kFull, j0, __ffs(s0) - 1);
+  } else if (s1) {
+    Lv = __shfl_sync(kFull, m1, __ffs(s1) - 1);
+    Li = __shfl_sync(kFull, j1, __ffs(s1) - 1);
+  }
+  auto keep = [&](float v, int32_t id) { return v >= -FLT_MAX && !better(Lv, Li, v, id); };
+  int cnt = 0;
+  for (int i = lane; i < n; i += 32) cnt += keep(vals[i], (int32_t)(row0 + i)) ? 1 : 0;
+  int off = cnt;  // inclusive prefix sum over lanes
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int j = lane + 32 * i;
-    c[i] = j < n ? buf[j] : Cand{-FLT_MAX, INT32_MAX};
-    taken[i] = j >= n;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(kFull, off, o);
+    if (lane >= o) off += t;
+  }
+  const int nc = __shfl_sync(kFull, off, 31);
+  off -= cnt;
+  if (nc <= kCandCap) {
+    for (int i = lane; i < n; i += 32) {
+      const float v = vals[i];
+      const int32_t id = (int32_t)(row0 + i);
+      if (keep(v, id)) scratch[off++] = Cand{v, id};
+    }
+    __syncwarp();
+    for (int q = lane; q < nc; q += 32) {
+      const Cand e = scratch[q];
+      int r = 0;
+      for (int o = 0; o < nc; ++o) r += better(scratch[o].v, scratch[o].id, e.v, e.id);
+      if (r < k) out[r] = e;
+    }
+    for (int j = nc + lane; j < k; j += 32) out[j] = Cand{-FLT_MAX, INT32_MAX};
+  } else {  // heavy ties: a sorted register list over every value
+    WarpList L;
+    list_init(L);
+    for (int b = 0; b < n; b += 32) {
+      const bool valid = b + lane < n;
+      list_offer(L, valid ? vals[b + lane] : -FLT_MAX, (int32_t)(row0 + b + lane), valid, k, lane);
+    }
+    if (lane < k) out[lane] = Cand{L.v0, L.i0};
+    if (32 + lane < k) out[32 + lane] = Cand{L.v1, L.i1};
   }
   __syncwarp();
-  const int keep = n < k ? n : k;
-  for (int r = 0; r < k; ++r) {
-    float bv = -FLT_MAX;
-    int32_t bi = INT32_MAX;
-    int bslot = -1;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i)
-      if (!taken[i] && (bslot < 0 || better(c[i].v, c[i].id, bv, bi))) { bv = c[i].v; bi = c[i].id; bslot = i; }
-    float wv = bv;
-    int32_t wi = bi;
-    warp_best(wv, wi);
-    // the owner of the winner marks it taken (ids are unique among real candidates)
-    if (r < keep && bslot >= 0 && bi == wi && bv == wv) taken[bslot] = true;
-    if (lane == 0) buf[r] = r < keep ? Cand{wv, wi} : Cand{-FLT_MAX, INT32_MAX};
-  }
-  __syncwarp();
-  return keep;
 }
 
 // Warp roles: warp 0..7 consumers (K split), warp 8 producer (bulk copies),
@@ -159,14 +255,18 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
   extern __shared__ __align__(128) uint8_t smem[];
   const int row_bytes = H * T::kElemBytes;
   const int stride = padded_stride(row_bytes);
-  const int tile_bytes = kTileRows * stride;
+  const int tile_bytes = stage_bytes(row_bytes);  // 16 rows at `stride`, then their 16 fp32 row scales
+  const int scale_off = kTileRows * stride;
 
-  // shared-memory carve-up: [ring][reduce buffers][top-k lists][barriers][scalars]
+  const int64_t ntiles = (V + kTileRows - 1) / kTileRows;
+  const int n_cap = (int)((ntiles + gridDim.x - 1) / gridDim.x) * kTileRows;  // rows of the largest CTA range
+
+  // shared-memory carve-up: [ring][reduce buffers][row scales][logits of this CTA's rows][barriers][scalars]
   uint8_t* ring = smem;
-  float* red = reinterpret_cast<float*>(ring + (size_t)stages * tile_bytes);       // [kRed][8][16][4]
-  Cand* lists = reinterpret_cast<Cand*>(red + kRed * kConsumerWarps * kTileRows * 4);  // [M][top_k]
-  Cand* cbuf = lists + 4 * 64;                                                       // [M][kCandBuf]
-  uint64_t* full = reinterpret_cast<uint64_t*>(cbuf + 4 * kCandBuf);
+  float* red = reinterpret_cast<float*>(ring + (size_t)stages * tile_bytes);  // [kRed][8][16][4]
+  float* rsc = red + kRed * kConsumerWarps * kTileRows * 4;                    // [kRed][16] row scales
+  float* cvals = rsc + kRed * kTileRows;                                       // [M][n_cap]
+  uint64_t* full = reinterpret_cast<uint64_t*>(cvals + (size_t)M * ((n_cap + 1) & ~1));
   uint64_t* empty = full + stages;
   uint64_t* red_full = empty + stages;
   uint64_t* red_empty = red_full + kRed;
@@ -175,7 +275,6 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
   int* s_last = s_sigma + 5;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t ntiles = (V + kTileRows - 1) / kTileRows;
   const int64_t t_begin = ntiles * blockIdx.x / gridDim.x;
   const int64_t t_end = ntiles * (blockIdx.x + 1) / gridDim.x;
 
@@ -207,7 +306,6 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
       s_sigma[warp] = sigma;
     }
   }
-  for (int i = threadIdx.x; i < M * top_k; i += blockDim.x) lists[i] = Cand{-FLT_MAX, INT32_MAX};
   __syncthreads();
 
   // bounded wait shared by all roles: lane 0 polls, the warp agrees on the result
@@ -233,12 +331,16 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
       if (*(volatile int*)s_poison) continue;
       const int64_t r0 = t * kTileRows;
       const int nrows = (int)(V - r0 < kTileRows ? V - r0 : kTileRows);
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(nrows * row_bytes));
+      // the row scales travel with the tile: 16 B per 4 rows (a ragged last
+      // tile's 1..3 leftover scales are read from global by the epilogue)
+      const uint32_t sbytes = row_scale ? (uint32_t)(nrows & ~3) * 4u : 0u;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(nrows * row_bytes) + sbytes);
       __syncwarp();
+      uint8_t* stage = ring + (size_t)s * tile_bytes;
       if (lane < nrows)
-        bulk_g2s(ring + (size_t)s * tile_bytes + (size_t)lane * stride,
-                 reinterpret_cast<const uint8_t*>(w) + (size_t)(r0 + lane) * row_bytes, (uint32_t)row_bytes,
-                 &full[s], policy);
+        bulk_g2s(stage + (size_t)lane * stride, reinterpret_cast<const uint8_t*>(w) + (size_t)(r0 + lane) * row_bytes,
+                 (uint32_t)row_bytes, &full[s], policy);
+      if (lane == 16 && sbytes) bulk_g2s(stage + scale_off, row_scale + r0, sbytes, &full[s], policy);
       issued = it + 1;
     }
     // every issued copy must land before this CTA may exit
@@ -343,13 +445,18 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
 #pragma unroll
         for (int j = 1; j < T::kMmasPerSlice; ++j) d[q] += acc[j][q];
       }
+      // warp 0 also passes the tile's row scales on (the stage is recycled next)
+      float sc = 1.0f;
+      if (warp == 0 && lane < kTileRows && row_scale && ok)
+        sc = *reinterpret_cast<const float*>(ring + (size_t)s * tile_bytes + scale_off + lane * 4);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
 
-      // hand the partial sums to the epilogue warp
+      // hand the partial sums to the epilogue warp of this tile
       const int r = (int)(it % kRed);
       if (it >= kRed) wait_all(&red_empty[r], (uint32_t)(((it / kRed) & 1) ^ 1));
       float* rb = red + (size_t)r * kConsumerWarps * kTileRows * 4;
+      if (warp == 0 && lane < kTileRows) rsc[r * kTileRows + lane] = sc;
       if (tq < 2) {  // tokens 2tq, 2tq+1 (M <= 4)
         rb[(warp * kTileRows + g) * 4 + 2 * tq] = d[0];
         rb[(warp * kTileRows + g) * 4 + 2 * tq + 1] = d[1];
@@ -361,59 +468,57 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
     }
   } else {
     // ------------------------------ epilogue ------------------------------
-    int cnt[4] = {0, 0, 0, 0};
-    Cand thr[4] = {{-FLT_MAX, INT32_MAX}, {-FLT_MAX, INT32_MAX}, {-FLT_MAX, INT32_MAX}, {-FLT_MAX, INT32_MAX}};
-    // Per token: a buffer of candidates better than the current threshold (the
-    // k-th best kept so far).  Appends are one ballot; when the buffer could
-    // overflow, a selection pass keeps the best k and raises the threshold.
-    int64_t it = 0;
-    for (int64_t t = t_begin; t < t_end; ++t, ++it) {
+    // Two epilogue warps take alternate tiles: sum the 8 partials, apply the
+    // row scale and 2^-sigma_m, write logits when asked, and keep each value
+    // in shared memory for this CTA's top-k, taken after the stream.
+    const int ew = warp - kConsumerWarps - 1;  // 0 or 1
+    float inv[4];  // 2^-sigma_m
+#pragma unroll
+    for (int m = 0; m < 4; ++m) inv[m] = __uint_as_float((uint32_t)(127 - (m < M ? s_sigma[m] : 0)) << 23);
+    int64_t it = ew;
+    for (int64_t t = t_begin + ew; t < t_end; t += kEpilogueWarps, it += kEpilogueWarps) {
       const int r = (int)(it % kRed);
       const int64_t row = t * kTileRows + lane;
-      const bool valid = lane < kTileRows && row < V;
-      const float rs = (valid && row_scale) ? __ldg(row_scale + row) : 1.0f;
+      const int nrows = (int)(V - t * kTileRows < kTileRows ? V - t * kTileRows : kTileRows);
+      const bool valid = lane < nrows;
       const bool ok = wait_all(&red_full[r], (uint32_t)((it / kRed) & 1));
       const float* rb = red + (size_t)r * kConsumerWarps * kTileRows * 4;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      float rs = 1.0f;
       if (valid && ok) {
 #pragma unroll
         for (int ww = 0; ww < kConsumerWarps; ++ww) {
           const float4 p = *reinterpret_cast<const float4*>(rb + (ww * kTileRows + lane) * 4);
           acc[0] += p.x; acc[1] += p.y; acc[2] += p.z; acc[3] += p.w;
         }
+        if (row_scale) rs = lane < (nrows & ~3) ? rsc[r * kTileRows + lane] : __ldg(row_scale + row);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&red_empty[r]);
-      for (int m = 0; m < M; ++m) {
-        float v = -FLT_MAX;
-        if (valid) {
-          v = acc[m] * rs * __uint_as_float((uint32_t)(127 - s_sigma[m]) << 23);
-          if (logits) logits[(size_t)m * V + row] = v;
+      if (valid) {
+        const int local = (int)((t - t_begin) * kTileRows) + lane;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          if (m < M) {
+            const float v = acc[m] * rs * inv[m];
+            if (logits) logits[(size_t)m * V + row] = v;
+            cvals[(size_t)m * n_cap + local] = v;
+          }
         }
-        Cand* buf = cbuf + m * kCandBuf;
-        if (cnt[m] + kTileRows > kCandBuf) {
-          cnt[m] = select_top(buf, cnt[m], top_k, lane);
-          if (cnt[m] >= top_k) thr[m] = buf[top_k - 1];
-        }
-        const bool pass = valid && better(v, (int32_t)row, thr[m].v, thr[m].id);
-        const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-        if (pass) buf[cnt[m] + __popc(bal & ((1u << lane) - 1u))] = Cand{v, (int32_t)row};
-        cnt[m] += __popc(bal);
-        __syncwarp();
       }
     }
-    for (int m = 0; m < M; ++m) {
-      Cand* buf = cbuf + m * kCandBuf;
-      select_top(buf, cnt[m], top_k, lane);
-      for (int i = lane; i < top_k; i += 32) lists[m * top_k + i] = buf[i];
-    }
-    __syncwarp();
   }
 
-  // ------------------------- CTA lists -> global ---------------------------
-  __syncthreads();
-  Cand* my = cand + (size_t)blockIdx.x * M * top_k;
-  for (int i = threadIdx.x; i < M * top_k; i += blockDim.x) my[i] = lists[i];
+  // ------------------- this CTA's top-k, one warp per token -------------------
+  __syncthreads();  // every value is in shared memory and every copy has landed: the ring is free
+  if (warp < M) {
+    const int64_t row0 = t_begin * kTileRows;
+    const int n_local = (int)((t_end * kTileRows < V ? t_end * kTileRows : V) - row0);
+    warp_topk_rows(cvals + (size_t)warp * n_cap, n_local, row0, top_k, lane,
+                   reinterpret_cast<Cand*>(ring) + warp * kCandCap, cand + ((size_t)blockIdx.x * M + warp) * top_k);
+  }
+
+  // ------------------------- all lists written? ----------------------------
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -427,59 +532,67 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
   __threadfence();
 
   // ------------------------ last CTA: merge the lists ------------------------
-  // Per token: stage every CTA's sorted list in shared memory.  The k best of
-  // the lists' first entries are k real candidates, so the k-th best of them,
-  // L, is a lower bound on the global k-th best: only entries not worse than
-  // L can be in the top k.  Keep those (typically a few dozen) and select the
-  // top k of them with one warp.
-  Cand* stage = reinterpret_cast<Cand*>(smem);                 // [G * top_k]  (the ring is free now)
-  Cand* surv = stage + (size_t)gridDim.x * top_k;              // [kSurvivors]
-  Cand* wbuf = surv + kSurvivors;                              // [kCandBuf] selection buffer of warp 0
-  int* s_cnt = reinterpret_cast<int*>(wbuf + kCandBuf);
-  Cand* s_bound = reinterpret_cast<Cand*>(s_cnt + 4);
-  const int nl = (int)gridDim.x * top_k;
-  // warp 0's chunked selection: the best top_k of src[0..n) into wbuf[0..top_k)
-  auto select_from = [&](const Cand* src, int n, int stride) {
-    int cnt = 0, pos = 0;
-    do {
-      const int take = min(kCandBuf - cnt, n - pos);
-      for (int i = lane; i < take; i += 32) wbuf[cnt + i] = src[(size_t)(pos + i) * stride];
-      __syncwarp();
-      pos += take;
-      cnt = select_top(wbuf, cnt + take, top_k, lane);
-    } while (pos < n);
-  };
+  // Per token, over G sorted lists of k entries (G = gridDim.x):
+  //  1. L = the k-th best of the lists' first entries.  Those are k real
+  //     candidates, so the global k-th best is not worse than L, and only
+  //     entries not worse than L can be in the top k.
+  //  2. Only a list whose first entry is not worse than L can hold such an
+  //     entry: exactly k lists (all G when G < k), so at most k * k survivors.
+  //  3. Each survivor's rank is the number of survivors better than it; ranks
+  //     are distinct because ids are.  Ranks below k are the output.
+  // Every step is spread over the whole CTA; the ring is free by now.
+  const int G = (int)gridDim.x;
+  Cand* heads = reinterpret_cast<Cand*>(smem);                       // [G]
+  int* qual = reinterpret_cast<int*>(heads + G);                     // [G]
+  Cand* surv = reinterpret_cast<Cand*>(qual + ((G + 1) & ~1));       // [k * k]
+  int* s_cnt = reinterpret_cast<int*>(surv + (size_t)top_k * top_k); // [2]: lists, survivors
+  Cand* s_bound = reinterpret_cast<Cand*>(s_cnt + 2);
   for (int m = 0; m < M; ++m) {
-    for (int i = threadIdx.x; i < nl; i += blockDim.x) {
-      const int cc = i / top_k, j = i - cc * top_k;
-      const Cand* src = cand + ((size_t)cc * M + m) * top_k + j;
-      stage[i] = Cand{__ldcg(&src->v), __ldcg(&src->id)};
+    for (int c = threadIdx.x; c < G; c += blockDim.x) {
+      const Cand* src = cand + ((size_t)c * M + m) * top_k;
+      heads[c] = Cand{__ldcg(&src->v), __ldcg(&src->id)};
     }
-    if (threadIdx.x == 0) *s_cnt = 0;
+    if (threadIdx.x == 0) {
+      s_cnt[0] = s_cnt[1] = 0;
+      *s_bound = Cand{-FLT_MAX, INT32_MAX};  // no bound when G < k
+    }
     __syncthreads();
-    if (warp == 0) {
-      select_from(stage, (int)gridDim.x, top_k);  // the lists' first entries
-      if (lane == 0) *s_bound = wbuf[top_k - 1];  // an empty slot (worst) when fewer than top_k lists
+    for (int c = threadIdx.x; c < G; c += blockDim.x) {
+      const Cand h = heads[c];
+      int rank = 0;
+      for (int o = 0; o < G; ++o) rank += better(heads[o].v, heads[o].id, h.v, h.id);
+      if (rank == top_k - 1) *s_bound = h;
     }
     __syncthreads();
     const Cand L = *s_bound;
-    for (int i = threadIdx.x; i < nl; i += blockDim.x) {
-      const Cand e = stage[i];
-      if (!better(L.v, L.id, e.v, e.id)) {  // e is L or better
-        const int pos = atomicAdd(s_cnt, 1);
-        if (pos < kSurvivors) surv[pos] = e;
+    for (int c = threadIdx.x; c < G; c += blockDim.x)
+      if (!better(L.v, L.id, heads[c].v, heads[c].id)) qual[atomicAdd(&s_cnt[0], 1)] = c;
+    __syncthreads();
+    const int nq = s_cnt[0];
+    for (int i = threadIdx.x; i < nq * top_k; i += blockDim.x) {
+      const int c = qual[i / top_k], j = i - (i / top_k) * top_k;
+      const Cand* src = cand + ((size_t)c * M + m) * top_k + j;
+      const Cand e{__ldcg(&src->v), __ldcg(&src->id)};
+      if (e.id != INT32_MAX && !better(L.v, L.id, e.v, e.id)) {
+        const int pos = atomicAdd(&s_cnt[1], 1);
+        if (pos < top_k * top_k) surv[pos] = e;  // never false: at most k lists hold survivors
       }
     }
     __syncthreads();
-    if (warp == 0) {
-      const int n = *s_cnt;
-      // more survivors than the buffer holds (heavy ties): select from all staged entries instead
-      if (n <= kSurvivors) select_from(surv, n, 1);
-      else select_from(stage, nl, 1);
-      for (int i = lane; i < top_k; i += 32) {
-        out_ids[m * top_k + i] = wbuf[i].id;
-        out_vals[m * top_k + i] = wbuf[i].v;
+    const int ns = min(s_cnt[1], top_k * top_k);
+    for (int i = threadIdx.x; i < ns; i += blockDim.x) {
+      const Cand e = surv[i];
+      int rank = 0;
+      for (int o = 0; o < ns; ++o) rank += better(surv[o].v, surv[o].id, e.v, e.id);
+      if (rank < top_k) {
+        out_ids[m * top_k + rank] = e.id;
+        out_vals[m * top_k + rank] = e.v;
       }
+    }
+    // fewer admissible candidates than k (only when logits are NaN or -inf): pad
+    for (int j = ns + threadIdx.x; j < top_k; j += blockDim.x) {
+      out_ids[m * top_k + j] = INT32_MAX;
+      out_vals[m * top_k + j] = -FLT_MAX;
     }
     __syncthreads();
   }
@@ -492,25 +605,34 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
 // host side
 // ----------------------------------------------------------------------------
 
-size_t lmhead_smem_bytes(int H, int elem_bytes, int stages);
-
-int lmhead_stages(int H, int elem_bytes) {
-  int stages = 4;
-  while (stages > 2 && lmhead_smem_bytes(H, elem_bytes, stages) > kMaxSmem) --stages;
-  return stages;
+static size_t merge_smem_bytes(int grid, int top_k) {
+  return (size_t)grid * sizeof(Cand) + (size_t)((grid + 1) & ~1) * sizeof(int) +
+         (size_t)top_k * top_k * sizeof(Cand) + 2 * sizeof(int) + sizeof(Cand);
 }
 
-size_t lmhead_merge_smem_bytes(int grid, int top_k) {
-  return ((size_t)grid * top_k + kSurvivors + kCandBuf) * sizeof(Cand) + 4 * sizeof(int) + sizeof(Cand);
-}
-
-size_t lmhead_smem_bytes(int H, int elem_bytes, int stages) {
-  const int stride = padded_stride(H * elem_bytes);
-  size_t bytes = (size_t)stages * kTileRows * stride;
-  bytes += 4 * kConsumerWarps * kTileRows * 4 * sizeof(float);  // kRed reduce buffers
-  bytes += 4 * 64 * sizeof(Cand) + 4 * kCandBuf * sizeof(Cand);
+static size_t stream_smem_bytes(int H, int elem_bytes, int stages, int M, int64_t V, int grid) {
+  const int64_t ntiles = (V + kTileRows - 1) / kTileRows;
+  const int64_t n_cap = (ntiles + grid - 1) / grid * kTileRows;
+  size_t bytes = (size_t)stages * stage_bytes(H * elem_bytes);
+  bytes += kRed * kConsumerWarps * kTileRows * 4 * sizeof(float);  // reduce buffers
+  bytes += kRed * kTileRows * sizeof(float);                        // row scales
+  bytes += (size_t)M * ((n_cap + 1) & ~1) * sizeof(float);          // this CTA's logits
   bytes += (2 * stages + 2 * 4) * sizeof(uint64_t) + 8 * sizeof(int);
   return bytes;
+}
+
+bool lmhead_plan(int H, int elem_bytes, int M, int top_k, int64_t V, int grid, int* stages, size_t* smem) {
+  for (int st = 4; st >= 2; --st) {
+    size_t b = stream_smem_bytes(H, elem_bytes, st, M, V, grid);
+    const size_t merge = merge_smem_bytes(grid, top_k);
+    if (merge > b) b = merge;  // the final merge reuses the whole dynamic buffer
+    if (b <= kMaxSmem) {
+      *stages = st;
+      *smem = b;
+      return true;
+    }
+  }
+  return false;
 }
 
 size_t lmhead_cand_bytes(int grid, int M, int top_k) { return (size_t)grid * M * top_k * sizeof(Cand); }
@@ -519,13 +641,11 @@ template <typename W, int kSlices>
 static cudaError_t launch_head_t(const uint16_t* x, const W* w, const float* s, int64_t V, int H, int M, int top_k,
                                  float* logits, int32_t* ids, float* vals, WsHeader* hdr, void* cand, int grid,
                                  cudaStream_t st) {
-  const int stages = lmhead_stages(H, (int)sizeof(W));
-  size_t smem = lmhead_smem_bytes(H, (int)sizeof(W), stages);
-  const size_t merge = lmhead_merge_smem_bytes(grid, top_k);
-  if (merge > smem) smem = merge;  // the final merge reuses the whole dynamic buffer
-  if (smem > kMaxSmem) return cudaErrorInvalidConfiguration;
+  int stages = 0;
+  size_t smem = 0;
+  if (!lmhead_plan(H, (int)sizeof(W), M, top_k, V, grid, &stages, &smem)) return cudaErrorInvalidConfiguration;
   auto kern = lmhead_topk_kernel<W, kSlices>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem_optin<lmhead_topk_kernel<W, kSlices>>();
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, st>>>(x, w, s, V, H, M, top_k, stages, logits, ids, vals, hdr,
                                      reinterpret_cast<Cand*>(cand));

@@ -13,13 +13,13 @@
 
 #include "../../include/moe_gemv.h"
 #include "common.cuh"
+#include "device_cache.h"
 #include "lmhead.h"
 
 namespace {
 
 constexpr size_t kScratchBytes = MOE_LMHEAD_NOALLOC_SCRATCH_BYTES;
 constexpr size_t kHeaderBytes = sizeof(moe::WsHeader);
-constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) uint8_t g_lmhead_scratch[kScratchBytes];
 
@@ -27,13 +27,13 @@ __device__ __align__(256) uint8_t g_lmhead_scratch[kScratchBytes];
 // host code the array's name is only a host-side stand-in, never a device
 // address, so it must not be passed to a kernel.
 std::mutex g_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
+void* g_scratch_ptr[moe::kMaxDevices] = {};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 moe_status scratch_for_current_device(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= moe::kMaxDevices) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
@@ -63,11 +63,13 @@ extern "C" moe_status lmhead_decode_noalloc(const uint16_t* hidden_bf16, const m
 
   // one CTA per SM, as lmhead_decode launches; its candidate lists must fit
   int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::current_device_sms(&dev, &sms) != cudaSuccess) return MOE_ERR_CUDA;
   const int64_t ntiles = (V + 15) / 16;
   const int grid = (int)(sms < ntiles ? sms : ntiles);
   if (kHeaderBytes + moe::lmhead_cand_bytes(grid, M, top_k) > kScratchBytes) return MOE_ERR_WORKSPACE;
+  int stages = 0;
+  size_t smem = 0;
+  if (!moe::lmhead_plan((int)H, 1, M, top_k, V, grid, &stages, &smem)) return MOE_ERR_UNSUPPORTED_SHAPE;
 
   void* scratch = nullptr;
   const moe_status st = scratch_for_current_device(&scratch);

@@ -1,4 +1,4 @@
-// moe.h -- internal interface of the MoE-layer kernels (moe_kernels.cu).
+// moe.h -- internal interface of the MoE-layer kernel (moe_fused.cu).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -20,51 +20,34 @@ struct MoeBank {
 };
 
 // Views into the caller's workspace.  Token-indexed arrays use a fixed stride
-// of 4 tokens; slot arrays hold at most kMaxSlots = 4 * 8 + 1 entries.
+// of 4 tokens; slot arrays hold at most kMaxSlots = 4 * 8 + 1 entries.  Every
+// array is fully written before it is read in each call, and the header's
+// barrier word returns to its starting value, so nothing needs resetting
+// between calls.
 struct MoeWs {
   static constexpr int kMaxSlots = 4 * 8 + 1;
   WsHeader* hdr;
   float* logits;        // [M][E]
-  int32_t* nslots;      // number of live slots
-  int32_t* slot_expert; // [kMaxSlots]: -1 for the shared expert
-  uint32_t* slot_mask;  // [kMaxSlots]: bit m set if token m uses the slot
-  float* slot_w;        // [kMaxSlots][4]: combine weight of the slot for token m
-  float* h;             // [kMaxSlots][4][I]
-  float* ypart;         // [kMaxSlots][4][H]
-  uint32_t* slot_ready; // [kMaxSlots]: rows of h written (reset by the kernel's last CTA)
-  uint32_t* hmax;       // [kMaxSlots][4]: max |h| as fp32 bits (reset likewise)
-  uint32_t* tile_ticket;// [H/32]: slots finished per 32-row output tile (self-resetting)
+  float* h;             // [kMaxSlots][4][I]: silu(gate) * up per slot and token
+  float* ypart;         // [kMaxSlots][4][H]: down(h) per slot and token, before the weighted combine
 
   static size_t align(size_t v) { return (v + 255) & ~size_t(255); }
   static size_t bytes(int M, int top_k, int E, int H, int I) {
     (void)M; (void)top_k;
     size_t b = align(sizeof(WsHeader));
     b += align((size_t)4 * E * sizeof(float));
-    b += align(64);
-    b += align(kMaxSlots * sizeof(int32_t));
-    b += align(kMaxSlots * sizeof(uint32_t));
-    b += align((size_t)kMaxSlots * 4 * sizeof(float));
     b += align((size_t)kMaxSlots * 4 * I * sizeof(float));
     b += align((size_t)kMaxSlots * 4 * H * sizeof(float));
-    b += align(kMaxSlots * sizeof(uint32_t));
-    b += align((size_t)kMaxSlots * 4 * sizeof(uint32_t));
-    b += align((size_t)(H / 32 + 1) * sizeof(uint32_t));
     return b;
   }
   static MoeWs carve(void* base, int E, int H, int I) {
+    (void)H;
     uint8_t* p = static_cast<uint8_t*>(base);
     MoeWs w;
     w.hdr = reinterpret_cast<WsHeader*>(p); p += align(sizeof(WsHeader));
     w.logits = reinterpret_cast<float*>(p); p += align((size_t)4 * E * sizeof(float));
-    w.nslots = reinterpret_cast<int32_t*>(p); p += align(64);
-    w.slot_expert = reinterpret_cast<int32_t*>(p); p += align(kMaxSlots * sizeof(int32_t));
-    w.slot_mask = reinterpret_cast<uint32_t*>(p); p += align(kMaxSlots * sizeof(uint32_t));
-    w.slot_w = reinterpret_cast<float*>(p); p += align((size_t)kMaxSlots * 4 * sizeof(float));
     w.h = reinterpret_cast<float*>(p); p += align((size_t)kMaxSlots * 4 * I * sizeof(float));
-    w.ypart = reinterpret_cast<float*>(p); p += align((size_t)kMaxSlots * 4 * H * sizeof(float));
-    w.slot_ready = reinterpret_cast<uint32_t*>(p); p += align(kMaxSlots * sizeof(uint32_t));
-    w.hmax = reinterpret_cast<uint32_t*>(p); p += align((size_t)kMaxSlots * 4 * sizeof(uint32_t));
-    w.tile_ticket = reinterpret_cast<uint32_t*>(p);
+    w.ypart = reinterpret_cast<float*>(p);
     return w;
   }
 };

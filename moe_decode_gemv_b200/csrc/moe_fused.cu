@@ -11,10 +11,10 @@
 // HBM busy from the first microsecond:
 //
 //  * One CTA per SM (cooperative launch: all CTAs are resident, which the
-//    grid barrier and the readiness counters below rely on).  A producer warp
-//    streams every weight tile the CTA will need into a ring of shared-memory
-//    stages with bulk copies (cp.async.bulk, no multicast); eight consumer
-//    warps compute.
+//    grid barriers below rely on).  A producer warp streams every weight tile
+//    the CTA will need into a ring of shared-memory stages with bulk copies
+//    (cp.async.bulk, no multicast); eight consumer warps compute; two
+//    epilogue warps finish each item and own everything that leaves the CTA.
 //  * Phase 0: each CTA scores its share of the router rows (fp32 weights,
 //    bf16 activations, fp32 sums) and arrives at a split grid barrier.  The
 //    shared expert needs no routing, so its tiles are loaded and computed
@@ -23,24 +23,29 @@
 //    same slot table (slot 0 = shared expert, then the distinct routed
 //    experts in first-appearance order), so each distinct expert is streamed
 //    once however many tokens chose it.  Items of 8 gate rows + 8 up rows of
-//    one slot form one 16-row MMA tile; h = silu(g) * u is written in fp32 and
-//    a per-slot counter is bumped.
-//  * Phase 2: items of 32 output rows of one slot's down matrix wait on that
-//    slot's counter (bounded), then multiply by h.  The last CTA to finish a
-//    32-row tile sums the slot partials in slot order: no float atomics, the
-//    result is reproducible run to run.
+//    one slot form one 16-row MMA tile; h = silu(g) * u is written in fp32.
+//  * A grid barrier publishes h.  No fence or atomic sits on the per-item
+//    path: the producer streams the down tiles meanwhile.
+//  * Phase 2: items of 32 output rows of one slot's down matrix multiply by h
+//    and write per-slot partial outputs.  After one more grid barrier each
+//    CTA sums, for the 32-row tiles it owns, the slot partials in slot order:
+//    no float atomics, the result is reproducible run to run.
 //
-// Arithmetic: mma.sync m16n8k16 f16 x f16 -> fp32.  E2M1 codes widen to f16
-// exactly (cvt.rn.f16x2.e2m1x2).  bf16 activations become f16 exactly after a
-// per-token power-of-two scale.  h (fp32) enters the down GEMV as an f16
-// hi/lo pair, which carries 22 of fp32's 24 significand bits.  Each MMA
-// spans one 32-element block (two k16 steps), so its fp32 result is scaled
-// by that block's E8M0 scale before it joins the running fp32 sum.
+// Arithmetic: mma.sync m16n8k32 E4M3 x E4M3 -> fp32, one MMA per 32-element
+// MX block, so that its fp32 result is scaled by that block's E8M0 scale
+// before it joins the running fp32 sum.  The weights need no conversion
+// instruction: an E2M1 code becomes the E4M3 code of its value times 2^-6 by
+// moving bits (e2m1x8_*_to_e4m3x4).  Activations are scaled by a per-token
+// power of two that puts their largest magnitude in [2^7, 2^8); bf16 x is
+// then carried exactly by two E4M3 parts (two MMAs per block).  h is scaled
+// per 32-element block and token (largest magnitude into [2^7, 2^8)) and
+// carried by three E4M3 parts (12 significant bits, three MMAs per block).
 #include <cuda_runtime.h>
 
 #include <cfloat>
 
 #include "common.cuh"
+#include "device_cache.h"
 #include "moe.h"
 
 namespace moe {
@@ -58,15 +63,7 @@ constexpr int kMaxDnBlocksPerWarp = 4;     // I <= 4 * 8 * 32 = 1024
 // launcher picks the smallest that fits.  The down GEMV's fragments are
 // rebuilt per item and sized for the largest case.
 constexpr int kGuBuckets[] = {1, 2, 4, 8, 10, 16};
-
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
+constexpr int kHParts = 3;  // E4M3 parts carrying h into the down GEMV
 
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
@@ -76,40 +73,173 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   return v;
 }
 
-// Fire-and-forget atomics with release semantics: writes ordered before them
-// (in this thread, or in lanes synchronised with it by __syncwarp) become
-// visible to a reader that acquires the counter.
-__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void red_max(uint32_t* p, uint32_t v) {
-  asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-// One round trip that both publishes this thread's (and its warp's) earlier
-// writes and makes other CTAs' published writes visible.
-__device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
-// f32 pair -> f16x2 (lo in the low half)
-__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
 __device__ __forceinline__ int pow2_sigma(float amax) {
-  // sigma such that amax * 2^sigma lies in [2^14, 2^15)
+  // sigma such that amax * 2^sigma lies in [2^7, 2^8): the largest value sits
+  // at the top of E4M3's normal range (max 448)
   if (!(amax > 0.f)) return 0;
   const uint32_t b = __float_as_uint(amax);
   const int e = (int)((b >> 23) & 0xffu);
   const int fl = e ? e - 127 : (31 - __clz(b & 0x7fffffu)) - 149;
-  int s = 14 - fl;
+  int s = 7 - fl;
   return s > 126 ? 126 : (s < -126 ? -126 : s);
 }
 
 __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
+
+// ---- routing: top-8 of up to 1,024 logits in one warp ----
+// (value, expert) pairs under `better`: larger value first, lower id on ties.
+struct VI {
+  float v;
+  int32_t i;
+};
+
+// Leave the better of the two in a.
+__device__ __forceinline__ void cas(VI& a, VI& b) {
+  const bool sw = better(b.v, b.i, a.v, a.i);
+  const VI t = a;
+  a = sw ? b : a;
+  b = sw ? t : b;
+}
+
+// Sorting network for 8 entries, best first (19 comparators, depth 6).
+__device__ __forceinline__ void sort8(VI (&a)[8]) {
+  cas(a[0], a[2]); cas(a[1], a[3]); cas(a[4], a[6]); cas(a[5], a[7]);
+  cas(a[0], a[4]); cas(a[1], a[5]); cas(a[2], a[6]); cas(a[3], a[7]);
+  cas(a[0], a[1]); cas(a[2], a[3]); cas(a[4], a[5]); cas(a[6], a[7]);
+  cas(a[2], a[4]); cas(a[3], a[5]);
+  cas(a[1], a[4]); cas(a[3], a[6]);
+  cas(a[1], a[2]); cas(a[3], a[4]); cas(a[5], a[6]);
+}
+
+// R (sorted) <- the best 8 of R and S (both sorted), sorted.  The pairwise
+// better of R[j] and S[7 - j] is exactly that set, in bitonic order; a
+// bitonic sorter of 8 (12 comparators) orders it.
+__device__ __forceinline__ void merge8(VI (&R)[8], const VI (&S)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const VI o = S[7 - j];
+    if (better(o.v, o.i, R[j].v, R[j].i)) R[j] = o;
+  }
+  cas(R[0], R[4]); cas(R[1], R[5]); cas(R[2], R[6]); cas(R[3], R[7]);
+  cas(R[0], R[2]); cas(R[1], R[3]); cas(R[4], R[6]); cas(R[5], R[7]);
+  cas(R[0], R[1]); cas(R[2], R[3]); cas(R[4], R[5]); cas(R[6], R[7]);
+}
+
+// The best 8 of logits[0..E) (E <= 1024), sorted, in every lane of the warp.
+// Logits that are NaN or -inf count as -FLT_MAX, so that every real expert
+// ranks above the padding entries (-FLT_MAX, INT32_MAX): with E >= 8 the
+// result holds only experts in [0, E).
+__device__ __forceinline__ void warp_top8(const float* logits, int E, int lane, VI (&R)[8]) {
+  float lv[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int e = lane + 32 * i;
+    const float v = e < E ? __ldcg(logits + e) : -FLT_MAX;
+    lv[i] = v > -FLT_MAX ? v : -FLT_MAX;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) R[j] = VI{-FLT_MAX, INT32_MAX};
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {  // this lane's values, 8 at a time
+    if (ch * 256 < E) {
+      VI S[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * (8 * ch + j);
+        S[j] = e < E ? VI{lv[8 * ch + j], e} : VI{-FLT_MAX, INT32_MAX};
+      }
+      sort8(S);
+      merge8(R, S);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {  // butterfly: both partners end with the same list
+    VI P[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      P[j].v = __shfl_xor_sync(0xffffffffu, R[j].v, o);
+      P[j].i = __shfl_xor_sync(0xffffffffu, R[j].i, o);
+    }
+    merge8(R, P);
+  }
+}
+
+// Top-k (k <= 8) of one token's logits[0..E) by one warp, with ids and
+// values in rank order written to ids[0..k) and vals[0..k) (shared memory).
+// A filter first: the k-th best of the 32 lanes' own best entries, L, is a
+// lower bound on the k-th best overall (those are k real entries), so only
+// entries not worse than L can be selected -- typically a dozen.  They are
+// ranked by counting.  With more than 64 of them (heavy ties) the sorting
+// network above ranks all E entries instead.  Logits that are NaN or -inf
+// count as -FLT_MAX; ties go to the lower expert id.
+__device__ __forceinline__ void warp_route(const float* logits, int E, int k, int lane, float* cv, int32_t* ci,
+                                           int32_t* ids, float* vals) {
+  float lv[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int e = lane + 32 * i;
+    const float v = e < E ? __ldcg(logits + e) : -FLT_MAX;
+    lv[i] = v > -FLT_MAX ? v : -FLT_MAX;
+  }
+  float mv = -FLT_MAX;
+  int32_t mi = INT32_MAX;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E && better(lv[i], e, mv, mi)) { mv = lv[i]; mi = e; }
+  }
+  int rank = 0;  // of this lane's best among the 32 lanes' bests
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float ov = __shfl_sync(0xffffffffu, mv, j);
+    const int32_t oi = __shfl_sync(0xffffffffu, mi, j);
+    rank += better(ov, oi, mv, mi);
+  }
+  // padding lanes (E < 32) tie among themselves but rank after all real ones,
+  // and E >= k, so exactly one lane has rank k - 1
+  const uint32_t sel = __ballot_sync(0xffffffffu, rank == k - 1);
+  const int src = sel ? __ffs(sel) - 1 : 0;
+  const float Lv = sel ? __shfl_sync(0xffffffffu, mv, src) : -FLT_MAX;
+  const int32_t Li = sel ? __shfl_sync(0xffffffffu, mi, src) : INT32_MAX;
+  int cnt = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int e = lane + 32 * i;
+    cnt += (e < E && !better(Lv, Li, lv[i], e)) ? 1 : 0;
+  }
+  int off = cnt;  // inclusive prefix sum over lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, off, o);
+    if (lane >= o) off += t;
+  }
+  const int n = __shfl_sync(0xffffffffu, off, 31);
+  off -= cnt;
+  if (n <= 64) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !better(Lv, Li, lv[i], e)) { cv[off] = lv[i]; ci[off] = e; ++off; }
+    }
+    __syncwarp();
+    for (int q = lane; q < n; q += 32) {
+      const float qv = cv[q];
+      const int32_t qi = ci[q];
+      int r = 0;
+      for (int o = 0; o < n; ++o) r += better(cv[o], ci[o], qv, qi);
+      if (r < k) { ids[r] = qi; vals[r] = qv; }
+    }
+  } else {
+    VI R[8];
+    warp_top8(logits, E, lane, R);
+    if (lane == 0) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < k) { ids[r] = R[r].i; vals[r] = R[r].v; }
+    }
+  }
+  __syncwarp();
+}
 
 struct FusedArgs {
   const uint16_t* x;
@@ -149,7 +279,7 @@ struct Geometry {
 };
 
 // Shared memory outside the ring.
-constexpr int kRed = 4;                    // partial-sum buffers between consumers and the epilogue warp
+constexpr int kRed = 4;                    // partial-sum buffers between consumers and the epilogue warps
 constexpr int kEpi = kCons + 1;            // first epilogue warp
 constexpr int kNumEpi = 2;                 // epilogue warps; item i goes to epilogue warp i % kNumEpi
 constexpr int kThreadsAll = (kCons + 1 + kNumEpi) * 32;
@@ -160,26 +290,45 @@ struct SmemCtl {
   uint64_t empty[kStages];
   uint64_t red_full[kRed];
   uint64_t red_empty[kRed];
-  uint64_t routed;                         // slot table ready (producer and epilogue wait on it)
+  uint64_t routed;                         // slot table ready (producer and epilogue warps wait on it)
+  uint64_t h_ready;                        // every CTA's h written (consumers wait on it)
   alignas(16) float red[kRed][kCons][32][8];  // per-item partials (float4 access)
   float logit_part[kCons][4];              // router: half-row partial sums
   int32_t ids[4][8];
   float wts[4][8];
+  float topv[4][8];
+  float cand_v[4][64];                     // routing candidates, per token
+  int32_t cand_i[4][64];
   int32_t slot_expert[MoeWs::kMaxSlots];
   uint32_t slot_mask[MoeWs::kMaxSlots];
   float slot_w[MoeWs::kMaxSlots][4];
   int sigma_x[4];
   int nslots;
   int poison;
-  int last;
 };
 
 __device__ __forceinline__ void consumer_bar_sync() {
   asm volatile("bar.sync 1, %0;" ::"r"(kCons * 32) : "memory");
 }
+__device__ __forceinline__ void epilogue_bar_sync() {
+  asm volatile("bar.sync 2, %0;" ::"r"(kNumEpi * 32) : "memory");
+}
+
+// Grid barrier on one word (all CTAs are resident: cooperative launch).  The
+// first CTA adds 2^31 - (G - 1), the others 1, so the top bit flips exactly
+// when all G have arrived and the low bits return to where they were: the
+// same word serves every barrier of every call.  Arrival publishes the
+// caller's earlier writes (fence first); the wait is bounded.
+__device__ __forceinline__ uint32_t grid_arrive(uint32_t* word, int c, int G) {
+  __threadfence();
+  return atomicAdd(word, c == 0 ? 0x80000000u - (uint32_t)(G - 1) : 1u);
+}
+__device__ __forceinline__ bool grid_wait(uint32_t* word, uint32_t old) {
+  return bounded_spin([&] { return ((ld_acquire(word) ^ old) & 0x80000000u) != 0u; });
+}
 
 // The work of one CTA, enumerated identically by the producer, the consumers
-// and the epilogue warp: phase-1 items are global items c, c+G, ... of
+// and the epilogue warps: phase-1 items are global items c, c+G, ... of
 // S * n_chunks (the first n_chunks belong to the shared expert, slot 0), then
 // phase-2 items c, c+G, ... of S * n_tiles.
 struct ItemIter {
@@ -201,6 +350,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
   const int M = a.M, H = a.H, I = a.I, E = a.E;
   const MoeWs ws = a.ws;
   const ItemIter items{c, G, geo.n_chunks, geo.n_tiles};
+  uint32_t* bar_word = &ws.hdr->barrier;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -212,6 +362,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       mbar_init(&C.red_empty[r], 1);
     }
     mbar_init(&C.routed, 1);
+    mbar_init(&C.h_ready, 1);
     fence_mbar_init();
     C.poison = 0;
   }
@@ -223,19 +374,26 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
   }
   __syncthreads();
 
-  auto bounded_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    bool ok = !*(volatile int*)&C.poison;
-    if (ok && lane == 0) ok = mbar_wait(bar, parity);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok && lane == 0 && !*(volatile int*)&C.poison) {
+  auto poisoned = [&]() -> bool { return *(volatile int*)&C.poison != 0; };
+  auto fail = [&]() {  // the first wait of this CTA that ran out
+    if (!poisoned()) {
       report(ws.hdr, MOE_ERR_TIMEOUT);
       atomicExch(&C.poison, 1);
     }
+  };
+  // bounded wait on an mbarrier phase: lane 0 polls, the warp agrees
+  auto bounded_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    bool ok = !poisoned();
+    if (ok && lane == 0) ok = mbar_wait(bar, parity);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok && lane == 0) fail();
     return ok;
   };
 
   if (warp == kProd) {
     // ============================== producer ==============================
+    // Streams every weight tile of this CTA's items, phase 1 then phase 2:
+    // no tile depends on h, so the down tiles arrive while phase 1 finishes.
     const uint64_t policy = l2_evict_first_policy();
     int it = 0, issued = 0;
     auto issue = [&](int s_slot, bool phase1, int row0) {
@@ -243,7 +401,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       const uint32_t ph = (uint32_t)((it / kStages) & 1);
       bool ok = true;
       if (it >= kStages) ok = bounded_wait(&C.empty[st], ph ^ 1u);
-      if (ok && !*(volatile int*)&C.poison) {
+      if (ok && !poisoned()) {
         uint8_t* dst = ring + (size_t)st * geo.stage_bytes;
         const int ex = s_slot == 0 ? -1 : C.slot_expert[s_slot];
         const MoeBank& b = ex < 0 ? a.shared : a.bank;
@@ -299,16 +457,14 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     }
   } else if (warp >= kEpi) {
     // ============================== epilogue ==============================
-    // Owns everything that leaves the CTA: h and its max, the readiness
-    // counters, the partial outputs, the tile tickets and the combine.  Items
-    // alternate between the epilogue warps so that one item's memory round
-    // trips overlap the next item's.
+    // Owns everything that leaves the CTA: h, the partial outputs, the two
+    // grid barriers that publish them, and the final combine.  Items
+    // alternate between the epilogue warps so that one item's memory traffic
+    // overlaps the next item's.  No fence or atomic sits on the per-item path.
     const int ew = warp - kEpi;
     const int g = lane >> 2, tq = lane & 3;
     int idx = 0;  // item index, counted by every epilogue warp
-    auto take = [&]() -> bool {
-      return bounded_wait(&C.red_full[idx % kRed], (uint32_t)((idx / kRed) & 1));
-    };
+    auto take = [&]() -> bool { return bounded_wait(&C.red_full[idx % kRed], (uint32_t)((idx / kRed) & 1)); };
     auto give = [&]() {
       __syncwarp();
       if (lane == 0) mbar_arrive(&C.red_empty[idx % kRed]);
@@ -327,23 +483,14 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const int m = 2 * tq + q;
-        float hv = 0.f;
         if (ok && tq < 2 && m < M && (mask >> m & 1u)) {
-          const float inv = exp2i(-C.sigma_x[m]);
+          const float inv = exp2i(6 - C.sigma_x[m]);  // undo 2^sigma and the E4M3 weights' 2^-6
           const float gg = gs[q] * inv, uu = us[q] * inv;
-          hv = gg / (1.0f + expf(-gg)) * uu;
-          ws.h[((size_t)slot * 4 + m) * I + row0 + g] = hv;
+          ws.h[((size_t)slot * 4 + m) * I + row0 + g] = gg / (1.0f + expf(-gg)) * uu;
         }
-        float mx = fabsf(hv);  // max |h| over the 8 rows (lanes with equal tq)
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        if (g == 0 && tq < 2 && m < M && mx > 0.f) red_max(&ws.hmax[slot * 4 + m], __float_as_uint(mx));
       }
-      __syncwarp();
-      if (lane == 0) red_release_add(&ws.slot_ready[slot], (uint32_t)kGuRows);
     };
-    auto down_out = [&](int slot, int row0, int S) {
+    auto down_out = [&](int slot, int row0) {
       const bool ok = take();
       const float* rb = &C.red[idx % kRed][0][0][0];
       float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -360,33 +507,23 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       for (int q = 0; q < 2; ++q) {
         const int m = 2 * tq + q;
         if (ok && tq < 2 && m < M && (mask >> m & 1u)) {
-          const float inv = exp2i(-pow2_sigma(__uint_as_float(__ldcg(&ws.hmax[slot * 4 + m]))));
           float* yp = ws.ypart + ((size_t)slot * 4 + m) * H + row0;
-          yp[g] = s8[q] * inv;            // row g of the first 16
-          yp[g + 8] = s8[2 + q] * inv;    // row g + 8
-          yp[16 + g] = s8[4 + q] * inv;   // second 16 rows
-          yp[24 + g] = s8[6 + q] * inv;
+          yp[g] = s8[q];            // row g of the first 16
+          yp[g + 8] = s8[2 + q];    // row g + 8
+          yp[16 + g] = s8[4 + q];   // second 16 rows
+          yp[24 + g] = s8[6 + q];
         }
       }
-      __syncwarp();
-      // the last CTA to finish this 32-row tile combines the slots in order
-      const int tile = row0 / kDnRows;
-      uint32_t tk = 0;
-      if (lane == 0) tk = atom_acq_rel_add(&ws.tile_ticket[tile], 1u);
-      tk = __shfl_sync(0xffffffffu, tk, 0);
-      __syncwarp();
-      if (tk == (uint32_t)(S - 1)) {
-        const int row = row0 + lane;
-        for (int m = 0; m < M; ++m) {
-          float y = 0.f;
-          for (int s2 = 0; s2 < S; ++s2) {
-            const uint32_t mk = s2 == 0 ? 0xfu : C.slot_mask[s2];
-            if (mk >> m & 1u) y = fmaf(C.slot_w[s2][m], __ldcg(&ws.ypart[((size_t)s2 * 4 + m) * H + row]), y);
-          }
-          a.out[(size_t)m * H + row] = y;
-        }
-        if (lane == 0) ws.tile_ticket[tile] = 0u;
+    };
+    // grid barrier of the epilogue warps: both finish their writes, one thread
+    // publishes and waits, both go on
+    auto epilogue_grid_barrier = [&]() {
+      epilogue_bar_sync();
+      if (ew == 0 && lane == 0) {
+        const uint32_t old = grid_arrive(bar_word, c, G);
+        if (!poisoned() && !grid_wait(bar_word, old)) fail();
       }
+      epilogue_bar_sync();
     };
     const int ns = items.n_shared();
     int S = 0, n1 = ns, n2 = 0;
@@ -401,10 +538,30 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       const int q = c + j * G;
       gateup_out(q / geo.n_chunks, (q % geo.n_chunks) * kGuRows);
     }
+    // h of every CTA is written: release the consumers into phase 2
+    epilogue_grid_barrier();
+    if (ew == 0 && lane == 0) mbar_arrive(&C.h_ready);
     for (int j = 0; j < n2; ++j, ++idx) {
       if (idx % kNumEpi != ew) continue;
       const int q = c + j * G;
-      down_out(q / geo.n_tiles, (q % geo.n_tiles) * kDnRows, S);
+      down_out(q / geo.n_tiles, (q % geo.n_tiles) * kDnRows);
+    }
+    // every slot's partial outputs are written: combine the 32-row tiles this
+    // CTA owns (tile t belongs to CTA t mod G), slots in order -- no float
+    // atomics, the same result on every run
+    epilogue_grid_barrier();
+    if (!poisoned()) {
+      for (int t = c + ew * G; t < geo.n_tiles; t += kNumEpi * G) {
+        const int row = t * kDnRows + lane;
+        for (int m = 0; m < M; ++m) {
+          float y = 0.f;
+          for (int s2 = 0; s2 < S; ++s2) {
+            const uint32_t mk = s2 == 0 ? 0xfu : C.slot_mask[s2];
+            if (mk >> m & 1u) y = fmaf(C.slot_w[s2][m], __ldcg(&ws.ypart[((size_t)s2 * 4 + m) * H + row]), y);
+          }
+          a.out[(size_t)m * H + row] = y;
+        }
+      }
     }
   } else {
     // ============================== consumers =============================
@@ -458,40 +615,42 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     }
     // split grid barrier: arrive now, wait after the shared expert's items
     uint32_t bar_old = 0;
-    if (threadIdx.x == 0) {
-      __threadfence();
-      const uint32_t inc = c == 0 ? 0x80000000u - (uint32_t)(G - 1) : 1u;
-      bar_old = atomicAdd(&ws.hdr->barrier, inc);
-    }
+    if (threadIdx.x == 0) bar_old = grid_arrive(bar_word, c, G);
 
-    // x as f16 B fragments for this warp's K blocks of the gate/up GEMV
+    // x as E4M3 B fragments for this warp's K blocks of the gate/up GEMV.
+    // Within a 32-element block, lane (g, tq) covers elements 8tq..8tq+7 of
+    // token g: the even ones fill k-slots 4tq..4tq+3 (b0), the odd ones
+    // 16+4tq.. (b1), matching the even/odd split of the weight nibbles.  The
+    // token, scaled by 2^sigma, is carried exactly by two E4M3 parts (hi, lo).
     const int nbw_gu = (geo.nbH + kCons - 1) / kCons;
     const int b0_gu = cw * nbw_gu;
-    uint32_t bx[kGuB][2][2];
+    uint32_t bx[kGuB][2][2];  // [block][part][b0, b1]
     {
       const bool live = g < M;
       const float scl = live ? exp2i(C.sigma_x[g]) : 0.f;
 #pragma unroll
       for (int bi = 0; bi < kGuB; ++bi) {
         const int blk = b0_gu + bi;
+        uint32_t pe[2] = {0u, 0u}, po[2] = {0u, 0u};
+        if (live && bi < nbw_gu && blk < geo.nbH) {
+          const uint4 q = *reinterpret_cast<const uint4*>(a.x + (size_t)g * H + blk * 32 + tq * 8);
+          const float v0 = bf16_bits_to_f32(q.x & 0xffffu) * scl, v1 = bf16_bits_to_f32(q.x >> 16) * scl;
+          const float v2 = bf16_bits_to_f32(q.y & 0xffffu) * scl, v3 = bf16_bits_to_f32(q.y >> 16) * scl;
+          const float v4 = bf16_bits_to_f32(q.z & 0xffffu) * scl, v5 = bf16_bits_to_f32(q.z >> 16) * scl;
+          const float v6 = bf16_bits_to_f32(q.w & 0xffffu) * scl, v7 = bf16_bits_to_f32(q.w >> 16) * scl;
+          split_e4m3x4<2>(v0, v2, v4, v6, pe);
+          split_e4m3x4<2>(v1, v3, v5, v7, po);
+        }
 #pragma unroll
-        for (int mm = 0; mm < 2; ++mm) {
-#pragma unroll
-          for (int p = 0; p < 2; ++p) {
-            uint32_t v = 0u;
-            if (live && bi < nbw_gu && blk < geo.nbH) {
-              const int k0 = blk * 32 + tq * 8 + mm * 4 + p * 2;
-              const uint32_t pair = *reinterpret_cast<const uint32_t*>(a.x + (size_t)g * H + k0);
-              v = pack_h2(bf16_bits_to_f32(pair & 0xffffu) * scl, bf16_bits_to_f32(pair >> 16) * scl);
-            }
-            bx[bi][mm][p] = v;
-          }
+        for (int part = 0; part < 2; ++part) {
+          bx[bi][part][0] = pe[part];
+          bx[bi][part][1] = po[part];
         }
       }
     }
 
     int it = 0;     // ring position
-    int nitem = 0;  // items handed to the epilogue warp
+    int nitem = 0;  // items handed to the epilogue warps
     auto hand_off = [&](const float (&v)[8]) {
       const int r = nitem % kRed;
       if (nitem >= kRed) bounded_wait(&C.red_empty[r], (uint32_t)(((nitem / kRed) & 1) ^ 1));
@@ -516,15 +675,16 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
         for (int bi = 0; bi < kGuB; ++bi) {
           const int blk = b0_gu + bi;
           if (bi < nbw_gu && blk < geo.nbH) {
-            const uint32_t ga = lds32(base + g * geo.gu_stride + blk * 16 + tq * 4);
-            const uint32_t ua = lds32(base + (8 + g) * geo.gu_stride + blk * 16 + tq * 4);
+            const uint32_t gw = lds32(base + g * geo.gu_stride + blk * 16 + tq * 4);
+            const uint32_t uw = lds32(base + (8 + g) * geo.gu_stride + blk * 16 + tq * 4);
             const float sg = e8m0_to_f32(gsc[g * geo.nbH + blk]);
             const float su = e8m0_to_f32(usc[g * geo.nbH + blk]);
+            // A: gate row g (a0, a2) and up row g (a1, a3), 32 elements = one MX block
+            const uint32_t ge = e2m1x8_even_to_e4m3x4(gw), go = e2m1x8_odd_to_e4m3x4(gw);
+            const uint32_t ue = e2m1x8_even_to_e4m3x4(uw), uo = e2m1x8_odd_to_e4m3x4(uw);
             float d[4] = {0.f, 0.f, 0.f, 0.f};
-            mma16816(d, e2m1x2_to_f16x2(ga & 0xffu), e2m1x2_to_f16x2(ua & 0xffu), e2m1x2_to_f16x2((ga >> 8) & 0xffu),
-                     e2m1x2_to_f16x2((ua >> 8) & 0xffu), bx[bi][0][0], bx[bi][0][1]);
-            mma16816(d, e2m1x2_to_f16x2((ga >> 16) & 0xffu), e2m1x2_to_f16x2((ua >> 16) & 0xffu),
-                     e2m1x2_to_f16x2(ga >> 24), e2m1x2_to_f16x2(ua >> 24), bx[bi][1][0], bx[bi][1][1]);
+            mma_e4m3(d, ge, ue, go, uo, bx[bi][0][0], bx[bi][0][1]);
+            mma_e4m3(d, ge, ue, go, uo, bx[bi][1][0], bx[bi][1][1]);
             acc[0] = fmaf(d[0], sg, acc[0]);
             acc[1] = fmaf(d[1], sg, acc[1]);
             acc[2] = fmaf(d[2], su, acc[2]);
@@ -542,22 +702,16 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     const int nbw_dn = (geo.nbI + kCons - 1) / kCons;
     const int b0_dn = cw * nbw_dn;
     auto down_item = [&](int slot) {
-      // wait until every row of h for this slot is written (bounded)
-      bool ok = !*(volatile int*)&C.poison;
-      if (ok && lane == 0) ok = bounded_spin([&] { return ld_acquire(&ws.slot_ready[slot]) >= (uint32_t)I; });
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      __syncwarp();  // orders lane 0's acquire before the other lanes' reads of h
-      if (!ok && lane == 0 && !*(volatile int*)&C.poison) {
-        report(ws.hdr, MOE_ERR_TIMEOUT);
-        atomicExch(&C.poison, 1);
-      }
       const uint32_t mask = slot == 0 ? 0xfu : C.slot_mask[slot];
-      // B fragments: h of token g as an f16 hi/lo pair, scaled by 2^sigma
-      uint32_t bh[kDnB][2][2], bl[kDnB][2][2];
+      // B fragments: h of token g, per 32-element block scaled by a power of
+      // two that puts the block's largest magnitude in [2^7, 2^8), then split
+      // into three E4M3 parts (12 significant bits), even/odd permuted as for
+      // x.  f0 / f1 undo the scales of tokens 2tq and 2tq+1 (and the E4M3
+      // weights' 2^-6) on the MMA results.
+      uint32_t bh[kDnB][kHParts][2];
+      float f0[kDnB], f1[kDnB];
       {
-        const bool live = ok && g < M && (mask >> g & 1u);
-        const float hm = live ? __uint_as_float(__ldcg(&ws.hmax[slot * 4 + g])) : 0.f;
-        const float scl = live ? exp2i(pow2_sigma(hm)) : 0.f;
+        const bool live = !poisoned() && g < M && (mask >> g & 1u);
         float v[kDnB][8];
 #pragma unroll
         for (int bi = 0; bi < kDnB; ++bi) {  // all loads first
@@ -575,18 +729,28 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
         }
 #pragma unroll
         for (int bi = 0; bi < kDnB; ++bi) {
+          float mx = 0.f;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float x0 = v[bi][2 * q] * scl, x1 = v[bi][2 * q + 1] * scl;
-            const __half2 hi = __floats2half2_rn(x0, x1);
-            const float2 hf = __half22float2(hi);
-            bh[bi][q >> 1][q & 1] = *reinterpret_cast<const uint32_t*>(&hi);
-            bl[bi][q >> 1][q & 1] = pack_h2(x0 - hf.x, x1 - hf.y);
+          for (int q = 0; q < 8; ++q) mx = fmaxf(mx, fabsf(v[bi][q]));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));  // the block of token g spans lanes 4g..4g+3
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          const int sig = pow2_sigma(mx);
+          const float scl = exp2i(sig);
+          const float f = exp2i(6 - sig);
+          f0[bi] = __shfl_sync(0xffffffffu, f, 8 * tq);      // token 2tq lives in lanes 8tq..8tq+3
+          f1[bi] = __shfl_sync(0xffffffffu, f, 8 * tq + 4);  // token 2tq+1
+          uint32_t pe[kHParts], po[kHParts];
+          split_e4m3x4<kHParts>(v[bi][0] * scl, v[bi][2] * scl, v[bi][4] * scl, v[bi][6] * scl, pe);
+          split_e4m3x4<kHParts>(v[bi][1] * scl, v[bi][3] * scl, v[bi][5] * scl, v[bi][7] * scl, po);
+#pragma unroll
+          for (int part = 0; part < kHParts; ++part) {
+            bh[bi][part][0] = pe[part];
+            bh[bi][part][1] = po[part];
           }
         }
       }
       const int st = it % kStages;
-      ok = bounded_wait(&C.full[st], (uint32_t)((it / kStages) & 1)) && ok;
+      const bool ok = bounded_wait(&C.full[st], (uint32_t)((it / kStages) & 1));
       const uint8_t* base = ring + (size_t)st * geo.stage_bytes;
       const uint8_t* dsc = base + kDnRows * geo.dn_stride;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -602,19 +766,15 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
               const uint32_t wb = lds32(base + r_hi * geo.dn_stride + blk * 16 + tq * 4);
               const float sa = e8m0_to_f32(dsc[r_lo * geo.nbI + blk]);
               const float sb = e8m0_to_f32(dsc[r_hi * geo.nbI + blk]);
-              const uint32_t a00 = e2m1x2_to_f16x2(wa & 0xffu), a01 = e2m1x2_to_f16x2(wb & 0xffu);
-              const uint32_t a02 = e2m1x2_to_f16x2((wa >> 8) & 0xffu), a03 = e2m1x2_to_f16x2((wb >> 8) & 0xffu);
-              const uint32_t a10 = e2m1x2_to_f16x2((wa >> 16) & 0xffu), a11 = e2m1x2_to_f16x2((wb >> 16) & 0xffu);
-              const uint32_t a12 = e2m1x2_to_f16x2(wa >> 24), a13 = e2m1x2_to_f16x2(wb >> 24);
+              const uint32_t ae = e2m1x8_even_to_e4m3x4(wa), ao = e2m1x8_odd_to_e4m3x4(wa);
+              const uint32_t be = e2m1x8_even_to_e4m3x4(wb), bo = e2m1x8_odd_to_e4m3x4(wb);
               float d[4] = {0.f, 0.f, 0.f, 0.f};
-              mma16816(d, a00, a01, a02, a03, bh[bi][0][0], bh[bi][0][1]);
-              mma16816(d, a00, a01, a02, a03, bl[bi][0][0], bl[bi][0][1]);
-              mma16816(d, a10, a11, a12, a13, bh[bi][1][0], bh[bi][1][1]);
-              mma16816(d, a10, a11, a12, a13, bl[bi][1][0], bl[bi][1][1]);
-              acc[4 * tt + 0] = fmaf(d[0], sa, acc[4 * tt + 0]);
-              acc[4 * tt + 1] = fmaf(d[1], sa, acc[4 * tt + 1]);
-              acc[4 * tt + 2] = fmaf(d[2], sb, acc[4 * tt + 2]);
-              acc[4 * tt + 3] = fmaf(d[3], sb, acc[4 * tt + 3]);
+#pragma unroll
+              for (int part = 0; part < kHParts; ++part) mma_e4m3(d, ae, be, ao, bo, bh[bi][part][0], bh[bi][part][1]);
+              acc[4 * tt + 0] = fmaf(d[0], sa * f0[bi], acc[4 * tt + 0]);
+              acc[4 * tt + 1] = fmaf(d[1], sa * f1[bi], acc[4 * tt + 1]);
+              acc[4 * tt + 2] = fmaf(d[2], sb * f0[bi], acc[4 * tt + 2]);
+              acc[4 * tt + 3] = fmaf(d[3], sb * f1[bi], acc[4 * tt + 3]);
             }
           }
         }
@@ -628,100 +788,78 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     // ---- phase 1: the shared expert's items (no routing needed), then,
     //      once every CTA's logits are in, routing and the routed items ----
     const int ns = items.n_shared();
-    int S = 0, n1 = ns, n2 = 0;
+    int n1 = ns, n2 = 0;
     for (int j = 0;; ++j) {
       if (j == ns) {
         // ---- wait for every CTA's logits (bounded), then route ----
-        if (threadIdx.x == 0 && !*(volatile int*)&C.poison) {
-          const bool ok = bounded_spin([&] { return ((ld_acquire(&ws.hdr->barrier) ^ bar_old) & 0x80000000u) != 0u; });
-          if (!ok) {
-            report(ws.hdr, MOE_ERR_TIMEOUT);
-            atomicExch(&C.poison, 1);
-          }
-        }
+        if (threadIdx.x == 0 && !poisoned() && !grid_wait(bar_word, bar_old)) fail();
         consumer_bar_sync();
-        if (cw < M) {
+        if (cw < M) {  // warp m routes token m
           const int m = cw;
-          float lv[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            lv[i] = (lane + 32 * i < E) ? __ldcg(&ws.logits[(size_t)m * E + lane + 32 * i]) : -FLT_MAX;
-          uint32_t taken = 0u;
-          float top[8];
-          for (int r = 0; r < a.top_k; ++r) {
-            float bv = -FLT_MAX;
-            int32_t bi = INT32_MAX;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int e2 = lane + 32 * i;
-              if (e2 < E && !(taken >> i & 1u) && better(lv[i], e2, bv, bi)) { bv = lv[i]; bi = e2; }
-            }
-            warp_best(bv, bi);
-            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-            top[r] = bv;
-            if (lane == 0) C.ids[m][r] = bi;
+          warp_route(ws.logits + (size_t)m * E, E, a.top_k, lane, C.cand_v[m], C.cand_i[m], C.ids[m], C.topv[m]);
+          if (lane == 0) {
+            float z = 0.f;
+            for (int r = 0; r < a.top_k; ++r) z += expf(C.topv[m][r] - C.topv[m][0]);
+            for (int r = 0; r < a.top_k; ++r) C.wts[m][r] = expf(C.topv[m][r] - C.topv[m][0]) / z;
           }
-          float z = 0.f;
-          for (int r = 0; r < a.top_k; ++r) z += expf(top[r] - top[0]);
-          if (lane == 0)
-            for (int r = 0; r < a.top_k; ++r) C.wts[m][r] = expf(top[r] - top[0]) / z;
         }
         consumer_bar_sync();
-        if (threadIdx.x == 0) {
-          int n = 1;
-          C.slot_expert[0] = -1;
-          C.slot_mask[0] = 0xfu;
-          for (int m = 0; m < 4; ++m) C.slot_w[0][m] = 1.0f;
-          for (int m = 0; m < M; ++m) {
-            for (int r = 0; r < a.top_k; ++r) {
-              const int32_t ex = C.ids[m][r];
-              int sl = 1;
-              while (sl < n && C.slot_expert[sl] != ex) ++sl;
-              if (sl == n) {
-                C.slot_expert[n] = ex;
-                C.slot_mask[n] = 0u;
-                for (int mm = 0; mm < 4; ++mm) C.slot_w[n][mm] = 0.f;
-                ++n;
-              }
-              C.slot_mask[sl] |= 1u << m;
-              C.slot_w[sl][m] = C.wts[m][r];
-            }
+        if (cw == 0) {
+          // Slot table: slot 0 is the shared expert, then one slot per distinct
+          // routed expert in order of first appearance over (token, rank).
+          // Lane l holds choice l = m * top_k + r (M * top_k <= 32).
+          const int k = a.top_k, n_in = M * k;
+          const bool act = lane < n_in;
+          const int m = act ? lane / k : 0, r = act ? lane - (lane / k) * k : 0;
+          int32_t ex = act ? C.ids[m][r] : -1 - lane;  // idle lanes get ids of their own
+          if (act && (ex < 0 || ex >= E)) {  // cannot happen (see warp_route); never index out of range
+            report(ws.hdr, MOE_ERR_DEVICE_CHECK);
+            ex = 0;
           }
-          C.nslots = n;
-          __threadfence_block();
-          mbar_arrive(&C.routed);  // the producer and the epilogue warp may go on
+          const uint32_t same = __match_any_sync(0xffffffffu, ex);
+          const int leader = __ffs(same) - 1;
+          const uint32_t leaders = __ballot_sync(0xffffffffu, act && leader == lane);
+          const int slot = 1 + __popc(leaders & ((1u << leader) - 1u));
+          if (act && leader == lane) {
+            C.slot_expert[slot] = ex;
+            C.slot_mask[slot] = 0u;
+            for (int mm = 0; mm < 4; ++mm) C.slot_w[slot][mm] = 0.f;
+          }
+          if (lane == 0) {
+            C.slot_expert[0] = -1;
+            C.slot_mask[0] = 0xfu;
+            for (int mm = 0; mm < 4; ++mm) C.slot_w[0][mm] = 1.0f;
+          }
+          __syncwarp();
+          if (act) {
+            atomicOr(&C.slot_mask[slot], 1u << m);
+            C.slot_w[slot][m] = C.wts[m][r];  // a token picks an expert at most once
+          }
+          __syncwarp();
+          if (lane == 0) {
+            C.nslots = 1 + __popc(leaders);
+            __threadfence_block();
+            mbar_arrive(&C.routed);  // the producer and the epilogue warps may go on
+          }
         }
         consumer_bar_sync();
-        S = C.nslots;
+        const int S = C.nslots;
         if (c == 0) {
           for (int i = threadIdx.x; i < M * a.top_k; i += kCons * 32) {
             if (a.ids_out) a.ids_out[i] = C.ids[i / a.top_k][i % a.top_k];
             if (a.w_out) a.w_out[i] = C.wts[i / a.top_k][i % a.top_k];
           }
         }
-
         n1 = items.n_phase1(S);
         n2 = items.n_phase2(S);
       }
       if (j >= n1) break;
       gateup_item();
     }
+    // phase 2 reads every CTA's h: wait until the epilogue warps have seen the
+    // grid barrier that follows phase 1
+    bounded_wait(&C.h_ready, 0);
     for (int j = 0; j < n2; ++j) down_item((c + j * G) / geo.n_tiles);
-  }
-
-  // ---- the last CTA to finish resets the per-call counters ----
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    C.last = atomicAdd(&ws.hdr->ticket, 1u) == (uint32_t)(G - 1);
-  }
-  __syncthreads();
-  if (C.last) {
-    __threadfence();
-    for (int i = threadIdx.x; i < MoeWs::kMaxSlots; i += blockDim.x) ws.slot_ready[i] = 0u;
-    for (int i = threadIdx.x; i < MoeWs::kMaxSlots * 4; i += blockDim.x) ws.hmax[i] = 0u;
-    __syncthreads();
-    if (threadIdx.x == 0) ws.hdr->ticket = 0u;
   }
 }
 
@@ -734,19 +872,18 @@ size_t moe_fused_smem_bytes(int H, int I) {
 
 bool moe_fused_supported(int H, int I) {
   return H % 64 == 0 && I % 64 == 0 && H / 32 <= kMaxGuBlocksPerWarp * kCons &&
-         I / 32 <= kMaxDnBlocksPerWarp * kCons && moe_fused_smem_bytes(H, I) <= 232448;
+         I / 32 <= kMaxDnBlocksPerWarp * kCons && moe_fused_smem_bytes(H, I) <= (size_t)kMaxDynamicSmem;
 }
 
 template <int kGuB>
 static cudaError_t launch_fused_t(const FusedArgs& a, size_t smem, cudaStream_t st) {
   auto kern = moe_fused_kernel<kGuB>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem_optin<moe_fused_kernel<kGuB>>();
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0, per_sm = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreadsAll, smem)) != cudaSuccess) return e;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  int dev = 0, sms = 0;
+  if ((e = current_device_sms(&dev, &sms)) != cudaSuccess) return e;
+  // one CTA per SM; the cooperative launch fails (it does not wait) if they
+  // cannot all be resident at once
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(sms);  // one CTA per SM; all resident (cooperative launch)
   cfg.blockDim = dim3(kThreadsAll);
@@ -757,7 +894,9 @@ static cudaError_t launch_fused_t(const FusedArgs& a, size_t smem, cudaStream_t 
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a);
+  e = cudaLaunchKernelEx(&cfg, kern, a);
+  if (e != cudaSuccess) (void)cudaGetLastError();  // leave no stale error for the next call to find
+  return e;
 }
 
 cudaError_t launch_moe_fused(const MoeArgs& m, cudaStream_t st) {
