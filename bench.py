@@ -175,7 +175,9 @@ class Workload:
                 del st
                 sh = I.expert_matrix(seed, s, "shared", kind, layer=l, device=device)
                 shared.append(B.moe_quantize_mxfp4(sh))
-            self.layers.append((router, tuple(banks), tuple(shared)))
+            # load time: regroup the quantised bytes into the layout moe_decode streams
+            self.layers.append((router, B.moe_pack_experts(tuple(banks)), B.moe_pack_experts(tuple(shared))))
+            del banks, shared
         self.head_bf16 = self.head = None
         if head:
             self.head_bf16 = I.normal(seed, "lmhead", (h.vocab, h.hidden), I.WEIGHT_STD, device=device)
@@ -321,7 +323,8 @@ class Stream:
                 del st
                 shared.append(B.moe_quantize_mxfp4(I.expert_matrix(seed, s, "shared", kind, layer=100 + l,
                                                                     device=device)))
-            self.layers.append((router, tuple(banks), tuple(shared)))
+            self.layers.append((router, B.moe_pack_experts(tuple(banks)), B.moe_pack_experts(tuple(shared))))
+            del banks, shared
         self.head = head
         self.table = I.normal(seed, "embed", (h.vocab, h.hidden), 1.0, device=device)
         self.ids = torch.arange(M, dtype=torch.int32, device=device).view(M, 1).repeat(1, 1) * 7 + 3

@@ -86,7 +86,8 @@ typedef enum {
     MOE_FMT_NONE = 0,
     MOE_FMT_BF16 = 1,
     MOE_FMT_MXFP4_E2M1_E8M0_32 = 2,
-    MOE_FMT_FP8_E4M3_ROWSCALE_F32 = 3
+    MOE_FMT_FP8_E4M3_ROWSCALE_F32 = 3,
+    MOE_FMT_MXFP4_MOE_PACKED = 4
 } moe_format;
 
 /* A stack of `count` MXFP4 matrices, each [rows][K]:
@@ -110,6 +111,29 @@ typedef struct {
     moe_mxfp4_tensor up;
     moe_mxfp4_tensor down;
 } moe_expert_bank;
+
+/* An expert bank re-laid out for moe_decode (moe_pack_experts): the same
+ * MXFP4 bytes, grouped so that each unit of the kernel's work is one
+ * contiguous run that a single bulk copy moves.
+ *   gateup [count][I/8][16 * (H/2 + H/32) bytes]: for each 8-row chunk q of an
+ *          expert, gate rows 8q..8q+7 then up rows 8q..8q+7 (H/2 bytes each),
+ *          then the 8 gate scale rows and the 8 up scale rows (H/32 bytes each);
+ *   down   [count][H/32][32 * (I/2 + I/32) bytes]: for each 32-row tile t,
+ *          down rows 32t..32t+31 (I/2 bytes each), then their 32 scale rows.
+ * Within a data row, the 16-byte unit c (one 32-element block) of row r is
+ * stored at position c ^ (r & mask), mask = min(8, largest power of two
+ * dividing the units per row) - 1, so that eight consecutive rows read
+ * together hit distinct shared-memory banks.  fmt must be
+ * MOE_FMT_MXFP4_MOE_PACKED.  The pages have no counterpart for this layout;
+ * it changes where bytes sit, never their values.                             */
+typedef struct {
+    int32_t fmt;
+    int32_t count;
+    int32_t hidden;
+    int32_t inter;
+    uint8_t* gateup;
+    uint8_t* down;
+} moe_packed_bank;
 
 /* The online-FP8 LM head: q [vocab][hidden] E4M3 and row_scale [vocab] fp32.
  * fmt must be MOE_FMT_FP8_E4M3_ROWSCALE_F32.                                   */
@@ -139,6 +163,18 @@ typedef struct {
  * the OCP MX conversion rule stated at the top of this header.               */
 MOE_API moe_status moe_quantize_mxfp4(const uint16_t* w_bf16, moe_mxfp4_tensor* out, void* stream);
 
+/* Bytes of the two packed arrays of a bank with `count` experts (0 if the
+ * sizes are unsupported: hidden and inter multiples of 64).                  */
+MOE_API size_t moe_packed_gateup_bytes(int32_t count, int32_t hidden, int32_t inter);
+MOE_API size_t moe_packed_down_bytes(int32_t count, int32_t hidden, int32_t inter);
+
+/* Re-lay out a quantised bank (`src`: gate and up count x [I][H], down
+ * count x [H][I], all tagged MXFP4) into `dst`, whose caller fills count,
+ * hidden, inter and the two device arrays (sizes above, 16-byte aligned).
+ * Enqueued on `stream`; on success sets dst->fmt.  The source is not needed
+ * by moe_decode afterwards.                                                  */
+MOE_API moe_status moe_pack_experts(const moe_expert_bank* src, moe_packed_bank* dst, void* stream);
+
 /* Quantise the bf16 head w [vocab][hidden] into `out` (caller fills vocab,
  * hidden, q, row_scale): s_v = fp32(amax_v / 448) (1 for an all-zero row),
  * q = E4M3 RNE satfinite of fp32(w / s_v).  On success sets out->fmt.
@@ -155,7 +191,8 @@ MOE_API size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts
 /* One MoE layer for M tokens (1 <= M <= 4):
  *   hidden      [M][H] bf16
  *   router_w    [E][H] fp32;  router_bias [E] fp32 or NULL (added to the logits)
- *   experts     routed bank (count E), shared: bank with count 1 (host structs)
+ *   experts     routed bank (count E), shared: bank with count 1; both packed
+ *               by moe_pack_experts (host structs, device arrays)
  *   out         [M][H] fp32:  sum_i w_i expert_{id_i}(x) + shared(x)
  *   topk_ids    [M][top_k] int32 or NULL: selected experts, by descending logit
  *   topk_w      [M][top_k] fp32 or NULL:  renormalised softmax weights
@@ -166,7 +203,7 @@ MOE_API size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts
  * (one CTA per SM, all resident).  Each distinct routed expert is streamed once per call, however
  * many of the M tokens chose it.                                             */
 MOE_API moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const float* router_bias,
-                      const moe_expert_bank* experts, const moe_expert_bank* shared,
+                      const moe_packed_bank* experts, const moe_packed_bank* shared,
                       int32_t M, int32_t top_k, float* out, int32_t* topk_ids, float* topk_w,
                       void* workspace, size_t workspace_bytes, void* stream);
 

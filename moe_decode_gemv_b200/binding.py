@@ -36,6 +36,7 @@ class Format(enum.IntEnum):
     BF16 = 1
     MXFP4_E2M1_E8M0_32 = 2
     FP8_E4M3_ROWSCALE_F32 = 3
+    MXFP4_MOE_PACKED = 4
 
 
 class MoEError(RuntimeError):
@@ -51,6 +52,11 @@ class _Mxfp4(ctypes.Structure):
 
 class _Bank(ctypes.Structure):
     _fields_ = [("gate", _Mxfp4), ("up", _Mxfp4), ("down", _Mxfp4)]
+
+
+class _Packed(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("count", ctypes.c_int32), ("hidden", ctypes.c_int32),
+                ("inter", ctypes.c_int32), ("gateup", ctypes.c_void_p), ("down", ctypes.c_void_p)]
 
 
 class _Fp8Head(ctypes.Structure):
@@ -73,7 +79,10 @@ def _load() -> ctypes.CDLL:
         "moe_quantize_mxfp4": ([P, ctypes.POINTER(_Mxfp4), P], I32),
         "lmhead_quantize_fp8": ([P, ctypes.POINTER(_Fp8Head), P], I32),
         "moe_workspace_bytes": ([I32, I32, I32, I32, I32], SZ),
-        "moe_decode": ([P, P, P, ctypes.POINTER(_Bank), ctypes.POINTER(_Bank), I32, I32, P, P, P, P, SZ, P], I32),
+        "moe_packed_gateup_bytes": ([I32, I32, I32], SZ),
+        "moe_packed_down_bytes": ([I32, I32, I32], SZ),
+        "moe_pack_experts": ([ctypes.POINTER(_Bank), ctypes.POINTER(_Packed), P], I32),
+        "moe_decode": ([P, P, P, ctypes.POINTER(_Packed), ctypes.POINTER(_Packed), I32, I32, P, P, P, P, SZ, P], I32),
         "lmhead_workspace_bytes": ([I32, I32, I64, I64], SZ),
         "lmhead_decode": ([P, ctypes.POINTER(_Fp8Head), I32, I32, P, P, P, P, SZ, P], I32),
         "lmhead_decode_bf16": ([P, ctypes.POINTER(_Bf16Head), I32, I32, P, P, P, P, SZ, P], I32),
@@ -148,6 +157,26 @@ def alloc_mxfp4_bank(count: int, rows: int, K: int, device="cuda") -> MXFP4Bank:
 
 
 @dataclass
+class PackedBank:
+    """An expert bank laid out for moe_decode (moe_pack_experts): gateup
+    [count * I/8 * 16 (H/2 + H/32)] and down [count * H/32 * 32 (I/2 + I/32)]
+    uint8, the MXFP4 bytes grouped into one contiguous run per unit of the
+    kernel's work."""
+    gateup: torch.Tensor
+    down: torch.Tensor
+    count: int
+    hidden: int
+    inter: int
+    fmt: int = Format.NONE
+
+    def _c(self) -> _Packed:
+        return _Packed(int(self.fmt), self.count, self.hidden, self.inter, self.gateup.data_ptr(), self.down.data_ptr())
+
+    def nbytes(self) -> int:
+        return self.gateup.numel() + self.down.numel()
+
+
+@dataclass
 class FP8Head:
     """The online-FP8 LM head: q [V, H] uint8 (E4M3) and row_scale [V] fp32."""
     q: torch.Tensor
@@ -183,6 +212,23 @@ def moe_quantize_mxfp4(w_bf16: torch.Tensor, out: MXFP4Bank | None = None, strea
     return out
 
 
+def moe_pack_experts(bank: tuple[MXFP4Bank, MXFP4Bank, MXFP4Bank], stream=None) -> PackedBank:
+    """(gate, up, down) quantised banks -> the packed bank moe_decode reads."""
+    gate, up, down = bank
+    E, H, I = gate.count, gate.K, gate.rows
+    gb = int(library.moe_packed_gateup_bytes(E, H, I))
+    db = int(library.moe_packed_down_bytes(E, H, I))
+    if gb == 0 or db == 0:
+        raise MoEError(Status.UNSUPPORTED_SHAPE, "moe_pack_experts")
+    dev = gate.data.device
+    out = PackedBank(torch.empty((gb,), dtype=torch.uint8, device=dev), torch.empty((db,), dtype=torch.uint8, device=dev),
+                     E, H, I)
+    src, c = _bank_c(gate, up, down), out._c()
+    _check(library.moe_pack_experts(ctypes.byref(src), ctypes.byref(c), _stream(stream)), "moe_pack_experts")
+    out.fmt = c.fmt
+    return out
+
+
 def lmhead_quantize_fp8(w_bf16: torch.Tensor, out: FP8Head | None = None, stream=None) -> FP8Head:
     assert w_bf16.dtype == torch.bfloat16 and w_bf16.is_cuda and w_bf16.is_contiguous()
     if out is None:
@@ -209,15 +255,15 @@ def new_workspace(nbytes: int, device="cuda", stream=None) -> torch.Tensor:
 
 
 def moe_decode(hidden: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None,
-               experts: tuple[MXFP4Bank, MXFP4Bank, MXFP4Bank], shared: tuple[MXFP4Bank, MXFP4Bank, MXFP4Bank],
-               top_k: int, out: torch.Tensor, topk_ids: torch.Tensor | None = None,
-               topk_w: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+               experts: PackedBank, shared: PackedBank, top_k: int, out: torch.Tensor,
+               topk_ids: torch.Tensor | None = None, topk_w: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """One MoE layer: out[M, H] fp32 = sum_i w_i expert_i(x) + shared(x)."""
     M = hidden.shape[0]
     if workspace is None:
-        workspace = new_workspace(moe_workspace_bytes(M, top_k, experts[0].count, experts[0].K, experts[0].rows),
+        workspace = new_workspace(moe_workspace_bytes(M, top_k, experts.count, experts.hidden, experts.inter),
                                   hidden.device, stream)
-    eb, sb = _bank_c(*experts), _bank_c(*shared)
+    eb, sb = experts._c(), shared._c()
     st = library.moe_decode(_ptr(hidden), _ptr(router_w), _ptr(router_bias), ctypes.byref(eb), ctypes.byref(sb),
                             M, top_k, _ptr(out), _ptr(topk_ids), _ptr(topk_w), _ptr(workspace), workspace.numel(),
                             _stream(stream))

@@ -13,6 +13,7 @@
 #include "device_cache.h"
 #include "lmhead.h"
 #include "moe.h"
+#include "pack.h"
 #include "quantize.h"
 #include "stack.h"
 
@@ -39,8 +40,17 @@ moe_status check_bank(const moe_expert_bank* b, int64_t count, int64_t H, int64_
   return check_mxfp4(b->down, count, H, I);
 }
 
-moe::MoeBank bank_ptrs(const moe_expert_bank* b) {
-  return moe::MoeBank{b->gate.data, b->gate.scales, b->up.data, b->up.scales, b->down.data, b->down.scales};
+bool pack_shape_ok(int64_t count, int64_t H, int64_t I) {
+  return count >= 1 && count <= (int64_t(1) << 20) && H >= 64 && I >= 64 && H % 64 == 0 && I % 64 == 0 &&
+         H <= 65536 && I <= 65536;
+}
+
+moe_status check_packed(const moe_packed_bank* b, int64_t count, int64_t H, int64_t I) {
+  if (b->fmt != MOE_FMT_MXFP4_MOE_PACKED) return MOE_ERR_FORMAT_MISMATCH;
+  if (!b->gateup || !b->down) return MOE_ERR_INVALID_ARG;
+  if (b->count != count || b->hidden != H || b->inter != I) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(b->gateup) || !aligned16(b->down)) return MOE_ERR_MISALIGNED;
+  return MOE_OK;
 }
 
 bool head_shape_ok(int64_t vocab, int64_t hidden, int elem_bytes) {
@@ -111,6 +121,32 @@ moe_status lmhead_quantize_fp8(const uint16_t* w_bf16, moe_fp8_head* out, void* 
   return MOE_OK;
 }
 
+size_t moe_packed_gateup_bytes(int32_t count, int32_t hidden, int32_t inter) {
+  return pack_shape_ok(count, hidden, inter) ? moe::packed_gateup_bytes(count, hidden, inter) : 0;
+}
+
+size_t moe_packed_down_bytes(int32_t count, int32_t hidden, int32_t inter) {
+  return pack_shape_ok(count, hidden, inter) ? moe::packed_down_bytes(count, hidden, inter) : 0;
+}
+
+moe_status moe_pack_experts(const moe_expert_bank* src, moe_packed_bank* dst, void* stream) {
+  if (!src || !dst || !dst->gateup || !dst->down) return MOE_ERR_INVALID_ARG;
+  for (const moe_mxfp4_tensor* t : {&src->gate, &src->up, &src->down})
+    if (t->fmt != MOE_FMT_MXFP4_E2M1_E8M0_32) return MOE_ERR_FORMAT_MISMATCH;
+  const int64_t E = src->gate.count, H = src->gate.K, I = src->gate.rows;
+  if (!pack_shape_ok(E, H, I) || dst->count != E || dst->hidden != H || dst->inter != I)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  moe_status s;
+  if ((s = check_bank(src, E, H, I)) != MOE_OK) return s;
+  if (!aligned16(dst->gateup) || !aligned16(dst->down)) return MOE_ERR_MISALIGNED;
+  cudaError_t e = moe::launch_pack_experts(src->gate.data, src->gate.scales, src->up.data, src->up.scales,
+                                           src->down.data, src->down.scales, E, (int)H, (int)I, dst->gateup,
+                                           dst->down, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  dst->fmt = MOE_FMT_MXFP4_MOE_PACKED;
+  return MOE_OK;
+}
+
 size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts, int32_t hidden, int32_t inter) {
   if (M < 1 || M > 4 || top_k < 1 || top_k > 8 || num_experts < 1 || num_experts > 1024) return 0;
   if (hidden < 64 || inter < 64 || !moe::moe_fused_supported(hidden, inter)) return 0;
@@ -118,21 +154,20 @@ size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts, int32_
 }
 
 moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const float* router_bias,
-                      const moe_expert_bank* experts, const moe_expert_bank* shared, int32_t M, int32_t top_k,
+                      const moe_packed_bank* experts, const moe_packed_bank* shared, int32_t M, int32_t top_k,
                       float* out, int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
                       void* stream) {
   if (!hidden_bf16 || !router_w || !experts || !shared || !out || !workspace) return MOE_ERR_INVALID_ARG;
   if (M < 1 || M > 4 || top_k < 1 || top_k > 8) return MOE_ERR_INVALID_ARG;
-  // every tag first: a wrong-format bank is the error to report, whatever else is wrong
-  for (const moe_mxfp4_tensor* t : {&experts->gate, &experts->up, &experts->down, &shared->gate, &shared->up,
-                                    &shared->down})
-    if (t->fmt != MOE_FMT_MXFP4_E2M1_E8M0_32) return MOE_ERR_FORMAT_MISMATCH;
-  const int64_t E = experts->gate.count, H = experts->gate.K, I = experts->gate.rows;
+  // both tags first: a wrong-format bank is the error to report, whatever else is wrong
+  if (experts->fmt != MOE_FMT_MXFP4_MOE_PACKED || shared->fmt != MOE_FMT_MXFP4_MOE_PACKED)
+    return MOE_ERR_FORMAT_MISMATCH;
+  const int64_t E = experts->count, H = experts->hidden, I = experts->inter;
   if (E < 1 || E > 1024 || top_k > E) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (H < 64 || I < 64 || !moe::moe_fused_supported((int)H, (int)I)) return MOE_ERR_UNSUPPORTED_SHAPE;
   moe_status s;
-  if ((s = check_bank(experts, E, H, I)) != MOE_OK) return s;
-  if ((s = check_bank(shared, 1, H, I)) != MOE_OK) return s;
+  if ((s = check_packed(experts, E, H, I)) != MOE_OK) return s;
+  if ((s = check_packed(shared, 1, H, I)) != MOE_OK) return s;
   if (!aligned16(hidden_bf16) || !aligned16(router_w) || (router_bias && !aligned16(router_bias)) ||
       !aligned16(out) || (topk_ids && !aligned16(topk_ids)) || (topk_w && !aligned16(topk_w)) ||
       !aligned16(workspace))
@@ -143,8 +178,8 @@ moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const 
   a.x = hidden_bf16;
   a.router_w = router_w;
   a.router_bias = router_bias;
-  a.bank = bank_ptrs(experts);
-  a.shared = bank_ptrs(shared);
+  a.bank = moe::MoeBank{experts->gateup, experts->down};
+  a.shared = moe::MoeBank{shared->gateup, shared->down};
   a.M = M; a.top_k = top_k; a.E = (int)E; a.H = (int)H; a.I = (int)I;
   a.out = out; a.ids_out = topk_ids; a.w_out = topk_w;
   a.ws = moe::MoeWs::carve(workspace, (int)E, (int)H, (int)I);

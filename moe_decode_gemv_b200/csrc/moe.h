@@ -9,14 +9,10 @@
 
 namespace moe {
 
-// Raw pointers of one expert bank (stacked over experts), see moe_expert_bank.
+// Device arrays of one packed expert bank (see moe_packed_bank and pack.h).
 struct MoeBank {
-  const uint8_t* gate_d;
-  const uint8_t* gate_s;
-  const uint8_t* up_d;
-  const uint8_t* up_s;
-  const uint8_t* down_d;
-  const uint8_t* down_s;
+  const uint8_t* gateup;  // [E][I/8][gateup_chunk_bytes(H)]
+  const uint8_t* down;    // [E][H/32][down_tile_bytes(I)]
 };
 
 // Views into the caller's workspace.  Token-indexed arrays use a fixed stride

@@ -11,10 +11,11 @@
 // HBM busy from the first microsecond:
 //
 //  * One CTA per SM (cooperative launch: all CTAs are resident, which the
-//    grid barriers below rely on).  A producer warp streams every weight tile
-//    the CTA will need into a ring of shared-memory stages with bulk copies
-//    (cp.async.bulk, no multicast); eight consumer warps compute; two
-//    epilogue warps finish each item and own everything that leaves the CTA.
+//    grid barriers below rely on).  A producer warp streams every weight unit
+//    the CTA will need into a ring of shared-memory stages, one bulk copy
+//    (cp.async.bulk, no multicast) per unit of the packed bank; eight
+//    consumer warps compute; two epilogue warps finish each item and own
+//    everything that leaves the CTA.
 //  * Phase 0: each CTA scores its share of the router rows (fp32 weights,
 //    bf16 activations, fp32 sums) and arrives at a split grid barrier.  The
 //    shared expert needs no routing, so its tiles are loaded and computed
@@ -47,6 +48,7 @@
 #include "common.cuh"
 #include "device_cache.h"
 #include "moe.h"
+#include "pack.h"
 
 namespace moe {
 namespace {
@@ -253,25 +255,25 @@ struct FusedArgs {
   MoeWs ws;
 };
 
-// Shared-memory layout of one ring stage.  Phase-1 item: 16 data rows
-// (8 gate, then 8 up) at a padded stride, then the 8 gate and 8 up scale rows.
-// Phase-2 item: 32 down data rows at a padded stride, then their 32 scale rows.
-// Strides are 16 * odd bytes, so the 8 rows a quarter of a warp reads from
-// land on distinct banks.
+// Shared-memory layout of one ring stage: one packed unit, exactly as it sits
+// in HBM (see pack.h), brought by one bulk copy.  Phase-1 item: 16 data rows
+// (8 gate, then 8 up) of H/2 bytes, then the 8 gate and 8 up scale rows.
+// Phase-2 item: 32 down data rows of I/2 bytes, then their 32 scale rows.
+// Within a data row the 16-byte units are XOR-permuted by the row index, so
+// the 8 rows a quarter of a warp reads from land on distinct banks.
 struct Geometry {
-  int H, I, nbH, nbI;   // blocks of 32 along H and along I
-  int gu_stride;        // H/2 + 16
-  int dn_stride;        // I/2 + 16
+  int H, I, nbH, nbI;   // blocks of 32 along H and along I (= 16-byte units per data row)
+  int mH, mI;           // unit swizzle masks of the gate/up and the down rows
   int gu_bytes, dn_bytes, stage_bytes;
   int n_chunks;         // I / 8 phase-1 items per slot
   int n_tiles;          // H / 32 phase-2 items per slot
   __host__ __device__ Geometry(int H_, int I_) : H(H_), I(I_) {
     nbH = H / 32;
     nbI = I / 32;
-    gu_stride = H / 2 + 16;
-    dn_stride = I / 2 + 16;
-    gu_bytes = 16 * gu_stride + 16 * nbH;
-    dn_bytes = kDnRows * dn_stride + kDnRows * nbI;
+    mH = swizzle_mask(nbH);
+    mI = swizzle_mask(nbI);
+    gu_bytes = gateup_chunk_bytes(H);
+    dn_bytes = down_tile_bytes(I);
     stage_bytes = ((gu_bytes > dn_bytes ? gu_bytes : dn_bytes) + 127) / 128 * 128;
     n_chunks = I / kGuRows;
     n_tiles = H / kDnRows;
@@ -406,29 +408,15 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
         const int ex = s_slot == 0 ? -1 : C.slot_expert[s_slot];
         const MoeBank& b = ex < 0 ? a.shared : a.bank;
         const size_t e = ex < 0 ? 0 : (size_t)ex;
-        if (phase1) {
-          const size_t mat_d = (size_t)I * H / 2, mat_s = (size_t)I * geo.nbH;
-          const uint32_t rowb = (uint32_t)(H / 2), scb = (uint32_t)(kGuRows * geo.nbH);
-          if (lane == 0) mbar_arrive_expect_tx(&C.full[st], 16u * rowb + 2u * scb);
-          __syncwarp();
-          if (lane < 16) {
-            const uint8_t* src = (lane < 8 ? b.gate_d : b.up_d) + e * mat_d + (size_t)(row0 + (lane & 7)) * rowb;
-            bulk_g2s(dst + lane * geo.gu_stride, src, rowb, &C.full[st], policy);
-          } else if (lane < 18) {
-            const uint8_t* src = (lane == 16 ? b.gate_s : b.up_s) + e * mat_s + (size_t)row0 * geo.nbH;
-            bulk_g2s(dst + 16 * geo.gu_stride + (lane - 16) * scb, src, scb, &C.full[st], policy);
-          }
-        } else {
-          const size_t mat_d = (size_t)H * I / 2, mat_s = (size_t)H * geo.nbI;
-          const uint32_t rowb = (uint32_t)(I / 2), scb = (uint32_t)(kDnRows * geo.nbI);
-          if (lane == 0) mbar_arrive_expect_tx(&C.full[st], kDnRows * rowb + scb);
-          __syncwarp();
-          bulk_g2s(dst + lane * geo.dn_stride, b.down_d + e * mat_d + (size_t)(row0 + lane) * rowb, rowb,
-                   &C.full[st], policy);
-          if (lane == 0)
-            bulk_g2s(dst + kDnRows * geo.dn_stride, b.down_s + e * mat_s + (size_t)row0 * geo.nbI, scb,
-                     &C.full[st], policy);
+        // one packed unit = one bulk copy
+        const uint8_t* src = phase1 ? b.gateup + (e * geo.n_chunks + row0 / kGuRows) * (size_t)geo.gu_bytes
+                                    : b.down + (e * geo.n_tiles + row0 / kDnRows) * (size_t)geo.dn_bytes;
+        const uint32_t bytes = (uint32_t)(phase1 ? geo.gu_bytes : geo.dn_bytes);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&C.full[st], bytes);
+          bulk_g2s(dst, src, bytes, &C.full[st], policy);
         }
+        __syncwarp();
         issued = it + 1;
       }
       ++it;
@@ -667,7 +655,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       const int st = it % kStages;
       const bool ok = bounded_wait(&C.full[st], (uint32_t)((it / kStages) & 1));
       const uint8_t* base = ring + (size_t)st * geo.stage_bytes;
-      const uint8_t* gsc = base + 16 * geo.gu_stride;
+      const int rowb = H / 2;
+      const uint8_t* gsc = base + 16 * rowb;
       const uint8_t* usc = gsc + kGuRows * geo.nbH;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (ok) {
@@ -675,8 +664,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
         for (int bi = 0; bi < kGuB; ++bi) {
           const int blk = b0_gu + bi;
           if (bi < nbw_gu && blk < geo.nbH) {
-            const uint32_t gw = lds32(base + g * geo.gu_stride + blk * 16 + tq * 4);
-            const uint32_t uw = lds32(base + (8 + g) * geo.gu_stride + blk * 16 + tq * 4);
+            const uint32_t gw = lds32(base + g * rowb + ((blk ^ (g & geo.mH)) * 16) + tq * 4);
+            const uint32_t uw = lds32(base + (8 + g) * rowb + ((blk ^ ((8 + g) & geo.mH)) * 16) + tq * 4);
             const float sg = e8m0_to_f32(gsc[g * geo.nbH + blk]);
             const float su = e8m0_to_f32(usc[g * geo.nbH + blk]);
             // A: gate row g (a0, a2) and up row g (a1, a3), 32 elements = one MX block
@@ -752,7 +741,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       const int st = it % kStages;
       const bool ok = bounded_wait(&C.full[st], (uint32_t)((it / kStages) & 1));
       const uint8_t* base = ring + (size_t)st * geo.stage_bytes;
-      const uint8_t* dsc = base + kDnRows * geo.dn_stride;
+      const int rowb = I / 2;
+      const uint8_t* dsc = base + kDnRows * rowb;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (ok) {
 #pragma unroll
@@ -762,8 +752,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
             const int blk = b0_dn + bi;
             if (bi < nbw_dn && blk < geo.nbI) {
               const int r_lo = 16 * tt + g, r_hi = r_lo + 8;
-              const uint32_t wa = lds32(base + r_lo * geo.dn_stride + blk * 16 + tq * 4);
-              const uint32_t wb = lds32(base + r_hi * geo.dn_stride + blk * 16 + tq * 4);
+              const uint32_t wa = lds32(base + r_lo * rowb + ((blk ^ (r_lo & geo.mI)) * 16) + tq * 4);
+              const uint32_t wb = lds32(base + r_hi * rowb + ((blk ^ (r_hi & geo.mI)) * 16) + tq * 4);
               const float sa = e8m0_to_f32(dsc[r_lo * geo.nbI + blk]);
               const float sb = e8m0_to_f32(dsc[r_hi * geo.nbI + blk]);
               const uint32_t ae = e2m1x8_even_to_e4m3x4(wa), ao = e2m1x8_odd_to_e4m3x4(wa);

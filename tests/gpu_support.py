@@ -101,6 +101,9 @@ class Layer:
         self.router_bias_dev = None if self.router_bias is None else self.router_bias.cuda()
         self.bank = tuple(self._quantize_bank(k, range(shape.experts)) for k in self.KINDS)
         self.shared = tuple(self._quantize_bank(k, ["shared"]) for k in self.KINDS)
+        # the layout moe_decode reads (same bytes, regrouped)
+        self.packed = B.moe_pack_experts(self.bank)
+        self.packed_shared = B.moe_pack_experts(self.shared)
 
     def _quantize_bank(self, kind, experts):
         s = self.shape
@@ -135,7 +138,7 @@ class Layer:
         out = torch.empty((M, self.shape.hidden), dtype=torch.float32, device="cuda")
         ids = torch.empty((M, k), dtype=torch.int32, device="cuda")
         w = torch.empty((M, k), dtype=torch.float32, device="cuda")
-        self.B.moe_decode(x_dev, self.router_w_dev, self.router_bias_dev, self.bank, self.shared, k, out, ids, w,
+        self.B.moe_decode(x_dev, self.router_w_dev, self.router_bias_dev, self.packed, self.packed_shared, k, out, ids, w,
                           workspace=workspace)
         torch.cuda.synchronize()
         return out.cpu().numpy(), ids.cpu().numpy(), w.cpu().numpy()

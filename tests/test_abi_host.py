@@ -75,6 +75,10 @@ def _bank(lib, fmt=2, E=16, H=256, I=64):
     return lib._Bank(_mx(lib, fmt, E, I, H), _mx(lib, fmt, E, I, H), _mx(lib, fmt, E, H, I))
 
 
+def _packed(lib, fmt=4, E=16, H=256, I=64, gateup=A, down=A):
+    return lib._Packed(fmt, E, H, I, gateup, down)
+
+
 def _decode(lib, experts, shared, M=1, top_k=2, x=A, ws=A, ws_bytes=1 << 24):
     L = lib.library
     return L.moe_decode(x, A, None, ctypes.byref(experts), ctypes.byref(shared), M, top_k, A, None, None,
@@ -83,23 +87,40 @@ def _decode(lib, experts, shared, M=1, top_k=2, x=A, ws=A, ws_bytes=1 << 24):
 
 def test_moe_decode_rejects_bad_arguments(lib):
     S = lib.Status
-    ok_bank, ok_shared = _bank(lib), _bank(lib, E=1)
-    # the integration trap: a bank tagged as something other than MXFP4
-    assert _decode(lib, _bank(lib, fmt=1), ok_shared) == S.FORMAT_MISMATCH
-    assert _decode(lib, ok_bank, _bank(lib, fmt=3, E=1)) == S.FORMAT_MISMATCH
+    ok_bank, ok_shared = _packed(lib), _packed(lib, E=1)
+    # the integration trap: a bank tagged as something other than the packed MXFP4 layout
+    assert _decode(lib, _packed(lib, fmt=2), ok_shared) == S.FORMAT_MISMATCH     # canonical MXFP4, not packed
+    assert _decode(lib, ok_bank, _packed(lib, fmt=3, E=1)) == S.FORMAT_MISMATCH
     assert _decode(lib, ok_bank, ok_shared, M=0) == S.INVALID_ARG
     assert _decode(lib, ok_bank, ok_shared, M=5) == S.INVALID_ARG
     assert _decode(lib, ok_bank, ok_shared, top_k=9) == S.INVALID_ARG
     assert _decode(lib, ok_bank, ok_shared, x=0) == S.INVALID_ARG
     assert _decode(lib, ok_bank, ok_shared, x=U) == S.MISALIGNED
     assert _decode(lib, ok_bank, ok_shared, ws_bytes=100) == S.WORKSPACE
-    assert _decode(lib, _bank(lib, H=250), _bank(lib, E=1, H=250)) == S.UNSUPPORTED_SHAPE
-    assert _decode(lib, ok_bank, _bank(lib, E=2)) == S.UNSUPPORTED_SHAPE          # shared count != 1
-    assert _decode(lib, ok_bank, _bank(lib, E=1, I=96)) == S.UNSUPPORTED_SHAPE    # shared width differs
+    assert _decode(lib, _packed(lib, H=250), _packed(lib, E=1, H=250)) == S.UNSUPPORTED_SHAPE
+    assert _decode(lib, ok_bank, _packed(lib, E=2)) == S.UNSUPPORTED_SHAPE          # shared count != 1
+    assert _decode(lib, ok_bank, _packed(lib, E=1, I=128)) == S.UNSUPPORTED_SHAPE   # shared width differs
+    assert _decode(lib, _packed(lib, gateup=U), ok_shared) == S.MISALIGNED
+    assert _decode(lib, _packed(lib, down=0), ok_shared) == S.INVALID_ARG
+
+
+def test_pack_rejects_bad_arguments_and_sizes(lib):
+    S, L = lib.Status, lib.library
+    # sizes: one gate/up chunk is 16 (H/2 + H/32) bytes per 8 rows, one down tile 32 (I/2 + I/32) per 32 rows
+    assert L.moe_packed_gateup_bytes(512, 2560, 768) == 512 * 96 * 16 * (1280 + 80)
+    assert L.moe_packed_down_bytes(512, 2560, 768) == 512 * 80 * 32 * (384 + 24)
+    assert L.moe_packed_gateup_bytes(512, 2560, 768) + L.moe_packed_down_bytes(512, 2560, 768) == 512 * 3133440
+    assert L.moe_packed_gateup_bytes(1, 250, 64) == 0 and L.moe_packed_down_bytes(1, 256, 96) == 0
+
+    def pack(src, dst):
+        return L.moe_pack_experts(ctypes.byref(src), ctypes.byref(dst), None)
+
+    assert pack(_bank(lib, fmt=1), _packed(lib, fmt=0)) == S.FORMAT_MISMATCH
+    assert pack(_bank(lib), _packed(lib, fmt=0, E=8)) == S.UNSUPPORTED_SHAPE        # dst count differs
+    assert pack(_bank(lib), _packed(lib, fmt=0, gateup=U)) == S.MISALIGNED
+    assert pack(_bank(lib), _packed(lib, fmt=0, down=0)) == S.INVALID_ARG
     bad_down = lib._Bank(_mx(lib, 2, 16, 64, 256), _mx(lib, 2, 16, 64, 256), _mx(lib, 2, 16, 64, 256))
-    assert _decode(lib, bad_down, ok_shared) == S.UNSUPPORTED_SHAPE               # down not [H][I]
-    misaligned = lib._Bank(_mx(lib, 2, 16, 64, 256, data=U), _mx(lib, 2, 16, 64, 256), _mx(lib, 2, 16, 256, 64))
-    assert _decode(lib, misaligned, ok_shared) == S.MISALIGNED
+    assert pack(bad_down, _packed(lib, fmt=0)) == S.UNSUPPORTED_SHAPE               # down not [H][I]
 
 
 def test_lmhead_rejects_bad_arguments(lib):

@@ -1,0 +1,77 @@
+"""The packed expert-bank layout, byte for byte, against a numpy statement of
+the layout that moe_gemv.h documents for moe_packed_bank (packing moves
+bytes only, so the comparison is exact)."""
+import numpy as np
+import pytest
+import torch
+
+from moe_decode_gemv_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B():
+    from moe_decode_gemv_b200 import build
+    build.build()
+    from moe_decode_gemv_b200 import binding
+    return binding
+
+
+def swizzle_mask(units):
+    low = units & -units
+    return min(8, low) - 1
+
+
+def expected_packed(gate, up, down):
+    """numpy: (data, scales) pairs of the canonical banks -> (gateup, down) bytes."""
+    (gd, gs), (ud, us), (dd, ds) = gate, up, down
+    E, I, Hh = gd.shape
+    H = 2 * Hh
+    nbH, nbI = H // 32, I // 32
+    mH, mI = swizzle_mask(nbH), swizzle_mask(nbI)
+    gu = []
+    for e in range(E):
+        for q in range(I // 8):
+            rows = np.concatenate([gd[e, 8 * q:8 * q + 8], ud[e, 8 * q:8 * q + 8]])  # [16][H/2]
+            units = rows.reshape(16, nbH, 16)
+            # unit c of row r is stored at position c ^ (r & mask): position p holds unit p ^ (r & mask)
+            perm = np.stack([units[r, np.arange(nbH) ^ (r & mH)] for r in range(16)])
+            gu.append(perm.reshape(-1))
+            gu.append(gs[e, 8 * q:8 * q + 8].reshape(-1))
+            gu.append(us[e, 8 * q:8 * q + 8].reshape(-1))
+    dn = []
+    for e in range(E):
+        for t in range(H // 32):
+            units = dd[e, 32 * t:32 * t + 32].reshape(32, nbI, 16)
+            perm = np.stack([units[r, np.arange(nbI) ^ (r & mI)] for r in range(32)])
+            dn.append(perm.reshape(-1))
+            dn.append(ds[e, 32 * t:32 * t + 32].reshape(-1))
+    return np.concatenate(gu), np.concatenate(dn)
+
+
+@pytest.mark.parametrize("E,H,Inter", [(3, 256, 64), (2, 192, 192), (2, 2560, 768)])
+def test_pack_matches_documented_layout(B, E, H, Inter):
+    g = torch.Generator().manual_seed(E * 1000 + H + Inter)
+    banks = []
+    for rows, cols in ((Inter, H), (Inter, H), (H, Inter)):
+        w = (torch.randn((E, rows, cols), generator=g) * 0.02).to(torch.bfloat16)
+        banks.append(B.moe_quantize_mxfp4(w.cuda()))
+    packed = B.moe_pack_experts(tuple(banks))
+    torch.cuda.synchronize()
+    assert packed.fmt == B.Format.MXFP4_MOE_PACKED
+    canon = [(b.data.cpu().numpy(), b.scales.cpu().numpy()) for b in banks]
+    want_gu, want_dn = expected_packed(*canon)
+    assert np.array_equal(packed.gateup.cpu().numpy(), want_gu)
+    assert np.array_equal(packed.down.cpu().numpy(), want_dn)
+    assert packed.nbytes() == sum(b.nbytes() for b in banks)  # same bytes, regrouped
+
+
+def test_pack_of_ling_shared_expert(B):
+    s = I.LING_MOE
+    banks = tuple(B.moe_quantize_mxfp4(I.expert_matrix(0, s, "shared", k).cuda()) for k in ("gate", "up", "down"))
+    packed = B.moe_pack_experts(banks)
+    canon = [(b.data.cpu().numpy(), b.scales.cpu().numpy()) for b in banks]
+    want_gu, want_dn = expected_packed(*canon)
+    assert np.array_equal(packed.gateup.cpu().numpy(), want_gu)
+    assert np.array_equal(packed.down.cpu().numpy(), want_dn)

@@ -54,7 +54,7 @@ class Stack:
         for _ in range(steps):
             B.moe_embed_gather(self.table_dev, ids, x, ids_stride=1)
             for layer in self.layers:
-                B.moe_decode(x, layer.router_w_dev, None, layer.bank, layer.shared, self.moe.top_k, y)
+                B.moe_decode(x, layer.router_w_dev, None, layer.packed, layer.packed_shared, self.moe.top_k, y)
                 B.moe_rmsnorm_bf16(y, x, EPS)
             B.lmhead_decode(x, self.head, 1, tk, tv)
             ids = tk.clone()
