@@ -120,9 +120,11 @@ __device__ __forceinline__ uint32_t e2m1x8_odd_to_e4m3x4(uint32_t w) {
 }
 
 // E4M3 x E4M3 -> fp32 tensor-core MMA, m16n8k32 (A row-major 16x32, B 32x8).
+// Not volatile: it has no effect beyond its outputs, so the compiler may
+// interleave independent MMAs instead of issuing them in source order.
 __device__ __forceinline__ void mma_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -164,8 +166,9 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // Ordering of (value, index) candidates: larger value first, then lower index.
+// Branch-free: evaluated with predicates, never a jump.
 __device__ __forceinline__ bool better(float va, int32_t ia, float vb, int32_t ib) {
-  return va > vb || (va == vb && ia < ib);
+  return (va > vb) | ((va == vb) & (ia < ib));
 }
 
 // Warp-wide best (value, index) under `better`; every lane gets the result.

@@ -53,18 +53,17 @@
 namespace moe {
 namespace {
 
-constexpr int kCons = 8;                   // consumer warps
+constexpr int kCons = 16;                  // consumer warps
 constexpr int kProd = kCons;               // producer warp index
 constexpr int kGuRows = 8;                 // gate rows (and up rows) per phase-1 item
 constexpr int kDnRows = 32;                // output rows per phase-2 item
 constexpr int kStages = 6;
-constexpr int kMaxGuBlocksPerWarp = 16;    // H <= 16 * 8 * 32 = 4096
-constexpr int kMaxDnBlocksPerWarp = 4;     // I <= 4 * 8 * 32 = 1024
+constexpr int kMaxGuBlocksPerWarp = 8;     // H <= 8 * 16 * 32 = 4096
+constexpr int kMaxDnBlocksPerWarp = 2;     // I <= 2 * 16 * 32 = 1024
 // The x fragments of the gate/up GEMV live in registers for the whole kernel:
-// the kernel is instantiated for these blocks-per-warp buckets and the
-// launcher picks the smallest that fits.  The down GEMV's fragments are
-// rebuilt per item and sized for the largest case.
-constexpr int kGuBuckets[] = {1, 2, 4, 8, 10, 16};
+// the kernel is instantiated for blocks-per-warp buckets (GuBuckets, at the
+// launcher) and a launch picks the smallest that fits.  The down GEMV's
+// fragments are rebuilt per item and sized for the largest case.
 constexpr int kHParts = 3;  // E4M3 parts carrying h into the down GEMV
 
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
@@ -87,6 +86,29 @@ __device__ __forceinline__ int pow2_sigma(float amax) {
 }
 
 __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
+
+// v rounded to 4 significant bits (E4M3's precision), to nearest even, as an
+// fp32 value: integer operations only.  For |v| in E4M3's normal range
+// [2^-6, 448] the result is exactly an E4M3 value.
+__device__ __forceinline__ float round_sig4(float v) {
+  uint32_t b = __float_as_uint(v);
+  b += 0x7ffffu + ((b >> 20) & 1u);
+  return __uint_as_float(b & 0xfff00000u);
+}
+
+// Four fp32 values -> three E4M3 parts (byte j of each part belongs to value
+// j) whose sum carries 12 significant bits of each value: each part is the
+// remainder so far rounded to 4 significant bits.  Parts in E4M3's normal
+// range are encoded exactly; only parts below 2^-6 (values at least 2^-13
+// below their block's largest) are rounded by the encoding.
+__device__ __forceinline__ void split3_e4m3x4(float a, float b, float c, float d, uint32_t (&p)[3]) {
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    const float ra = round_sig4(a), rb = round_sig4(b), rc = round_sig4(c), rd = round_sig4(d);
+    p[q] = f32x2_to_e4m3x2(ra, rb) | (f32x2_to_e4m3x2(rc, rd) << 16);
+    a -= ra; b -= rb; c -= rc; d -= rd;
+  }
+}
 
 // ---- routing: top-8 of up to 1,024 logits in one warp ----
 // (value, expert) pairs under `better`: larger value first, lower id on ties.
@@ -130,29 +152,23 @@ __device__ __forceinline__ void merge8(VI (&R)[8], const VI (&S)[8]) {
 // The best 8 of logits[0..E) (E <= 1024), sorted, in every lane of the warp.
 // Logits that are NaN or -inf count as -FLT_MAX, so that every real expert
 // ranks above the padding entries (-FLT_MAX, INT32_MAX): with E >= 8 the
-// result holds only experts in [0, E).
+// result holds only experts in [0, E).  Each lane sorts its logits 8 at a time
+// (loaded chunk by chunk, to keep few registers live) into its running best 8;
+// a butterfly of merges then gives every lane the warp's best 8.
 __device__ __forceinline__ void warp_top8(const float* logits, int E, int lane, VI (&R)[8]) {
-  float lv[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = lane + 32 * i;
-    const float v = e < E ? __ldcg(logits + e) : -FLT_MAX;
-    lv[i] = v > -FLT_MAX ? v : -FLT_MAX;
-  }
 #pragma unroll
   for (int j = 0; j < 8; ++j) R[j] = VI{-FLT_MAX, INT32_MAX};
+#pragma unroll 1
+  for (int ch = 0; ch * 256 < E; ++ch) {  // this lane's values lane + 32 i, i in [8 ch, 8 ch + 8)
+    VI S[8];
 #pragma unroll
-  for (int ch = 0; ch < 4; ++ch) {  // this lane's values, 8 at a time
-    if (ch * 256 < E) {
-      VI S[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = lane + 32 * (8 * ch + j);
-        S[j] = e < E ? VI{lv[8 * ch + j], e} : VI{-FLT_MAX, INT32_MAX};
-      }
-      sort8(S);
-      merge8(R, S);
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * (8 * ch + j);
+      const float v = e < E ? __ldcg(logits + e) : -FLT_MAX;
+      S[j] = e < E ? VI{v > -FLT_MAX ? v : -FLT_MAX, e} : VI{-FLT_MAX, INT32_MAX};
     }
+    sort8(S);
+    merge8(R, S);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {  // butterfly: both partners end with the same list
@@ -164,83 +180,6 @@ __device__ __forceinline__ void warp_top8(const float* logits, int E, int lane, 
     }
     merge8(R, P);
   }
-}
-
-// Top-k (k <= 8) of one token's logits[0..E) by one warp, with ids and
-// values in rank order written to ids[0..k) and vals[0..k) (shared memory).
-// A filter first: the k-th best of the 32 lanes' own best entries, L, is a
-// lower bound on the k-th best overall (those are k real entries), so only
-// entries not worse than L can be selected -- typically a dozen.  They are
-// ranked by counting.  With more than 64 of them (heavy ties) the sorting
-// network above ranks all E entries instead.  Logits that are NaN or -inf
-// count as -FLT_MAX; ties go to the lower expert id.
-__device__ __forceinline__ void warp_route(const float* logits, int E, int k, int lane, float* cv, int32_t* ci,
-                                           int32_t* ids, float* vals) {
-  float lv[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = lane + 32 * i;
-    const float v = e < E ? __ldcg(logits + e) : -FLT_MAX;
-    lv[i] = v > -FLT_MAX ? v : -FLT_MAX;
-  }
-  float mv = -FLT_MAX;
-  int32_t mi = INT32_MAX;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E && better(lv[i], e, mv, mi)) { mv = lv[i]; mi = e; }
-  }
-  int rank = 0;  // of this lane's best among the 32 lanes' bests
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const float ov = __shfl_sync(0xffffffffu, mv, j);
-    const int32_t oi = __shfl_sync(0xffffffffu, mi, j);
-    rank += better(ov, oi, mv, mi);
-  }
-  // padding lanes (E < 32) tie among themselves but rank after all real ones,
-  // and E >= k, so exactly one lane has rank k - 1
-  const uint32_t sel = __ballot_sync(0xffffffffu, rank == k - 1);
-  const int src = sel ? __ffs(sel) - 1 : 0;
-  const float Lv = sel ? __shfl_sync(0xffffffffu, mv, src) : -FLT_MAX;
-  const int32_t Li = sel ? __shfl_sync(0xffffffffu, mi, src) : INT32_MAX;
-  int cnt = 0;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = lane + 32 * i;
-    cnt += (e < E && !better(Lv, Li, lv[i], e)) ? 1 : 0;
-  }
-  int off = cnt;  // inclusive prefix sum over lanes
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(0xffffffffu, off, o);
-    if (lane >= o) off += t;
-  }
-  const int n = __shfl_sync(0xffffffffu, off, 31);
-  off -= cnt;
-  if (n <= 64) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !better(Lv, Li, lv[i], e)) { cv[off] = lv[i]; ci[off] = e; ++off; }
-    }
-    __syncwarp();
-    for (int q = lane; q < n; q += 32) {
-      const float qv = cv[q];
-      const int32_t qi = ci[q];
-      int r = 0;
-      for (int o = 0; o < n; ++o) r += better(cv[o], ci[o], qv, qi);
-      if (r < k) { ids[r] = qi; vals[r] = qv; }
-    }
-  } else {
-    VI R[8];
-    warp_top8(logits, E, lane, R);
-    if (lane == 0) {
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (r < k) { ids[r] = R[r].i; vals[r] = R[r].v; }
-    }
-  }
-  __syncwarp();
 }
 
 struct FusedArgs {
@@ -285,7 +224,8 @@ constexpr int kRed = 4;                    // partial-sum buffers between consum
 constexpr int kEpi = kCons + 1;            // first epilogue warp
 constexpr int kNumEpi = 2;                 // epilogue warps; item i goes to epilogue warp i % kNumEpi
 constexpr int kThreadsAll = (kCons + 1 + kNumEpi) * 32;
-constexpr int kRouterF4 = 16;              // float4 loads per lane per half router row: H <= 4096
+constexpr int kRouterSplit = 4;           // consumer warps per router row
+constexpr int kRouterF4 = 8;               // float4 loads per lane per quarter router row: H <= 4096
 
 struct SmemCtl {
   uint64_t full[kStages];
@@ -295,12 +235,10 @@ struct SmemCtl {
   uint64_t routed;                         // slot table ready (producer and epilogue warps wait on it)
   uint64_t h_ready;                        // every CTA's h written (consumers wait on it)
   alignas(16) float red[kRed][kCons][32][8];  // per-item partials (float4 access)
-  float logit_part[kCons][4];              // router: half-row partial sums
+  float logit_part[kCons][4];              // router: quarter-row partial sums
   int32_t ids[4][8];
   float wts[4][8];
   float topv[4][8];
-  float cand_v[4][64];                     // routing candidates, per token
-  int32_t cand_i[4][64];
   int32_t slot_expert[MoeWs::kMaxSlots];
   uint32_t slot_mask[MoeWs::kMaxSlots];
   float slot_w[MoeWs::kMaxSlots][4];
@@ -554,19 +492,20 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
   } else {
     // ============================== consumers =============================
     const int g = lane >> 2, tq = lane & 3;
-    const int cw = warp;  // consumer warp index 0..7
+    const int cw = warp;  // consumer warp index 0..kCons-1
 
-    // ---- phase 0: router rows of this CTA (2 warps per expert row) ----
+    // ---- phase 0: router rows of this CTA (4 warps per expert row) ----
     const int e_begin = (int)((int64_t)E * c / G), e_end = (int)((int64_t)E * (c + 1) / G);
-    for (int base = e_begin; base < e_end; base += kCons / 2) {
-      const int e = base + (cw >> 1), half = cw & 1;
-      const int hw = H / 2;
+    constexpr int kRowsPerRound = kCons / kRouterSplit;
+    for (int base = e_begin; base < e_end; base += kRowsPerRound) {
+      const int e = base + cw / kRouterSplit, part = cw % kRouterSplit;
+      const int hw = H / kRouterSplit;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
       if (e < e_end) {
-        const float* row = a.router_w + (size_t)e * H + half * hw;
+        const float* row = a.router_w + (size_t)e * H + part * hw;
         float4 wv[kRouterF4];
 #pragma unroll
-        for (int i = 0; i < kRouterF4; ++i) {  // every load of the half row in flight at once
+        for (int i = 0; i < kRouterF4; ++i) {  // every load of the quarter row in flight at once
           const int jj = lane * 4 + i * 128;
           wv[i] = jj < hw ? ld_stream_f4(row + jj) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
@@ -577,7 +516,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
               if (m < M) {
-                const uint2 xv = *reinterpret_cast<const uint2*>(a.x + (size_t)m * H + half * hw + jj);
+                const uint2 xv = *reinterpret_cast<const uint2*>(a.x + (size_t)m * H + part * hw + jj);
                 acc[m] += wv[i].x * bf16_bits_to_f32(xv.x & 0xffffu) + wv[i].y * bf16_bits_to_f32(xv.x >> 16) +
                           wv[i].z * bf16_bits_to_f32(xv.y & 0xffffu) + wv[i].w * bf16_bits_to_f32(xv.y >> 16);
               }
@@ -591,10 +530,12 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
         if (lane == 0) C.logit_part[cw][m] = v;
       }
       consumer_bar_sync();
-      if (threadIdx.x < (kCons / 2) * 4) {
-        const int ee = base + threadIdx.x / 4, m = threadIdx.x % 4;
+      if (threadIdx.x < kRowsPerRound * 4) {
+        const int rr = threadIdx.x / 4, m = threadIdx.x % 4, ee = base + rr;
         if (ee < e_end && m < M) {
-          float l = C.logit_part[2 * (threadIdx.x / 4)][m] + C.logit_part[2 * (threadIdx.x / 4) + 1][m];
+          float l = 0.f;
+#pragma unroll
+          for (int q = 0; q < kRouterSplit; ++q) l += C.logit_part[rr * kRouterSplit + q][m];
           if (a.router_bias) l += a.router_bias[ee];
           ws.logits[(size_t)m * E + ee] = l;
         }
@@ -610,17 +551,15 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     // token g: the even ones fill k-slots 4tq..4tq+3 (b0), the odd ones
     // 16+4tq.. (b1), matching the even/odd split of the weight nibbles.  The
     // token, scaled by 2^sigma, is carried exactly by two E4M3 parts (hi, lo).
-    const int nbw_gu = (geo.nbH + kCons - 1) / kCons;
-    const int b0_gu = cw * nbw_gu;
-    uint32_t bx[kGuB][2][2];  // [block][part][b0, b1]
+    uint32_t bx[kGuB][2][2];  // [block][part][b0, b1]; this warp's blocks are cw, cw + kCons, ...
     {
       const bool live = g < M;
       const float scl = live ? exp2i(C.sigma_x[g]) : 0.f;
 #pragma unroll
       for (int bi = 0; bi < kGuB; ++bi) {
-        const int blk = b0_gu + bi;
+        const int blk = cw + kCons * bi;
         uint32_t pe[2] = {0u, 0u}, po[2] = {0u, 0u};
-        if (live && bi < nbw_gu && blk < geo.nbH) {
+        if (live && blk < geo.nbH) {
           const uint4 q = *reinterpret_cast<const uint4*>(a.x + (size_t)g * H + blk * 32 + tq * 8);
           const float v0 = bf16_bits_to_f32(q.x & 0xffffu) * scl, v1 = bf16_bits_to_f32(q.x >> 16) * scl;
           const float v2 = bf16_bits_to_f32(q.y & 0xffffu) * scl, v3 = bf16_bits_to_f32(q.y >> 16) * scl;
@@ -636,7 +575,13 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
         }
       }
     }
-
+    // Shared-memory offsets of this lane's words.  Block blk = cw + kCons*bi of
+    // row r sits at unit blk ^ (r & mask) = kCons*bi + (cw ^ (r & mask)) (the
+    // mask is below 8 and cw below kCons), so every block is a constant stride
+    // from the lane's base; rows g and 8+g share the permutation.
+    const int gu_rowb = H / 2;
+    const int gu_lane = g * gu_rowb + ((cw ^ (g & geo.mH)) * 16) + tq * 4;  // gate row g; up row 8+g adds 8 rows
+    const int gu_scl = 16 * gu_rowb + g * geo.nbH + cw;                    // gate scale; up scale adds 8 rows
     int it = 0;     // ring position
     int nitem = 0;  // items handed to the epilogue warps
     auto hand_off = [&](const float (&v)[8]) {
@@ -655,19 +600,15 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       const int st = it % kStages;
       const bool ok = bounded_wait(&C.full[st], (uint32_t)((it / kStages) & 1));
       const uint8_t* base = ring + (size_t)st * geo.stage_bytes;
-      const int rowb = H / 2;
-      const uint8_t* gsc = base + 16 * rowb;
-      const uint8_t* usc = gsc + kGuRows * geo.nbH;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (ok) {
 #pragma unroll
         for (int bi = 0; bi < kGuB; ++bi) {
-          const int blk = b0_gu + bi;
-          if (bi < nbw_gu && blk < geo.nbH) {
-            const uint32_t gw = lds32(base + g * rowb + ((blk ^ (g & geo.mH)) * 16) + tq * 4);
-            const uint32_t uw = lds32(base + (8 + g) * rowb + ((blk ^ ((8 + g) & geo.mH)) * 16) + tq * 4);
-            const float sg = e8m0_to_f32(gsc[g * geo.nbH + blk]);
-            const float su = e8m0_to_f32(usc[g * geo.nbH + blk]);
+          if (cw + kCons * bi < geo.nbH) {
+            const uint32_t gw = lds32(base + gu_lane + 256 * bi);
+            const uint32_t uw = lds32(base + gu_lane + 8 * gu_rowb + 256 * bi);
+            const float sg = e8m0_to_f32(base[gu_scl + kCons * bi]);
+            const float su = e8m0_to_f32(base[gu_scl + 8 * geo.nbH + kCons * bi]);
             // A: gate row g (a0, a2) and up row g (a1, a3), 32 elements = one MX block
             const uint32_t ge = e2m1x8_even_to_e4m3x4(gw), go = e2m1x8_odd_to_e4m3x4(gw);
             const uint32_t ue = e2m1x8_even_to_e4m3x4(uw), uo = e2m1x8_odd_to_e4m3x4(uw);
@@ -688,10 +629,30 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     };
 
     // ---- phase-2 item: partial sums of 32 output rows of one slot's down matrix ----
-    const int nbw_dn = (geo.nbI + kCons - 1) / kCons;
-    const int b0_dn = cw * nbw_dn;
-    auto down_item = [&](int slot) {
+    const int dn_rowb = I / 2;
+    const int dn_lane = g * dn_rowb + ((cw ^ (g & geo.mI)) * 16) + tq * 4;  // rows 16tt + g (+ 8) share it
+    const int dn_scl = kDnRows * dn_rowb + g * geo.nbI + cw;
+    // h of token g for this warp's blocks of one slot's down item (issued one
+    // item ahead, so the L2 round trip overlaps the previous item)
+    auto load_h = [&](int slot, float (&v)[kDnB][8]) {
       const uint32_t mask = slot == 0 ? 0xfu : C.slot_mask[slot];
+      const bool live = !poisoned() && g < M && (mask >> g & 1u);
+#pragma unroll
+      for (int bi = 0; bi < kDnB; ++bi) {
+        const int blk = cw + kCons * bi;
+        if (live && blk < geo.nbI) {
+          const float* hp = ws.h + ((size_t)slot * 4 + g) * I + blk * 32 + tq * 8;
+          const float4 v0 = __ldcg(reinterpret_cast<const float4*>(hp));
+          const float4 v1 = __ldcg(reinterpret_cast<const float4*>(hp + 4));
+          v[bi][0] = v0.x; v[bi][1] = v0.y; v[bi][2] = v0.z; v[bi][3] = v0.w;
+          v[bi][4] = v1.x; v[bi][5] = v1.y; v[bi][6] = v1.z; v[bi][7] = v1.w;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) v[bi][q] = 0.f;
+        }
+      }
+    };
+    auto down_item = [&](const float (&v)[kDnB][8]) {
       // B fragments: h of token g, per 32-element block scaled by a power of
       // two that puts the block's largest magnitude in [2^7, 2^8), then split
       // into three E4M3 parts (12 significant bits), even/odd permuted as for
@@ -699,63 +660,42 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       // weights' 2^-6) on the MMA results.
       uint32_t bh[kDnB][kHParts][2];
       float f0[kDnB], f1[kDnB];
-      {
-        const bool live = !poisoned() && g < M && (mask >> g & 1u);
-        float v[kDnB][8];
 #pragma unroll
-        for (int bi = 0; bi < kDnB; ++bi) {  // all loads first
-          const int blk = b0_dn + bi;
-          if (live && bi < nbw_dn && blk < geo.nbI) {
-            const float* hp = ws.h + ((size_t)slot * 4 + g) * I + blk * 32 + tq * 8;
-            const float4 v0 = __ldcg(reinterpret_cast<const float4*>(hp));
-            const float4 v1 = __ldcg(reinterpret_cast<const float4*>(hp + 4));
-            v[bi][0] = v0.x; v[bi][1] = v0.y; v[bi][2] = v0.z; v[bi][3] = v0.w;
-            v[bi][4] = v1.x; v[bi][5] = v1.y; v[bi][6] = v1.z; v[bi][7] = v1.w;
-          } else {
+      for (int bi = 0; bi < kDnB; ++bi) {
+        float mx = 0.f;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) v[bi][q] = 0.f;
-          }
-        }
+        for (int q = 0; q < 8; ++q) mx = fmaxf(mx, fabsf(v[bi][q]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));  // the block of token g spans lanes 4g..4g+3
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const int sig = pow2_sigma(mx);
+        const float scl = exp2i(sig);
+        const float f = exp2i(6 - sig);
+        f0[bi] = __shfl_sync(0xffffffffu, f, 8 * tq);      // token 2tq lives in lanes 8tq..8tq+3
+        f1[bi] = __shfl_sync(0xffffffffu, f, 8 * tq + 4);  // token 2tq+1
+        uint32_t pe[kHParts], po[kHParts];
+        split3_e4m3x4(v[bi][0] * scl, v[bi][2] * scl, v[bi][4] * scl, v[bi][6] * scl, pe);
+        split3_e4m3x4(v[bi][1] * scl, v[bi][3] * scl, v[bi][5] * scl, v[bi][7] * scl, po);
 #pragma unroll
-        for (int bi = 0; bi < kDnB; ++bi) {
-          float mx = 0.f;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) mx = fmaxf(mx, fabsf(v[bi][q]));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));  // the block of token g spans lanes 4g..4g+3
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          const int sig = pow2_sigma(mx);
-          const float scl = exp2i(sig);
-          const float f = exp2i(6 - sig);
-          f0[bi] = __shfl_sync(0xffffffffu, f, 8 * tq);      // token 2tq lives in lanes 8tq..8tq+3
-          f1[bi] = __shfl_sync(0xffffffffu, f, 8 * tq + 4);  // token 2tq+1
-          uint32_t pe[kHParts], po[kHParts];
-          split_e4m3x4<kHParts>(v[bi][0] * scl, v[bi][2] * scl, v[bi][4] * scl, v[bi][6] * scl, pe);
-          split_e4m3x4<kHParts>(v[bi][1] * scl, v[bi][3] * scl, v[bi][5] * scl, v[bi][7] * scl, po);
-#pragma unroll
-          for (int part = 0; part < kHParts; ++part) {
-            bh[bi][part][0] = pe[part];
-            bh[bi][part][1] = po[part];
-          }
+        for (int part = 0; part < kHParts; ++part) {
+          bh[bi][part][0] = pe[part];
+          bh[bi][part][1] = po[part];
         }
       }
       const int st = it % kStages;
       const bool ok = bounded_wait(&C.full[st], (uint32_t)((it / kStages) & 1));
       const uint8_t* base = ring + (size_t)st * geo.stage_bytes;
-      const int rowb = I / 2;
-      const uint8_t* dsc = base + kDnRows * rowb;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (ok) {
 #pragma unroll
         for (int tt = 0; tt < 2; ++tt) {
 #pragma unroll
           for (int bi = 0; bi < kDnB; ++bi) {
-            const int blk = b0_dn + bi;
-            if (bi < nbw_dn && blk < geo.nbI) {
-              const int r_lo = 16 * tt + g, r_hi = r_lo + 8;
-              const uint32_t wa = lds32(base + r_lo * rowb + ((blk ^ (r_lo & geo.mI)) * 16) + tq * 4);
-              const uint32_t wb = lds32(base + r_hi * rowb + ((blk ^ (r_hi & geo.mI)) * 16) + tq * 4);
-              const float sa = e8m0_to_f32(dsc[r_lo * geo.nbI + blk]);
-              const float sb = e8m0_to_f32(dsc[r_hi * geo.nbI + blk]);
+            if (cw + kCons * bi < geo.nbI) {
+              const int off = dn_lane + 16 * tt * dn_rowb + 256 * bi;
+              const uint32_t wa = lds32(base + off);
+              const uint32_t wb = lds32(base + off + 8 * dn_rowb);
+              const float sa = e8m0_to_f32(base[dn_scl + 16 * tt * geo.nbI + kCons * bi]);
+              const float sb = e8m0_to_f32(base[dn_scl + (16 * tt + 8) * geo.nbI + kCons * bi]);
               const uint32_t ae = e2m1x8_even_to_e4m3x4(wa), ao = e2m1x8_odd_to_e4m3x4(wa);
               const uint32_t be = e2m1x8_even_to_e4m3x4(wb), bo = e2m1x8_odd_to_e4m3x4(wb);
               float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -786,8 +726,12 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
         consumer_bar_sync();
         if (cw < M) {  // warp m routes token m
           const int m = cw;
-          warp_route(ws.logits + (size_t)m * E, E, a.top_k, lane, C.cand_v[m], C.cand_i[m], C.ids[m], C.topv[m]);
+          VI R[8];
+          warp_top8(ws.logits + (size_t)m * E, E, lane, R);
           if (lane == 0) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+              if (r < a.top_k) { C.ids[m][r] = R[r].i; C.topv[m][r] = R[r].v; }
             float z = 0.f;
             for (int r = 0; r < a.top_k; ++r) z += expf(C.topv[m][r] - C.topv[m][0]);
             for (int r = 0; r < a.top_k; ++r) C.wts[m][r] = expf(C.topv[m][r] - C.topv[m][0]) / z;
@@ -802,7 +746,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
           const bool act = lane < n_in;
           const int m = act ? lane / k : 0, r = act ? lane - (lane / k) * k : 0;
           int32_t ex = act ? C.ids[m][r] : -1 - lane;  // idle lanes get ids of their own
-          if (act && (ex < 0 || ex >= E)) {  // cannot happen (see warp_route); never index out of range
+          if (act && (ex < 0 || ex >= E)) {  // cannot happen (see warp_top8); never index out of range
             report(ws.hdr, MOE_ERR_DEVICE_CHECK);
             ex = 0;
           }
@@ -849,7 +793,17 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     // phase 2 reads every CTA's h: wait until the epilogue warps have seen the
     // grid barrier that follows phase 1
     bounded_wait(&C.h_ready, 0);
-    for (int j = 0; j < n2; ++j) down_item((c + j * G) / geo.n_tiles);
+    float hv[kDnB][8];
+    if (n2 > 0) load_h(c / geo.n_tiles, hv);
+    for (int j = 0; j < n2; ++j) {
+      float cur[kDnB][8];
+#pragma unroll
+      for (int bi = 0; bi < kDnB; ++bi)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) cur[bi][q] = hv[bi][q];
+      if (j + 1 < n2) load_h((c + (j + 1) * G) / geo.n_tiles, hv);
+      down_item(cur);
+    }
   }
 }
 
@@ -889,22 +843,26 @@ static cudaError_t launch_fused_t(const FusedArgs& a, size_t smem, cudaStream_t 
   return e;
 }
 
+// The instantiations of the gate/up blocks-per-warp buckets, smallest first;
+// a launch takes the first bucket that covers ceil((H / 32) / kCons).
+template <int... kBuckets>
+struct GuDispatch {
+  static cudaError_t run(int, const FusedArgs&, size_t, cudaStream_t) { return cudaErrorInvalidValue; }
+};
+template <int kB, int... kRest>
+struct GuDispatch<kB, kRest...> {
+  static cudaError_t run(int need, const FusedArgs& a, size_t smem, cudaStream_t st) {
+    return need <= kB ? launch_fused_t<kB>(a, smem, st) : GuDispatch<kRest...>::run(need, a, smem, st);
+  }
+};
+using GuBuckets = GuDispatch<1, 2, 4, 5, kMaxGuBlocksPerWarp>;
+
 cudaError_t launch_moe_fused(const MoeArgs& m, cudaStream_t st) {
   FusedArgs a{m.x, m.router_w, m.router_bias, m.bank, m.shared, m.M, m.top_k, m.E, m.H, m.I,
               m.out, m.ids_out, m.w_out, m.ws};
   const size_t smem = moe_fused_smem_bytes(m.H, m.I);
   const int need_gu = (m.H / 32 + kCons - 1) / kCons;
-  int gub = 0;
-  for (int b : kGuBuckets) if (!gub && b >= need_gu) gub = b;
-  switch (gub) {
-    case 1: return launch_fused_t<1>(a, smem, st);
-    case 2: return launch_fused_t<2>(a, smem, st);
-    case 4: return launch_fused_t<4>(a, smem, st);
-    case 8: return launch_fused_t<8>(a, smem, st);
-    case 10: return launch_fused_t<10>(a, smem, st);
-    case 16: return launch_fused_t<16>(a, smem, st);
-    default: return cudaErrorInvalidValue;
-  }
+  return GuBuckets::run(need_gu, a, smem, st);
 }
 
 }  // namespace moe
