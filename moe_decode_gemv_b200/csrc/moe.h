@@ -25,6 +25,9 @@ struct MoeWs {
   WsHeader* hdr;
   float* logits;        // [M][E]
   float* h;             // [kMaxSlots][4][I]: silu(gate) * up per slot and token
+  uint8_t* hq;          // [kMaxSlots][4][I/32][3][32]: h per 32-element block as three E4M3 parts,
+                        //   bytes in MMA B-fragment order (see moe_fused.cu)
+  float* hf;            // [kMaxSlots][4][I/32]: 2^(6 - sigma) of each block (undoes its scale)
   float* ypart;         // [kMaxSlots][4][H]: down(h) per slot and token, before the weighted combine
 
   static size_t align(size_t v) { return (v + 255) & ~size_t(255); }
@@ -33,6 +36,8 @@ struct MoeWs {
     size_t b = align(sizeof(WsHeader));
     b += align((size_t)4 * E * sizeof(float));
     b += align((size_t)kMaxSlots * 4 * I * sizeof(float));
+    b += align((size_t)kMaxSlots * 4 * (I / 32) * 3 * 32);
+    b += align((size_t)kMaxSlots * 4 * (I / 32) * sizeof(float));
     b += align((size_t)kMaxSlots * 4 * H * sizeof(float));
     return b;
   }
@@ -43,6 +48,8 @@ struct MoeWs {
     w.hdr = reinterpret_cast<WsHeader*>(p); p += align(sizeof(WsHeader));
     w.logits = reinterpret_cast<float*>(p); p += align((size_t)4 * E * sizeof(float));
     w.h = reinterpret_cast<float*>(p); p += align((size_t)kMaxSlots * 4 * I * sizeof(float));
+    w.hq = p; p += align((size_t)kMaxSlots * 4 * (I / 32) * 3 * 32);
+    w.hf = reinterpret_cast<float*>(p); p += align((size_t)kMaxSlots * 4 * (I / 32) * sizeof(float));
     w.ypart = reinterpret_cast<float*>(p);
     return w;
   }

@@ -27,6 +27,10 @@
 //    one slot form one 16-row MMA tile; h = silu(g) * u is written in fp32.
 //  * A grid barrier publishes h.  No fence or atomic sits on the per-item
 //    path: the producer streams the down tiles meanwhile.
+//  * Split pass: one warp per (slot, token, 32-element block) of h scales the
+//    block by a power of two and writes it as three E4M3 parts in MMA
+//    fragment order -- once, instead of once per down item that reads it.
+//    Another grid barrier publishes the parts.
 //  * Phase 2: items of 32 output rows of one slot's down matrix multiply by h
 //    and write per-slot partial outputs.  After one more grid barrier each
 //    CTA sums, for the 32-row tiles it owns, the slot partials in slot order:
@@ -94,20 +98,6 @@ __device__ __forceinline__ float round_sig4(float v) {
   uint32_t b = __float_as_uint(v);
   b += 0x7ffffu + ((b >> 20) & 1u);
   return __uint_as_float(b & 0xfff00000u);
-}
-
-// Four fp32 values -> three E4M3 parts (byte j of each part belongs to value
-// j) whose sum carries 12 significant bits of each value: each part is the
-// remainder so far rounded to 4 significant bits.  Parts in E4M3's normal
-// range are encoded exactly; only parts below 2^-6 (values at least 2^-13
-// below their block's largest) are rounded by the encoding.
-__device__ __forceinline__ void split3_e4m3x4(float a, float b, float c, float d, uint32_t (&p)[3]) {
-#pragma unroll
-  for (int q = 0; q < 3; ++q) {
-    const float ra = round_sig4(a), rb = round_sig4(b), rc = round_sig4(c), rd = round_sig4(d);
-    p[q] = f32x2_to_e4m3x2(ra, rb) | (f32x2_to_e4m3x2(rc, rd) << 16);
-    a -= ra; b -= rb; c -= rc; d -= rd;
-  }
 }
 
 // ---- routing: top-8 of up to 1,024 logits in one warp ----
@@ -234,6 +224,7 @@ struct SmemCtl {
   uint64_t red_empty[kRed];
   uint64_t routed;                         // slot table ready (producer and epilogue warps wait on it)
   uint64_t h_ready;                        // every CTA's h written (consumers wait on it)
+  uint64_t parts_ready;                    // this CTA passed the split-pass barrier (epilogue waits on it)
   alignas(16) float red[kRed][kCons][32][8];  // per-item partials (float4 access)
   float logit_part[kCons][4];              // router: quarter-row partial sums
   int32_t ids[4][8];
@@ -257,8 +248,12 @@ __device__ __forceinline__ void epilogue_bar_sync() {
 // Grid barrier on one word (all CTAs are resident: cooperative launch).  The
 // first CTA adds 2^31 - (G - 1), the others 1, so the top bit flips exactly
 // when all G have arrived and the low bits return to where they were: the
-// same word serves every barrier of every call.  Arrival publishes the
-// caller's earlier writes (fence first); the wait is bounded.
+// same word serves every barrier of every call.  A CTA may arrive at barrier
+// n + 1 only after it has seen barrier n complete -- otherwise its early
+// arrival would count toward barrier n -- which the warps that arrive for a
+// CTA (consumers: router, split pass; epilogue: h, partial outputs) ensure
+// with the CTA-local mbarriers h_ready and parts_ready.  Arrival publishes
+// the caller's earlier writes (fence first); the wait is bounded.
 __device__ __forceinline__ uint32_t grid_arrive(uint32_t* word, int c, int G) {
   __threadfence();
   return atomicAdd(word, c == 0 ? 0x80000000u - (uint32_t)(G - 1) : 1u);
@@ -303,6 +298,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     }
     mbar_init(&C.routed, 1);
     mbar_init(&C.h_ready, 1);
+    mbar_init(&C.parts_ready, 1);
     fence_mbar_init();
     C.poison = 0;
   }
@@ -467,6 +463,10 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     // h of every CTA is written: release the consumers into phase 2
     epilogue_grid_barrier();
     if (ew == 0 && lane == 0) mbar_arrive(&C.h_ready);
+    // This CTA's next arrival on the grid-barrier word must follow its
+    // consumers' arrival at the split-pass barrier, even when it has no
+    // phase-2 items: arrivals on the word stay in barrier order.
+    bounded_wait(&C.parts_ready, 0);
     for (int j = 0; j < n2; ++j, ++idx) {
       if (idx % kNumEpi != ew) continue;
       const int q = c + j * G;
@@ -632,54 +632,42 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     const int dn_rowb = I / 2;
     const int dn_lane = g * dn_rowb + ((cw ^ (g & geo.mI)) * 16) + tq * 4;  // rows 16tt + g (+ 8) share it
     const int dn_scl = kDnRows * dn_rowb + g * geo.nbI + cw;
-    // h of token g for this warp's blocks of one slot's down item (issued one
-    // item ahead, so the L2 round trip overlaps the previous item)
-    auto load_h = [&](int slot, float (&v)[kDnB][8]) {
+    // The B fragments of a down item: h of token g for this warp's blocks of
+    // one slot, already split into three E4M3 parts by the split pass
+    // (uint2 = the lane's even and odd 4-byte groups of one part) and the
+    // factor that undoes the block's scale.  Issued one item ahead, so the L2
+    // round trip overlaps the previous item.
+    struct HFrag {
+      uint2 q[kDnB][kHParts];
+      float f[kDnB];
+    };
+    auto load_h = [&](int slot, HFrag& hf) {
       const uint32_t mask = slot == 0 ? 0xfu : C.slot_mask[slot];
       const bool live = !poisoned() && g < M && (mask >> g & 1u);
 #pragma unroll
       for (int bi = 0; bi < kDnB; ++bi) {
         const int blk = cw + kCons * bi;
+        const size_t unit = ((size_t)slot * 4 + g) * geo.nbI + blk;
         if (live && blk < geo.nbI) {
-          const float* hp = ws.h + ((size_t)slot * 4 + g) * I + blk * 32 + tq * 8;
-          const float4 v0 = __ldcg(reinterpret_cast<const float4*>(hp));
-          const float4 v1 = __ldcg(reinterpret_cast<const float4*>(hp + 4));
-          v[bi][0] = v0.x; v[bi][1] = v0.y; v[bi][2] = v0.z; v[bi][3] = v0.w;
-          v[bi][4] = v1.x; v[bi][5] = v1.y; v[bi][6] = v1.z; v[bi][7] = v1.w;
+#pragma unroll
+          for (int part = 0; part < kHParts; ++part)
+            hf.q[bi][part] = __ldcg(reinterpret_cast<const uint2*>(ws.hq + (unit * kHParts + part) * 32 + tq * 8));
+          hf.f[bi] = __ldcg(ws.hf + unit);
         } else {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) v[bi][q] = 0.f;
+          for (int part = 0; part < kHParts; ++part) hf.q[bi][part] = make_uint2(0u, 0u);
+          hf.f[bi] = 0.f;
         }
       }
     };
-    auto down_item = [&](const float (&v)[kDnB][8]) {
-      // B fragments: h of token g, per 32-element block scaled by a power of
-      // two that puts the block's largest magnitude in [2^7, 2^8), then split
-      // into three E4M3 parts (12 significant bits), even/odd permuted as for
-      // x.  f0 / f1 undo the scales of tokens 2tq and 2tq+1 (and the E4M3
-      // weights' 2^-6) on the MMA results.
-      uint32_t bh[kDnB][kHParts][2];
+    auto down_item = [&](const HFrag& hf) {
+      // f0 / f1 undo the block scales of tokens 2tq and 2tq+1 (and the E4M3
+      // weights' 2^-6) on the MMA results
       float f0[kDnB], f1[kDnB];
 #pragma unroll
       for (int bi = 0; bi < kDnB; ++bi) {
-        float mx = 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mx = fmaxf(mx, fabsf(v[bi][q]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));  // the block of token g spans lanes 4g..4g+3
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const int sig = pow2_sigma(mx);
-        const float scl = exp2i(sig);
-        const float f = exp2i(6 - sig);
-        f0[bi] = __shfl_sync(0xffffffffu, f, 8 * tq);      // token 2tq lives in lanes 8tq..8tq+3
-        f1[bi] = __shfl_sync(0xffffffffu, f, 8 * tq + 4);  // token 2tq+1
-        uint32_t pe[kHParts], po[kHParts];
-        split3_e4m3x4(v[bi][0] * scl, v[bi][2] * scl, v[bi][4] * scl, v[bi][6] * scl, pe);
-        split3_e4m3x4(v[bi][1] * scl, v[bi][3] * scl, v[bi][5] * scl, v[bi][7] * scl, po);
-#pragma unroll
-        for (int part = 0; part < kHParts; ++part) {
-          bh[bi][part][0] = pe[part];
-          bh[bi][part][1] = po[part];
-        }
+        f0[bi] = __shfl_sync(0xffffffffu, hf.f[bi], 8 * tq);      // token 2tq lives in lanes 8tq..8tq+3
+        f1[bi] = __shfl_sync(0xffffffffu, hf.f[bi], 8 * tq + 4);  // token 2tq+1
       }
       const int st = it % kStages;
       const bool ok = bounded_wait(&C.full[st], (uint32_t)((it / kStages) & 1));
@@ -700,7 +688,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
               const uint32_t be = e2m1x8_even_to_e4m3x4(wb), bo = e2m1x8_odd_to_e4m3x4(wb);
               float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int part = 0; part < kHParts; ++part) mma_e4m3(d, ae, be, ao, bo, bh[bi][part][0], bh[bi][part][1]);
+              for (int part = 0; part < kHParts; ++part) mma_e4m3(d, ae, be, ao, bo, hf.q[bi][part].x, hf.q[bi][part].y);
               acc[4 * tt + 0] = fmaf(d[0], sa * f0[bi], acc[4 * tt + 0]);
               acc[4 * tt + 1] = fmaf(d[1], sa * f1[bi], acc[4 * tt + 1]);
               acc[4 * tt + 2] = fmaf(d[2], sb * f0[bi], acc[4 * tt + 2]);
@@ -793,15 +781,46 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     // phase 2 reads every CTA's h: wait until the epilogue warps have seen the
     // grid barrier that follows phase 1
     bounded_wait(&C.h_ready, 0);
-    float hv[kDnB][8];
-    if (n2 > 0) load_h(c / geo.n_tiles, hv);
+    // ---- split pass: h -> per-block scale and three E4M3 parts, once per
+    //      (slot, token, 32-element block) across the grid (one warp per
+    //      block: lane l holds element l), instead of once per down item ----
+    {
+      const int S = C.nslots;
+      const int units = S * M * geo.nbI;
+      for (int u = c * kCons + cw; u < units; u += G * kCons) {
+        const int blk = u % geo.nbI, sm = u / geo.nbI, m = sm % M, slot = sm / M;
+        const uint32_t mask = slot == 0 ? 0xfu : C.slot_mask[slot];
+        const size_t unit = ((size_t)slot * 4 + m) * geo.nbI + blk;
+        if (!(mask >> m & 1u)) continue;  // this token does not use the slot: its h is never read
+        const float v = __ldcg(ws.h + ((size_t)slot * 4 + m) * I + blk * 32 + lane);
+        const int sig = pow2_sigma(warp_max(fabsf(v)));
+        float r = v * exp2i(sig);
+        // element l goes to the lane tq = l / 8 of the B fragment: even ones
+        // to its first 4-byte group (b0), odd ones to its second (b1)
+        const int j = lane & 7;
+        uint8_t* dst = ws.hq + unit * kHParts * 32 + (lane >> 3) * 8 + (j & 1) * 4 + (j >> 1);
+#pragma unroll
+        for (int part = 0; part < kHParts; ++part) {
+          const float q = round_sig4(r);
+          dst[part * 32] = (uint8_t)f32x2_to_e4m3x2(q, 0.f);
+          r -= q;
+        }
+        if (lane == 0) ws.hf[unit] = exp2i(6 - sig);
+      }
+      // every CTA's parts are written before any down item reads them
+      consumer_bar_sync();
+      if (threadIdx.x == 0) {
+        const uint32_t old = grid_arrive(bar_word, c, G);
+        if (!poisoned() && !grid_wait(bar_word, old)) fail();
+        mbar_arrive(&C.parts_ready);  // the epilogue warps may arrive at the next barrier
+      }
+      consumer_bar_sync();
+    }
+    HFrag nxt;
+    if (n2 > 0) load_h(c / geo.n_tiles, nxt);
     for (int j = 0; j < n2; ++j) {
-      float cur[kDnB][8];
-#pragma unroll
-      for (int bi = 0; bi < kDnB; ++bi)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) cur[bi][q] = hv[bi][q];
-      if (j + 1 < n2) load_h((c + (j + 1) * G) / geo.n_tiles, hv);
+      const HFrag cur = nxt;
+      if (j + 1 < n2) load_h((c + (j + 1) * G) / geo.n_tiles, nxt);
       down_item(cur);
     }
   }
