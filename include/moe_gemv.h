@@ -232,6 +232,33 @@ MOE_API moe_status lmhead_decode_bf16(const uint16_t* hidden_bf16, const moe_bf1
                               int32_t M, int32_t top_k, int32_t* topk_ids, float* topk_vals,
                               float* logits, void* workspace, size_t workspace_bytes, void* stream);
 
+/* One draw per token from the head's top-k (ids and values as lmhead_decode
+ * returns them: values sorted descending), with temperature and top-p -- the
+ * sampled workload of the ncijnetwork.com summary ("What are the 3
+ * optimizations?": temperature 0.6, top-p 0.95, top-k 29).  In fp64, in this
+ * order, per token m with values v_0 >= v_1 >= ... and u = uniforms[m]:
+ *   p_i = exp((v_i - v_0) / temperature), total = p_0 + ... + p_{k-1};
+ *   n = the smallest prefix whose mass p_0 + ... + p_{n-1} reaches top_p * total;
+ *   i = the first index < n with p_0 + ... + p_i > u * (p_0 + ... + p_{n-1});
+ *   out_ids[m] = topk_ids[m][i].
+ *   topk_ids [M][top_k] int32, topk_vals [M][top_k] fp32, uniforms [M] fp32 in
+ *   [0, 1) (the caller's random numbers), out_ids [M] int32: device memory.
+ * 1 <= top_k <= 64, temperature > 0, 0 < top_p <= 1.  Enqueued on `stream`;
+ * argument errors are returned before anything is enqueued.                 */
+MOE_API moe_status lmhead_sample(const int32_t* topk_ids, const float* topk_vals, int32_t M, int32_t top_k,
+                                 float temperature, float top_p, const float* uniforms, int32_t* out_ids,
+                                 void* stream);
+
+/* Greedy acceptance of D draft tokens against the D + 1 argmaxes of the
+ * verify step (the saipien.org essay, "Draft three tokens, verify four":
+ * D = 3).  Draft i is accepted while it equals verify_ids[i] and every
+ * earlier draft was accepted; emitted_ids = the accepted drafts followed by
+ * verify_ids[accepted]; *n_emitted = accepted + 1 (1 .. D + 1).
+ *   draft_ids [D], verify_ids [D + 1], emitted_ids [D + 1], n_emitted [1]:
+ *   int32 device memory; 1 <= D <= 64.                                        */
+MOE_API moe_status moe_mtp_accept(const int32_t* draft_ids, const int32_t* verify_ids, int32_t D,
+                                  int32_t* emitted_ids, int32_t* n_emitted, void* stream);
+
 /* lmhead_decode for callers that cannot provide a workspace: hosts that own
  * every device allocation and give a plugin only its inputs and outputs, or
  * loops that must not call cudaMalloc (it can synchronise the device).  No

@@ -94,6 +94,8 @@ def _load() -> ctypes.CDLL:
         "moe_query_path": ([ctypes.c_char_p, SZ], I32),
         "moe_status_string": ([I32], ctypes.c_char_p),
         "moe_selftest_wait_timeout": ([P, SZ, ctypes.c_uint32, P], I32),
+        "lmhead_sample": ([P, P, I32, I32, ctypes.c_float, ctypes.c_float, P, P, P], I32),
+        "moe_mtp_accept": ([P, P, I32, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -308,6 +310,29 @@ def lmhead_decode_noalloc(hidden: torch.Tensor, head: FP8Head, top_k: int, topk_
                                        _ptr(topk_vals), _ptr(logits), _stream(stream))
     _check(st, "lmhead_decode_noalloc")
     return topk_ids, topk_vals
+
+
+def lmhead_sample(topk_ids: torch.Tensor, topk_vals: torch.Tensor, temperature: float, top_p: float,
+                  uniforms: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One draw per token from the head's sorted top-k (temperature, top-p);
+    uniforms [M] fp32 in [0, 1) are the caller's random numbers."""
+    M, k = topk_ids.shape
+    if out is None:
+        out = torch.empty((M,), dtype=torch.int32, device=topk_ids.device)
+    _check(library.lmhead_sample(_ptr(topk_ids), _ptr(topk_vals), M, k, float(temperature), float(top_p),
+                                 _ptr(uniforms), _ptr(out), _stream(stream)), "lmhead_sample")
+    return out
+
+
+def moe_mtp_accept(draft_ids: torch.Tensor, verify_ids: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Greedy acceptance of D drafts against D + 1 verify argmaxes; returns
+    (emitted [D + 1] int32, n_emitted [1] int32), device tensors."""
+    D = draft_ids.numel()
+    emitted = torch.empty((D + 1,), dtype=torch.int32, device=draft_ids.device)
+    n = torch.empty((1,), dtype=torch.int32, device=draft_ids.device)
+    _check(library.moe_mtp_accept(_ptr(draft_ids), _ptr(verify_ids), D, _ptr(emitted), _ptr(n), _stream(stream)),
+           "moe_mtp_accept")
+    return emitted, n
 
 
 def moe_rmsnorm_bf16(y: torch.Tensor, out: torch.Tensor, eps: float = 1e-6, stream=None) -> torch.Tensor:

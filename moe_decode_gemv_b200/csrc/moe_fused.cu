@@ -139,11 +139,12 @@ __device__ __forceinline__ void merge8(VI (&R)[8], const VI (&S)[8]) {
   cas(R[0], R[1]); cas(R[2], R[3]); cas(R[4], R[5]); cas(R[6], R[7]);
 }
 
-// The best 8 of logits[0..E) (E <= 1024), sorted, in every lane of the warp.
+// The best 8 of logits[0..E) (E <= 1024, in shared memory), sorted, in every
+// lane of the warp.
 // Logits that are NaN or -inf count as -FLT_MAX, so that every real expert
 // ranks above the padding entries (-FLT_MAX, INT32_MAX): with E >= 8 the
 // result holds only experts in [0, E).  Each lane sorts its logits 8 at a time
-// (loaded chunk by chunk, to keep few registers live) into its running best 8;
+// (read chunk by chunk, to keep few registers live) into its running best 8;
 // a butterfly of merges then gives every lane the warp's best 8.
 __device__ __forceinline__ void warp_top8(const float* logits, int E, int lane, VI (&R)[8]) {
 #pragma unroll
@@ -154,7 +155,7 @@ __device__ __forceinline__ void warp_top8(const float* logits, int E, int lane, 
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = lane + 32 * (8 * ch + j);
-      const float v = e < E ? __ldcg(logits + e) : -FLT_MAX;
+      const float v = e < E ? logits[e] : -FLT_MAX;
       S[j] = e < E ? VI{v > -FLT_MAX ? v : -FLT_MAX, e} : VI{-FLT_MAX, INT32_MAX};
     }
     sort8(S);
@@ -225,6 +226,7 @@ struct SmemCtl {
   uint64_t routed;                         // slot table ready (producer and epilogue warps wait on it)
   uint64_t h_ready;                        // every CTA's h written (consumers wait on it)
   uint64_t parts_ready;                    // this CTA passed the split-pass barrier (epilogue waits on it)
+  uint64_t partials_ready;                 // every CTA's partial outputs written (consumers wait on it)
   alignas(16) float red[kRed][kCons][32][8];  // per-item partials (float4 access)
   float logit_part[kCons][4];              // router: quarter-row partial sums
   int32_t ids[4][8];
@@ -237,6 +239,8 @@ struct SmemCtl {
   int nslots;
   int poison;
 };
+
+static_assert(sizeof(SmemCtl::red) >= 4 * 1024 * sizeof(float), "routing stages M x E <= 4 x 1024 logits in red");
 
 __device__ __forceinline__ void consumer_bar_sync() {
   asm volatile("bar.sync 1, %0;" ::"r"(kCons * 32) : "memory");
@@ -299,6 +303,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     mbar_init(&C.routed, 1);
     mbar_init(&C.h_ready, 1);
     mbar_init(&C.parts_ready, 1);
+    mbar_init(&C.partials_ready, 1);
     fence_mbar_init();
     C.poison = 0;
   }
@@ -472,23 +477,9 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       const int q = c + j * G;
       down_out(q / geo.n_tiles, (q % geo.n_tiles) * kDnRows);
     }
-    // every slot's partial outputs are written: combine the 32-row tiles this
-    // CTA owns (tile t belongs to CTA t mod G), slots in order -- no float
-    // atomics, the same result on every run
+    // every slot's partial outputs are written: the consumers combine them
     epilogue_grid_barrier();
-    if (!poisoned()) {
-      for (int t = c + ew * G; t < geo.n_tiles; t += kNumEpi * G) {
-        const int row = t * kDnRows + lane;
-        for (int m = 0; m < M; ++m) {
-          float y = 0.f;
-          for (int s2 = 0; s2 < S; ++s2) {
-            const uint32_t mk = s2 == 0 ? 0xfu : C.slot_mask[s2];
-            if (mk >> m & 1u) y = fmaf(C.slot_w[s2][m], __ldcg(&ws.ypart[((size_t)s2 * 4 + m) * H + row]), y);
-          }
-          a.out[(size_t)m * H + row] = y;
-        }
-      }
-    }
+    if (ew == 0 && lane == 0) mbar_arrive(&C.partials_ready);
   } else {
     // ============================== consumers =============================
     const int g = lane >> 2, tq = lane & 3;
@@ -703,19 +694,25 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       hand_off(acc);
     };
 
-    // ---- phase 1: the shared expert's items (no routing needed), then,
-    //      once every CTA's logits are in, routing and the routed items ----
-    const int ns = items.n_shared();
-    int n1 = ns, n2 = 0;
+    // ---- phase 1: once every CTA's logits are in, routing; then the shared
+    //      expert's items (prefetched by the producer while the barrier
+    //      completed) and the routed items.  Routing comes first so that the
+    //      routed items' copies start as early as possible. ----
+    int n1 = 1, n2 = 0;
     for (int j = 0;; ++j) {
-      if (j == ns) {
+      if (j == 0) {
         // ---- wait for every CTA's logits (bounded), then route ----
         if (threadIdx.x == 0 && !poisoned() && !grid_wait(bar_word, bar_old)) fail();
+        consumer_bar_sync();
+        // all M x E logits into shared memory with one round of loads (the
+        // reduce buffers are idle until the first item is handed off)
+        float* lg = &C.red[0][0][0][0];
+        for (int i = threadIdx.x; i < M * E; i += kCons * 32) lg[i] = __ldcg(ws.logits + i);
         consumer_bar_sync();
         if (cw < M) {  // warp m routes token m
           const int m = cw;
           VI R[8];
-          warp_top8(ws.logits + (size_t)m * E, E, lane, R);
+          warp_top8(lg + (size_t)m * E, E, lane, R);
           if (lane == 0) {
 #pragma unroll
             for (int r = 0; r < 8; ++r)
@@ -822,6 +819,28 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       const HFrag cur = nxt;
       if (j + 1 < n2) load_h((c + (j + 1) * G) / geo.n_tiles, nxt);
       down_item(cur);
+    }
+    // ---- combine: out = sum over slots, in slot order, of w * partial.  One
+    //      warp per (32-row tile, token) across the grid, lane = row, every
+    //      slot's load in flight at once: no float atomics, the same result
+    //      on every run ----
+    if (bounded_wait(&C.partials_ready, 0)) {
+      const int S = C.nslots;
+      for (int u = c + G * cw; u < geo.n_tiles * M; u += G * kCons) {
+        const int tile = u % geo.n_tiles, m = u / geo.n_tiles;
+        const int row = tile * kDnRows + lane;
+        float p[MoeWs::kMaxSlots];
+#pragma unroll
+        for (int s2 = 0; s2 < MoeWs::kMaxSlots; ++s2) {
+          const uint32_t mk = s2 == 0 ? 0xfu : C.slot_mask[s2 < S ? s2 : 0];
+          p[s2] = (s2 < S && (mk >> m & 1u)) ? __ldcg(&ws.ypart[((size_t)s2 * 4 + m) * H + row]) : 0.f;
+        }
+        float y = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < MoeWs::kMaxSlots; ++s2)
+          if (s2 < S) y = fmaf(C.slot_w[s2][m], p[s2], y);
+        a.out[(size_t)m * H + row] = y;
+      }
     }
   }
 }

@@ -87,6 +87,10 @@ class Oracle:
         L.orc_lmhead_fp8.argtypes = [_I64, _I64, _INT, _P, _P, _P, _P, _P]
         L.orc_lmhead_bf16.argtypes = [_I64, _I64, _INT, _P, _P, _P]
         L.orc_topk.argtypes = [_I64, _P, _INT, _P, _P]
+        L.orc_sample_topk.restype = _INT
+        L.orc_sample_topk.argtypes = [_INT, _P, _DBL, _DBL, _DBL]
+        L.orc_mtp_accept.restype = _INT
+        L.orc_mtp_accept.argtypes = [_INT, _P, _P, _P]
         L.orc_rmsnorm_bf16.argtypes = [_INT, _P, _DBL, _P]
 
     # ---- scalar formats -------------------------------------------------
@@ -218,6 +222,18 @@ class Oracle:
         vals = np.empty((k,), np.float64)
         self._L.orc_topk(v.shape[0], _ptr(v), k, _ptr(ids), _ptr(vals))
         return ids, vals
+
+    def sample_topk(self, vals, temperature: float, top_p: float, u: float) -> int:
+        v = np.ascontiguousarray(np.asarray(vals, dtype=np.float64))
+        return int(self._L.orc_sample_topk(len(v), _ptr(v), float(temperature), float(top_p), float(u)))
+
+    def mtp_accept(self, draft, verify) -> np.ndarray:
+        d = np.ascontiguousarray(np.asarray(draft, dtype=np.int32))
+        v = np.ascontiguousarray(np.asarray(verify, dtype=np.int32))
+        assert len(v) == len(d) + 1
+        out = np.zeros(len(v), np.int32)
+        n = self._L.orc_mtp_accept(len(d), _ptr(d), _ptr(v), _ptr(out))
+        return out[:n]
 
     def rmsnorm_bf16(self, y: np.ndarray, eps: float = 1e-6) -> np.ndarray:
         y = np.ascontiguousarray(y, np.float64)

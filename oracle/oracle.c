@@ -370,3 +370,48 @@ void orc_rmsnorm_bf16(int H, const double* y, double eps, uint16_t* out)
     for (int j = 0; j < H; ++j)
         out[j] = orc_double_to_bf16(y[j] / rms);
 }
+
+/* ---- sampled decode and speculative verify ---- */
+
+int orc_sample_topk(int k, const double* vals, double temperature, double top_p, double u)
+{
+    double* p = (double*)malloc(sizeof(double) * (size_t)k);
+    double total = 0.0;
+    for (int i = 0; i < k; ++i) {
+        p[i] = exp((vals[i] - vals[0]) / temperature);
+        total += p[i];
+    }
+    /* nucleus: the smallest prefix whose mass reaches top_p of the total */
+    int n = 0;
+    double before = 0.0;
+    while (n < k && before < top_p * total) {
+        before += p[n];
+        ++n;
+    }
+    double kept = 0.0;
+    for (int i = 0; i < n; ++i)
+        kept += p[i];
+    const double r = u * kept;
+    int pick = n - 1;
+    double cum = 0.0;
+    for (int i = 0; i < n; ++i) {
+        cum += p[i];
+        if (cum > r) {
+            pick = i;
+            break;
+        }
+    }
+    free(p);
+    return pick;
+}
+
+int orc_mtp_accept(int D, const int32_t* draft, const int32_t* verify, int32_t* emitted)
+{
+    int a = 0;
+    while (a < D && draft[a] == verify[a]) {
+        emitted[a] = draft[a];
+        ++a;
+    }
+    emitted[a] = verify[a];
+    return a + 1;
+}

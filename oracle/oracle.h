@@ -122,6 +122,22 @@ void orc_lmhead_bf16(int64_t V, int64_t H, int M, const uint16_t* x_bf16,
 /* The k largest of v[0..n), sorted descending, ties -> lower index.            */
 void orc_topk(int64_t n, const double* v, int k, int32_t* ids, double* vals);
 
+/* ---- sampled decode and speculative verify ---- */
+/* One draw from a sorted top-k list (the sampled workload of the ncijnetwork
+ * summary, "What are the 3 optimizations?": temperature 0.6, top-p 0.95,
+ * top-k 29).  With vals[0] >= vals[1] >= ...:
+ *   p_i = exp((vals[i] - vals[0]) / temperature), i < k        (softmax up to a factor)
+ *   keep the smallest prefix n whose mass reaches top_p:
+ *        i is kept while (p_0 + ... + p_{i-1}) < top_p * (p_0 + ... + p_{k-1})
+ *   return the first i < n with p_0 + ... + p_i > u * (p_0 + ... + p_{n-1}), u in [0, 1).    */
+int orc_sample_topk(int k, const double* vals, double temperature, double top_p, double u);
+/* Greedy acceptance of D draft tokens against the D+1 argmaxes of the verify
+ * step (the saipien.org essay, "Draft three tokens, verify four"): draft i is
+ * accepted while it equals verify i and every earlier draft was accepted.
+ * emitted = the accepted drafts, then verify[accepted] (the verify step's own
+ * next token); returns accepted + 1 (1 .. D+1).                                */
+int orc_mtp_accept(int D, const int32_t* draft, const int32_t* verify, int32_t* emitted);
+
 /* ---- between-layer op of the layer stack ---- */
 /* out[j] = bf16_RNE( y[j] / sqrt(mean(y^2) + eps) )  (gain 1).                 */
 void orc_rmsnorm_bf16(int H, const double* y, double eps, uint16_t* out);

@@ -406,9 +406,54 @@ def pin_rmsnorm(O) -> None:
         assert a in (lo, hi) and abs(a - b) <= abs((hi if a == lo else lo) - b) + 1e-300, (a, b)
 
 
+def pin_sample_topk(O) -> None:
+    """Closed forms of top-k / top-p / temperature sampling."""
+    # equal logits, no nucleus cut: the draw is floor(u * k)
+    for k in (1, 4, 29):
+        for u in (0.0, 0.2, 0.26, 0.5, 0.74, 0.999):
+            assert O.sample_topk([1.5] * k, 0.6, 1.0, u) == min(int(u * k), k - 1), (k, u)
+    # equal logits and a nucleus: the kept prefix is the smallest whose mass reaches top_p
+    assert all(O.sample_topk([0.0] * 4, 1.0, 0.5, u) == int(u * 2) for u in (0.1, 0.49, 0.51, 0.99))
+    assert all(O.sample_topk([0.0] * 4, 1.0, 0.51, u) == int(u * 3) for u in (0.1, 0.34, 0.67, 0.99))
+    # two candidates, gap d at temperature T: P(first) = 1 / (1 + exp(-d / T))
+    for d, T in ((1.0, 0.6), (0.3, 1.0), (2.0, 2.5)):
+        p0 = 1.0 / (1.0 + math.exp(-d / T))
+        assert O.sample_topk([d, 0.0], T, 1.0, p0 - 1e-9) == 0
+        assert O.sample_topk([d, 0.0], T, 1.0, p0 + 1e-9) == 1
+        # a nucleus below the first probability keeps only the first
+        assert O.sample_topk([d, 0.0], T, p0 * 0.999, 0.999) == 0
+    # a near-zero temperature is greedy
+    assert all(O.sample_topk([3.0, 2.9, 1.0, -2.0], 1e-3, 0.95, u) == 0 for u in (0.0, 0.5, 0.9999))
+    # stratified draws reproduce the nucleus distribution of scipy's softmax
+    from scipy.special import softmax
+    rng = np.random.default_rng(5)
+    v = np.sort(rng.normal(0, 1.5, 29))[::-1].copy()
+    T, top_p, N = 0.6, 0.95, 20000
+    p = softmax(v / T)
+    n = int(np.searchsorted(np.cumsum(p), top_p) + 1)  # first prefix whose mass reaches top_p
+    q = p[:n] / p[:n].sum()
+    counts = np.bincount([O.sample_topk(v, T, top_p, (i + 0.5) / N) for i in range(N)], minlength=29)
+    assert counts[n:].sum() == 0
+    assert np.all(np.abs(counts[:n] - q * N) <= 1.0 + 1e-6), (counts[:n], q * N)
+
+
+def pin_mtp_accept(O) -> None:
+    """Greedy acceptance, enumerated from its definition."""
+    cases = [
+        ([5, 6, 7], [5, 6, 7, 8], [5, 6, 7, 8]),    # all drafts accepted, plus the verify step's next token
+        ([5, 6, 7], [4, 6, 7, 8], [4]),             # the first draft rejected: only the verify token
+        ([5, 6, 7], [5, 9, 7, 8], [5, 9]),          # a later match after a mismatch does not count
+        ([5, 6, 7], [5, 6, 1, 8], [5, 6, 1]),
+        ([3], [3, 2], [3, 2]),
+        ([3], [2, 3], [2]),
+    ]
+    for draft, verify, want in cases:
+        assert O.mtp_accept(draft, verify).tolist() == want, (draft, verify)
+
+
 ALL_PINS = [
     pin_e2m1_table, pin_e8m0_table, pin_e4m3_table, pin_e2m1_encode, pin_e4m3_encode,
     pin_bf16_round, pin_mxfp4_quantize, pin_mxfp4_roundtrip, pin_fp8_rowquant, pin_router,
     pin_expert_special_case, pin_expert_vs_torch, pin_moe_layer, pin_lmhead, pin_topk,
-    pin_rmsnorm,
+    pin_rmsnorm, pin_sample_topk, pin_mtp_accept,
 ]

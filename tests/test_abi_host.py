@@ -156,3 +156,18 @@ def test_quantizers_reject_bad_arguments(lib):
     assert L.lmhead_quantize_fp8(A, ctypes.byref(h), None) == S.UNSUPPORTED_SHAPE
     h = lib._Fp8Head(0, 16, 256, U, A)
     assert L.lmhead_quantize_fp8(A, ctypes.byref(h), None) == S.MISALIGNED
+
+
+def test_sampling_and_accept_reject_bad_arguments(lib):
+    S, L = lib.Status, lib.library
+    f = ctypes.c_float
+    assert L.lmhead_sample(A, A, 1, 29, f(0.0), f(0.95), A, A, None) == S.INVALID_ARG   # temperature 0
+    assert L.lmhead_sample(A, A, 1, 29, f(0.6), f(1.5), A, A, None) == S.INVALID_ARG    # top_p > 1
+    assert L.lmhead_sample(A, A, 1, 65, f(0.6), f(0.95), A, A, None) == S.INVALID_ARG   # top_k > 64
+    assert L.lmhead_sample(A, A, 0, 29, f(0.6), f(0.95), A, A, None) == S.INVALID_ARG   # M = 0
+    assert L.lmhead_sample(None, A, 1, 29, f(0.6), f(0.95), A, A, None) == S.INVALID_ARG
+    assert L.lmhead_sample(A + 2, A, 1, 29, f(0.6), f(0.95), A, A, None) == S.MISALIGNED
+    assert L.moe_mtp_accept(A, A, 0, A, A, None) == S.INVALID_ARG
+    assert L.moe_mtp_accept(A, A, 65, A, A, None) == S.INVALID_ARG
+    assert L.moe_mtp_accept(A, None, 3, A, A, None) == S.INVALID_ARG
+    assert L.moe_mtp_accept(A, A + 1, 3, A, A, None) == S.MISALIGNED

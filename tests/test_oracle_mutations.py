@@ -44,6 +44,11 @@ MUTATIONS = {
     "lmhead_scale_dropped": ("logits[(int64_t)m * V + v] = (double)s[v] * acc;", "logits[(int64_t)m * V + v] = acc;"),
     "bf16_truncate": ("double t = nearbyint(ldexp(f, 8));", "double t = floor(ldexp(f, 8));"),
     "rmsnorm_mean": ("sqrt(ss / (double)H + eps)", "sqrt(ss / (double)(H - 1) + eps)"),
+    "sample_temperature_multiplies": ("p[i] = exp((vals[i] - vals[0]) / temperature);",
+                                      "p[i] = exp((vals[i] - vals[0]) * temperature);"),
+    "sample_nucleus_inclusive": ("while (n < k && before < top_p * total) {", "while (n < k && before <= top_p * total) {"),
+    "sample_draw_unnormalised": ("const double r = u * kept;", "const double r = u * total;"),
+    "mtp_accept_skips_mismatch": ("while (a < D && draft[a] == verify[a]) {", "while (a < D && draft[a] != verify[a] + 1) {"),
 }
 
 
