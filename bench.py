@@ -238,10 +238,45 @@ def time_steps(wl, M, steps, warmup, dist, device):
     moe = [e[0].elapsed_time(e[1]) * 1e3 for e in evs]
     head = [e[1].elapsed_time(e[2]) * 1e3 for e in evs]
     total_ms = max_over_ranks(total_ms, dist, device)
+    q = lambda v, f: sorted(v)[min(len(v) - 1, int(f * len(v)))]
     return {"total_us": total_ms * 1e3, "per_step_us": total_ms * 1e3 / steps,
             "moe_us_mean": statistics.fmean(moe), "moe_us_median": statistics.median(moe),
+            "moe_us_p10": q(moe, 0.1), "moe_us_p90": q(moe, 0.9),
             "head_us_mean": statistics.fmean(head), "head_us_median": statistics.median(head),
+            "head_us_p10": q(head, 0.1), "head_us_p90": q(head, 0.9),
             "wall": (t0, t1)}
+
+
+def distinct_experts(wl, M, n):
+    """|U|, the distinct routed experts one M-token step streams, over n steps."""
+    torch = wl.torch
+    us = []
+    for i in range(n):
+        wl.step(i, M)
+        torch.cuda.synchronize()
+        us.append(len(set(wl.ids[M].cpu().numpy().reshape(-1).tolist())))
+    return {"mean": statistics.fmean(us), "min": min(us), "max": max(us), "steps": n}
+
+
+def read_ceiling(B, buf, reps=20):
+    """This GPU's practical HBM read rate: moe_stream_read over a buffer larger
+    than L2, CUDA events, best and median of `reps` runs."""
+    import torch
+    sink = torch.zeros((1,), dtype=torch.int32, device=buf.device)
+    nbytes = buf.numel() * buf.element_size() // 16 * 16
+    for _ in range(3):
+        B.moe_stream_read(buf, sink)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        B.moe_stream_read(buf, sink)
+        e1.record()
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    us = [a.elapsed_time(b) * 1e3 for a, b in ts]
+    return {"kernel": "moe_stream_read", "bytes": nbytes, "gbs_best": nbytes / (min(us) * 1e-6) / 1e9,
+            "gbs_median": nbytes / (statistics.median(us) * 1e-6) / 1e9}
 
 
 def time_e2e(wl, M, steps, warmup, dist, device):
@@ -608,7 +643,9 @@ def main():
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": profiled_traffic(), "algorithmic_bytes_per_launch": head_bytes},
         "breakdown_m1": {"moe_us_mean": m1["moe_us_mean"], "moe_us_median": m1["moe_us_median"],
+                         "moe_us_p10": m1["moe_us_p10"], "moe_us_p90": m1["moe_us_p90"],
                          "head_us_mean": m1["head_us_mean"], "head_us_median": m1["head_us_median"],
+                         "head_us_p10": m1["head_us_p10"], "head_us_p90": m1["head_us_p90"],
                          "moe_bytes": moe_bytes_m1,
                          "moe_gbs": moe_bytes_m1 / (m1["moe_us_mean"] * 1e-6) / 1e9,
                          "head_gbs": achieved},
@@ -616,12 +653,14 @@ def main():
         "bf16_head_gbs": A.lmhead_bf16_bytes(I.LING_HEAD) / (bf16_head_us * 1e-6) / 1e9,
         "clocks": clocks,
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": 2 * args.steps,  # one MoE and one LM-head kernel per timed step
         "path": B.moe_query_path(),
     }
     if m4 is not None:
         line["m4"] = {"us_per_step": m4["per_step_us"], "moe_us_mean": m4["moe_us_mean"],
-                      "head_us_mean": m4["head_us_mean"], "steps": max(args.steps // 2, 1)}
+                      "head_us_mean": m4["head_us_mean"], "steps": max(args.steps // 2, 1),
+                      "distinct_experts": distinct_experts(wl, 4, 16)}
+    line["read_ceiling"] = read_ceiling(B, wl.head.q)
     if not args.no_stream:
         try:
             line["stream_16_layers"] = stream_leg(wl, B, I, A, args.seed + rank, device, args.stream_steps)

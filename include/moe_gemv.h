@@ -123,9 +123,11 @@ typedef struct {
  * Within a data row, the 16-byte unit c (one 32-element block) of row r is
  * stored at position c ^ (r & mask), mask = min(8, largest power of two
  * dividing the units per row) - 1, so that eight consecutive rows read
- * together hit distinct shared-memory banks.  fmt must be
- * MOE_FMT_MXFP4_MOE_PACKED.  The pages have no counterpart for this layout;
- * it changes where bytes sit, never their values.                             */
+ * together hit distinct shared-memory banks.  Within every data byte the
+ * bits of its two E2M1 codes are re-placed: element 2j's sign, e1, e0, m go
+ * to bits 7, 3, 2, 1 and element 2j+1's to bits 0, 6, 5, 4 (scale bytes are
+ * unchanged).  fmt must be MOE_FMT_MXFP4_MOE_PACKED.  The pages have no
+ * counterpart for this layout; it moves bits, never changes a value.          */
 typedef struct {
     int32_t fmt;
     int32_t count;
@@ -292,6 +294,13 @@ MOE_API moe_status moe_rmsnorm_bf16(const float* y, int32_t M, int32_t H, float 
  * H a multiple of 8.                                                         */
 MOE_API moe_status moe_embed_gather(const uint16_t* table, int64_t V, int64_t H, const int32_t* ids,
                                     int32_t ids_stride, int32_t M, uint16_t* out, void* stream);
+
+/* Measurement aid, not a step of the path: read `bytes` (a multiple of 16)
+ * from device memory `src` (16-byte aligned) with 128-bit non-allocating loads
+ * from every SM, folding the words into the device word *sink by XOR, so that
+ * a caller timing it sees this GPU's practical HBM read ceiling -- the
+ * yardstick for the weight streams above.  Enqueued on `stream`.            */
+MOE_API moe_status moe_stream_read(const void* src, size_t bytes, uint32_t* sink, void* stream);
 
 /* ---- housekeeping --------------------------------------------------------- */
 

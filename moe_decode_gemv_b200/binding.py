@@ -95,6 +95,7 @@ def _load() -> ctypes.CDLL:
         "moe_status_string": ([I32], ctypes.c_char_p),
         "moe_selftest_wait_timeout": ([P, SZ, ctypes.c_uint32, P], I32),
         "lmhead_sample": ([P, P, I32, I32, ctypes.c_float, ctypes.c_float, P, P, P], I32),
+        "moe_stream_read": ([P, SZ, P, P], I32),
         "moe_mtp_accept": ([P, P, I32, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
@@ -333,6 +334,12 @@ def moe_mtp_accept(draft_ids: torch.Tensor, verify_ids: torch.Tensor, stream=Non
     _check(library.moe_mtp_accept(_ptr(draft_ids), _ptr(verify_ids), D, _ptr(emitted), _ptr(n), _stream(stream)),
            "moe_mtp_accept")
     return emitted, n
+
+
+def moe_stream_read(src: torch.Tensor, sink: torch.Tensor, stream=None) -> None:
+    """Read all of `src` (measurement aid for the HBM read ceiling)."""
+    nbytes = src.numel() * src.element_size() // 16 * 16
+    _check(library.moe_stream_read(_ptr(src), nbytes, _ptr(sink), _stream(stream)), "moe_stream_read")
 
 
 def moe_rmsnorm_bf16(y: torch.Tensor, out: torch.Tensor, eps: float = 1e-6, stream=None) -> torch.Tensor:

@@ -226,6 +226,14 @@ moe_status moe_embed_gather(const uint16_t* table, int64_t V, int64_t H, const i
                                               static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_stream_read(const void* src, size_t bytes, uint32_t* sink, void* stream) {
+  if (!src || !sink || bytes < 16 || bytes % 16 != 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(src) || (reinterpret_cast<uintptr_t>(sink) & 3u)) return MOE_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  if (moe::current_device_sms(&dev, &sms) != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(moe::launch_stream_read(src, bytes, sink, sms, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_workspace_reset(void* workspace, size_t workspace_bytes, void* stream) {
   if (!workspace || workspace_bytes < sizeof(moe::WsHeader)) return MOE_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)));
@@ -247,9 +255,11 @@ moe_status moe_workspace_status(void* workspace, void* stream) {
 moe_status moe_query_path(char* buf, size_t n) {
   if (!buf || n == 0) return MOE_ERR_INVALID_ARG;
   const char* desc =
-      "sm_100a; moe: one persistent kernel (router fp32 GEMV + top-k, MXFP4 E2M1/E8M0-32 gate/up + SiLU, "
-      "down, ordered combine; bulk-copy ring, mma.sync f16); lm-head: FP8 E4M3 per-row-scale GEMV "
-      "(bulk-copy ring, mma.sync f16) fused top-k; comparator: BF16 head GEMV";
+      "sm_100a; moe: one cooperative persistent kernel (router fp32 GEMV, top-k softmax routing, "
+      "MXFP4 E2M1/E8M0-32 gate/up + SiLU and down over packed banks, one bulk copy per work item, "
+      "E2M1->E5M2 by bit moves into mma.sync m16n8k32 e5m2 x e4m3, output rows summed over slots in order); "
+      "lm-head: online-FP8 E4M3 per-row-scale GEMV (bulk-copy ring, mma.sync m16n8k32 e4m3) fused top-k "
+      "with temperature/top-p sampling; comparator: BF16 head GEMV";
   std::snprintf(buf, n, "%s", desc);
   return std::strlen(desc) < n ? MOE_OK : MOE_ERR_INVALID_ARG;
 }

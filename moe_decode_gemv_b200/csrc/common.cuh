@@ -119,6 +119,34 @@ __device__ __forceinline__ uint32_t e2m1x8_odd_to_e4m3x4(uint32_t w) {
   return ((w >> 2) & 0x1c1c1c1cu) | (w & 0x80808080u);
 }
 
+// The packed expert banks (pack_kernels.cu) place the two E2M1 codes of a
+// byte as element 2j: sign|e1 e0 m at bits 7|3 2 1 and element 2j+1 at bits
+// 0|6 5 4.  E5M2 s|0 0 0 e1 e0|m 0 carries the E2M1 value times 2^-14 for
+// every code (the E2M1 subnormal 0.5 becomes the E5M2 subnormal 2^-15), so
+// the even elements of a packed word are E5M2 codes after one mask, and the
+// odd ones after two shifts.  Bytes 0..3 of the result hold elements 0, 2,
+// 4, 6 (even) or 1, 3, 5, 7 (odd) of the word.
+__device__ __forceinline__ uint32_t packed_even_to_e5m2x4(uint32_t w) { return w & 0x8e8e8e8eu; }
+__device__ __forceinline__ uint32_t packed_odd_to_e5m2x4(uint32_t w) {
+  return ((w >> 3) & 0x0e0e0e0eu) | ((w << 7) & 0x80808080u);
+}
+
+// E8M0 code -> fp32 2^(code - 127) by one integer multiply (the FMA pipe, not
+// the logic pipe): exact for codes 1..254.  Code 0 gives 0 instead of 2^-127
+// (a block at that scale adds less than 2^-116 of its largest product to any
+// sum) and code 255 gives +inf instead of NaN, so a block that carries it
+// still turns its dot products into NaN when its elements are zero -- as the
+// quantiser writes them -- and into +-inf otherwise.
+__device__ __forceinline__ float e8m0_to_f32_fast(uint32_t code) { return __uint_as_float(code * 0x800000u); }
+
+// E5M2 (A) x E4M3 (B) -> fp32 tensor-core MMA, m16n8k32.
+__device__ __forceinline__ void mma_e5m2_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.f32.e5m2.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // E4M3 x E4M3 -> fp32 tensor-core MMA, m16n8k32 (A row-major 16x32, B 32x8).
 // Not volatile: it has no effect beyond its outputs, so the compiler may
 // interleave independent MMAs instead of issuing them in source order.

@@ -36,15 +36,17 @@
 //    CTA sums, for the 32-row tiles it owns, the slot partials in slot order:
 //    no float atomics, the result is reproducible run to run.
 //
-// Arithmetic: mma.sync m16n8k32 E4M3 x E4M3 -> fp32, one MMA per 32-element
-// MX block, so that its fp32 result is scaled by that block's E8M0 scale
-// before it joins the running fp32 sum.  The weights need no conversion
-// instruction: an E2M1 code becomes the E4M3 code of its value times 2^-6 by
-// moving bits (e2m1x8_*_to_e4m3x4).  Activations are scaled by a per-token
-// power of two that puts their largest magnitude in [2^7, 2^8); bf16 x is
-// then carried exactly by two E4M3 parts (two MMAs per block).  h is scaled
-// per 32-element block and token (largest magnitude into [2^7, 2^8)) and
-// carried by three E4M3 parts (12 significant bits, three MMAs per block).
+// Arithmetic: mma.sync m16n8k32 E5M2 (weights) x E4M3 (activations) -> fp32,
+// one MMA per 32-element MX block and 16 weight rows, so that its fp32
+// result is scaled by that block's E8M0 scale before it joins the running
+// fp32 sum.  The weights need no conversion instruction: the packed bank
+// places each E2M1 code's bits so that a mask (even elements) or two shifts
+// (odd ones) give the E5M2 code of its value times 2^-14.  Activations are
+// scaled by a per-token power of two that puts their largest magnitude in
+// [2^7, 2^8); bf16 x is then carried exactly by two E4M3 parts, which ride in
+// two columns of the same MMA.  h is scaled per 32-element block and token
+// (largest magnitude into [2^7, 2^8)) and carried by three E4M3 parts (12
+// significant bits) in three columns; one MMA covers two tokens.
 #include <cuda_runtime.h>
 
 #include <cfloat>
@@ -268,13 +270,17 @@ __device__ __forceinline__ bool grid_wait(uint32_t* word, uint32_t old) {
 
 // The work of one CTA, enumerated identically by the producer, the consumers
 // and the epilogue warps: phase-1 items are global items c, c+G, ... of
-// S * n_chunks (the first n_chunks belong to the shared expert, slot 0), then
-// phase-2 items c, c+G, ... of S * n_tiles.
+// S * n_chunks (the first n_chunks belong to the shared expert, slot 0, so
+// that most CTAs have one to load before routing), then phase-2 items are
+// the contiguous range [S n_tiles c / G, S n_tiles (c + 1) / G) of
+// S * n_tiles: consecutive down tiles of the same slot, which share their
+// B fragments (h of that slot).
 struct ItemIter {
   int c, G, n_chunks, n_tiles;
   __device__ int n_shared() const { return c < n_chunks ? (n_chunks - c + G - 1) / G : 0; }
   __device__ int n_phase1(int S) const { return c < S * n_chunks ? (S * n_chunks - c + G - 1) / G : 0; }
-  __device__ int n_phase2(int S) const { return c < S * n_tiles ? (S * n_tiles - c + G - 1) / G : 0; }
+  __device__ int p2_begin(int S) const { return (int)((int64_t)S * n_tiles * c / G); }
+  __device__ int n_phase2(int S) const { return (int)((int64_t)S * n_tiles * (c + 1) / G) - p2_begin(S); }
 };
 
 template <int kGuB>
@@ -373,8 +379,9 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       const int q = c + j * G;
       issue(q / geo.n_chunks, true, (q % geo.n_chunks) * kGuRows);
     }
+    const int q2 = n2 > 0 ? items.p2_begin(*(volatile int*)&C.nslots) : 0;
     for (int j = 0; j < n2; ++j) {
-      const int q = c + j * G;
+      const int q = q2 + j;
       issue(q / geo.n_tiles, false, (q % geo.n_tiles) * kDnRows);
     }
     // every issued copy must land before this CTA may exit
@@ -399,22 +406,20 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     auto gateup_out = [&](int slot, int row0) {
       const bool ok = take();
       const float* rb = &C.red[idx % kRed][0][0][0];
-      float gs[2] = {0.f, 0.f}, us[2] = {0.f, 0.f};
+      float gs = 0.f, us = 0.f;  // gate row g and up row g of token tq: the two parts summed
 #pragma unroll
       for (int w2 = 0; w2 < kCons; ++w2) {
         const float4 p = *reinterpret_cast<const float4*>(rb + (w2 * 32 + lane) * 8);
-        gs[0] += p.x; gs[1] += p.y; us[0] += p.z; us[1] += p.w;
+        gs += p.x + p.y;
+        us += p.z + p.w;
       }
       give();
       const uint32_t mask = slot == 0 ? 0xfu : C.slot_mask[slot];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int m = 2 * tq + q;
-        if (ok && tq < 2 && m < M && (mask >> m & 1u)) {
-          const float inv = exp2i(6 - C.sigma_x[m]);  // undo 2^sigma and the E4M3 weights' 2^-6
-          const float gg = gs[q] * inv, uu = us[q] * inv;
-          ws.h[((size_t)slot * 4 + m) * I + row0 + g] = gg / (1.0f + expf(-gg)) * uu;
-        }
+      const int m = tq;
+      if (ok && m < M && (mask >> m & 1u)) {
+        const float inv = exp2i(6 - C.sigma_x[m]) * 256.0f;  // undo 2^sigma and the E5M2 weights' 2^-14
+        const float gg = gs * inv, uu = us * inv;
+        ws.h[((size_t)slot * 4 + m) * I + row0 + g] = gg / (1.0f + expf(-gg)) * uu;
       }
     };
     auto down_out = [&](int slot, int row0) {
@@ -429,16 +434,23 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
         s8[4] += p1.x; s8[5] += p1.y; s8[6] += p1.z; s8[7] += p1.w;
       }
       give();
-      const uint32_t mask = slot == 0 ? 0xfu : C.slot_mask[slot];
+      // lanes tq and tq ^ 1 hold the parts of the same token: after the sum,
+      // the even lanes hold s8[4 tt + 2 half + r] = row 16tt + 8half + g of
+      // token 2r + (tq >> 1)
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int m = 2 * tq + q;
-        if (ok && tq < 2 && m < M && (mask >> m & 1u)) {
-          float* yp = ws.ypart + ((size_t)slot * 4 + m) * H + row0;
-          yp[g] = s8[q];            // row g of the first 16
-          yp[g + 8] = s8[2 + q];    // row g + 8
-          yp[16 + g] = s8[4 + q];   // second 16 rows
-          yp[24 + g] = s8[6 + q];
+      for (int q = 0; q < 8; ++q) s8[q] += __shfl_xor_sync(0xffffffffu, s8[q], 1);
+      const uint32_t mask = slot == 0 ? 0xfu : C.slot_mask[slot];
+      if (ok && (tq & 1) == 0) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int m = 2 * r + (tq >> 1);
+          if (m < M && (mask >> m & 1u)) {
+            float* yp = ws.ypart + ((size_t)slot * 4 + m) * H + row0;
+            yp[g] = s8[r];
+            yp[8 + g] = s8[2 + r];
+            yp[16 + g] = s8[4 + r];
+            yp[24 + g] = s8[6 + r];
+          }
         }
       }
     };
@@ -472,9 +484,10 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     // consumers' arrival at the split-pass barrier, even when it has no
     // phase-2 items: arrivals on the word stay in barrier order.
     bounded_wait(&C.parts_ready, 0);
+    const int q2 = items.p2_begin(S);
     for (int j = 0; j < n2; ++j, ++idx) {
       if (idx % kNumEpi != ew) continue;
-      const int q = c + j * G;
+      const int q = q2 + j;
       down_out(q / geo.n_tiles, (q % geo.n_tiles) * kDnRows);
     }
     // every slot's partial outputs are written: the consumers combine them
@@ -538,20 +551,23 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     if (threadIdx.x == 0) bar_old = grid_arrive(bar_word, c, G);
 
     // x as E4M3 B fragments for this warp's K blocks of the gate/up GEMV.
+    // Column n of B is part n & 1 of token n >> 1: each token, scaled by
+    // 2^sigma, is carried exactly by two E4M3 parts (hi, lo), and the two
+    // parts ride in two columns of ONE MMA (their sum is taken after it).
     // Within a 32-element block, lane (g, tq) covers elements 8tq..8tq+7 of
-    // token g: the even ones fill k-slots 4tq..4tq+3 (b0), the odd ones
-    // 16+4tq.. (b1), matching the even/odd split of the weight nibbles.  The
-    // token, scaled by 2^sigma, is carried exactly by two E4M3 parts (hi, lo).
-    uint32_t bx[kGuB][2][2];  // [block][part][b0, b1]; this warp's blocks are cw, cw + kCons, ...
+    // column g: the even ones fill k-slots 4tq..4tq+3 (b0), the odd ones
+    // 16+4tq.. (b1), matching the even/odd split of the weight nibbles.
+    uint32_t bx[kGuB][2];  // [block][b0, b1]; this warp's blocks are cw, cw + kCons, ...
     {
-      const bool live = g < M;
-      const float scl = live ? exp2i(C.sigma_x[g]) : 0.f;
+      const int m = g >> 1, part = g & 1;
+      const bool live = m < M;
+      const float scl = live ? exp2i(C.sigma_x[m]) : 0.f;
 #pragma unroll
       for (int bi = 0; bi < kGuB; ++bi) {
         const int blk = cw + kCons * bi;
         uint32_t pe[2] = {0u, 0u}, po[2] = {0u, 0u};
         if (live && blk < geo.nbH) {
-          const uint4 q = *reinterpret_cast<const uint4*>(a.x + (size_t)g * H + blk * 32 + tq * 8);
+          const uint4 q = *reinterpret_cast<const uint4*>(a.x + (size_t)m * H + blk * 32 + tq * 8);
           const float v0 = bf16_bits_to_f32(q.x & 0xffffu) * scl, v1 = bf16_bits_to_f32(q.x >> 16) * scl;
           const float v2 = bf16_bits_to_f32(q.y & 0xffffu) * scl, v3 = bf16_bits_to_f32(q.y >> 16) * scl;
           const float v4 = bf16_bits_to_f32(q.z & 0xffffu) * scl, v5 = bf16_bits_to_f32(q.z >> 16) * scl;
@@ -559,11 +575,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
           split_e4m3x4<2>(v0, v2, v4, v6, pe);
           split_e4m3x4<2>(v1, v3, v5, v7, po);
         }
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          bx[bi][part][0] = pe[part];
-          bx[bi][part][1] = po[part];
-        }
+        bx[bi][0] = part ? pe[1] : pe[0];
+        bx[bi][1] = part ? po[1] : po[0];
       }
     }
     // Shared-memory offsets of this lane's words.  Block blk = cw + kCons*bi of
@@ -575,115 +588,138 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
     const int gu_scl = 16 * gu_rowb + g * geo.nbH + cw;                    // gate scale; up scale adds 8 rows
     int it = 0;     // ring position
     int nitem = 0;  // items handed to the epilogue warps
-    auto hand_off = [&](const float (&v)[8]) {
+    auto hand_off = [&](const float (&v)[8], bool two) {
       const int r = nitem % kRed;
       if (nitem >= kRed) bounded_wait(&C.red_empty[r], (uint32_t)(((nitem / kRed) & 1) ^ 1));
       float* rb = &C.red[r][0][0][0];
       *reinterpret_cast<float4*>(rb + (cw * 32 + lane) * 8) = make_float4(v[0], v[1], v[2], v[3]);
-      *reinterpret_cast<float4*>(rb + (cw * 32 + lane) * 8 + 4) = make_float4(v[4], v[5], v[6], v[7]);
+      if (two) *reinterpret_cast<float4*>(rb + (cw * 32 + lane) * 8 + 4) = make_float4(v[4], v[5], v[6], v[7]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&C.red_full[r]);
       ++nitem;
     };
 
     // ---- phase-1 item: partial gate/up sums for 8 rows of one slot ----
+    // All shared loads first, then one MMA per block (E5M2 weights from the
+    // packed nibbles, x's two parts in two columns), then the block scales.
     auto gateup_item = [&]() {
       const int st = it % kStages;
       const bool ok = bounded_wait(&C.full[st], (uint32_t)((it / kStages) & 1));
       const uint8_t* base = ring + (size_t)st * geo.stage_bytes;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (ok) {
+        uint32_t gw[kGuB], uw[kGuB];
+#pragma unroll
+        for (int bi = 0; bi < kGuB; ++bi) {
+          const bool in = cw + kCons * bi < geo.nbH;
+          gw[bi] = in ? lds32(base + gu_lane + 256 * bi) : 0u;
+          uw[bi] = in ? lds32(base + gu_lane + 8 * gu_rowb + 256 * bi) : 0u;
+        }
+        float d[kGuB][4];
+#pragma unroll
+        for (int bi = 0; bi < kGuB; ++bi) {
+          // A: gate row g (a0, a2) and up row g (a1, a3), 32 elements = one MX block
+          d[bi][0] = d[bi][1] = d[bi][2] = d[bi][3] = 0.f;
+          if (cw + kCons * bi < geo.nbH)
+            mma_e5m2_e4m3(d[bi], packed_even_to_e5m2x4(gw[bi]), packed_even_to_e5m2x4(uw[bi]),
+                          packed_odd_to_e5m2x4(gw[bi]), packed_odd_to_e5m2x4(uw[bi]), bx[bi][0], bx[bi][1]);
+        }
 #pragma unroll
         for (int bi = 0; bi < kGuB; ++bi) {
           if (cw + kCons * bi < geo.nbH) {
-            const uint32_t gw = lds32(base + gu_lane + 256 * bi);
-            const uint32_t uw = lds32(base + gu_lane + 8 * gu_rowb + 256 * bi);
-            const float sg = e8m0_to_f32(base[gu_scl + kCons * bi]);
-            const float su = e8m0_to_f32(base[gu_scl + 8 * geo.nbH + kCons * bi]);
-            // A: gate row g (a0, a2) and up row g (a1, a3), 32 elements = one MX block
-            const uint32_t ge = e2m1x8_even_to_e4m3x4(gw), go = e2m1x8_odd_to_e4m3x4(gw);
-            const uint32_t ue = e2m1x8_even_to_e4m3x4(uw), uo = e2m1x8_odd_to_e4m3x4(uw);
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_e4m3(d, ge, ue, go, uo, bx[bi][0][0], bx[bi][0][1]);
-            mma_e4m3(d, ge, ue, go, uo, bx[bi][1][0], bx[bi][1][1]);
-            acc[0] = fmaf(d[0], sg, acc[0]);
-            acc[1] = fmaf(d[1], sg, acc[1]);
-            acc[2] = fmaf(d[2], su, acc[2]);
-            acc[3] = fmaf(d[3], su, acc[3]);
+            const float sg = e8m0_to_f32_fast(base[gu_scl + kCons * bi]);
+            const float su = e8m0_to_f32_fast(base[gu_scl + 8 * geo.nbH + kCons * bi]);
+            acc[0] = fmaf(d[bi][0], sg, acc[0]);  // gate row g, token tq: hi part
+            acc[1] = fmaf(d[bi][1], sg, acc[1]);  //                       lo part
+            acc[2] = fmaf(d[bi][2], su, acc[2]);  // up row g, token tq
+            acc[3] = fmaf(d[bi][3], su, acc[3]);
           }
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&C.empty[st]);
       ++it;
-      hand_off(acc);
+      hand_off(acc, false);
     };
 
     // ---- phase-2 item: partial sums of 32 output rows of one slot's down matrix ----
     const int dn_rowb = I / 2;
     const int dn_lane = g * dn_rowb + ((cw ^ (g & geo.mI)) * 16) + tq * 4;  // rows 16tt + g (+ 8) share it
     const int dn_scl = kDnRows * dn_rowb + g * geo.nbI + cw;
-    // The B fragments of a down item: h of token g for this warp's blocks of
-    // one slot, already split into three E4M3 parts by the split pass
-    // (uint2 = the lane's even and odd 4-byte groups of one part) and the
-    // factor that undoes the block's scale.  Issued one item ahead, so the L2
-    // round trip overlaps the previous item.
+    // The B fragments of a down item: h of one slot for this warp's blocks,
+    // already split into three E4M3 parts by the split pass.  MMA group r
+    // covers tokens 2r and 2r+1: column n holds part n & 3 of token
+    // 2r + (n >> 2) (part 3 is zero), so lane (g, tq) loads one part of one
+    // token (uint2 = its even and odd 4-byte groups) and its results are the
+    // parts of token 2r + (tq >> 1), whose block factor (undoing the block's
+    // scale and the E5M2 weights' 2^-14) it holds in f.  Issued one item
+    // ahead, so the L2 round trip overlaps the previous item.
     struct HFrag {
-      uint2 q[kDnB][kHParts];
-      float f[kDnB];
+      uint2 q[kDnB][2];
+      float f[kDnB][2];
     };
     auto load_h = [&](int slot, HFrag& hf) {
       const uint32_t mask = slot == 0 ? 0xfu : C.slot_mask[slot];
-      const bool live = !poisoned() && g < M && (mask >> g & 1u);
+      const bool ok = !poisoned();
 #pragma unroll
       for (int bi = 0; bi < kDnB; ++bi) {
         const int blk = cw + kCons * bi;
-        const size_t unit = ((size_t)slot * 4 + g) * geo.nbI + blk;
-        if (live && blk < geo.nbI) {
 #pragma unroll
-          for (int part = 0; part < kHParts; ++part)
-            hf.q[bi][part] = __ldcg(reinterpret_cast<const uint2*>(ws.hq + (unit * kHParts + part) * 32 + tq * 8));
-          hf.f[bi] = __ldcg(ws.hf + unit);
-        } else {
-#pragma unroll
-          for (int part = 0; part < kHParts; ++part) hf.q[bi][part] = make_uint2(0u, 0u);
-          hf.f[bi] = 0.f;
+        for (int r = 0; r < 2; ++r) {
+          const int mb = 2 * r + (g >> 2), p = g & 3, mo = 2 * r + (tq >> 1);
+          const bool lb = ok && blk < geo.nbI && p < kHParts && mb < M && (mask >> mb & 1u);
+          const bool lf = ok && blk < geo.nbI && mo < M && (mask >> mo & 1u);
+          const size_t ub = ((size_t)slot * 4 + mb) * geo.nbI + blk, uo = ((size_t)slot * 4 + mo) * geo.nbI + blk;
+          hf.q[bi][r] = lb ? __ldcg(reinterpret_cast<const uint2*>(ws.hq + (ub * kHParts + p) * 32 + tq * 8))
+                           : make_uint2(0u, 0u);
+          hf.f[bi][r] = lf ? __ldcg(ws.hf + uo) : 0.f;
         }
       }
     };
     auto down_item = [&](const HFrag& hf) {
-      // f0 / f1 undo the block scales of tokens 2tq and 2tq+1 (and the E4M3
-      // weights' 2^-6) on the MMA results
-      float f0[kDnB], f1[kDnB];
-#pragma unroll
-      for (int bi = 0; bi < kDnB; ++bi) {
-        f0[bi] = __shfl_sync(0xffffffffu, hf.f[bi], 8 * tq);      // token 2tq lives in lanes 8tq..8tq+3
-        f1[bi] = __shfl_sync(0xffffffffu, hf.f[bi], 8 * tq + 4);  // token 2tq+1
-      }
       const int st = it % kStages;
       const bool ok = bounded_wait(&C.full[st], (uint32_t)((it / kStages) & 1));
       const uint8_t* base = ring + (size_t)st * geo.stage_bytes;
+      // acc[4 tt + 2 half + r]: rows 16tt + 8half + g, token group r, the
+      // lane's columns summed (parts of token 2r + (tq >> 1))
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (ok) {
+        uint32_t wa[2][kDnB], wb[2][kDnB];  // rows 16tt + g and 16tt + 8 + g
 #pragma unroll
         for (int tt = 0; tt < 2; ++tt) {
 #pragma unroll
           for (int bi = 0; bi < kDnB; ++bi) {
-            if (cw + kCons * bi < geo.nbI) {
-              const int off = dn_lane + 16 * tt * dn_rowb + 256 * bi;
-              const uint32_t wa = lds32(base + off);
-              const uint32_t wb = lds32(base + off + 8 * dn_rowb);
-              const float sa = e8m0_to_f32(base[dn_scl + 16 * tt * geo.nbI + kCons * bi]);
-              const float sb = e8m0_to_f32(base[dn_scl + (16 * tt + 8) * geo.nbI + kCons * bi]);
-              const uint32_t ae = e2m1x8_even_to_e4m3x4(wa), ao = e2m1x8_odd_to_e4m3x4(wa);
-              const uint32_t be = e2m1x8_even_to_e4m3x4(wb), bo = e2m1x8_odd_to_e4m3x4(wb);
-              float d[4] = {0.f, 0.f, 0.f, 0.f};
+            const bool in = cw + kCons * bi < geo.nbI;
+            const int off = dn_lane + 16 * tt * dn_rowb + 256 * bi;
+            wa[tt][bi] = in ? lds32(base + off) : 0u;
+            wb[tt][bi] = in ? lds32(base + off + 8 * dn_rowb) : 0u;
+          }
+        }
 #pragma unroll
-              for (int part = 0; part < kHParts; ++part) mma_e4m3(d, ae, be, ao, bo, hf.q[bi][part].x, hf.q[bi][part].y);
-              acc[4 * tt + 0] = fmaf(d[0], sa * f0[bi], acc[4 * tt + 0]);
-              acc[4 * tt + 1] = fmaf(d[1], sa * f1[bi], acc[4 * tt + 1]);
-              acc[4 * tt + 2] = fmaf(d[2], sb * f0[bi], acc[4 * tt + 2]);
-              acc[4 * tt + 3] = fmaf(d[3], sb * f1[bi], acc[4 * tt + 3]);
+        for (int r = 0; r < 2; ++r) {
+          if (r == 1 && M <= 2) break;
+          float d[2][kDnB][4];
+#pragma unroll
+          for (int tt = 0; tt < 2; ++tt) {
+#pragma unroll
+            for (int bi = 0; bi < kDnB; ++bi) {
+              d[tt][bi][0] = d[tt][bi][1] = d[tt][bi][2] = d[tt][bi][3] = 0.f;
+              if (cw + kCons * bi < geo.nbI)
+                mma_e5m2_e4m3(d[tt][bi], packed_even_to_e5m2x4(wa[tt][bi]), packed_even_to_e5m2x4(wb[tt][bi]),
+                              packed_odd_to_e5m2x4(wa[tt][bi]), packed_odd_to_e5m2x4(wb[tt][bi]), hf.q[bi][r].x,
+                              hf.q[bi][r].y);
+            }
+          }
+#pragma unroll
+          for (int tt = 0; tt < 2; ++tt) {
+#pragma unroll
+            for (int bi = 0; bi < kDnB; ++bi) {
+              if (cw + kCons * bi < geo.nbI) {
+                const float ta = e8m0_to_f32_fast(base[dn_scl + 16 * tt * geo.nbI + kCons * bi]) * hf.f[bi][r];
+                const float tb = e8m0_to_f32_fast(base[dn_scl + (16 * tt + 8) * geo.nbI + kCons * bi]) * hf.f[bi][r];
+                acc[4 * tt + r] = fmaf(d[tt][bi][1], ta, fmaf(d[tt][bi][0], ta, acc[4 * tt + r]));
+                acc[4 * tt + 2 + r] = fmaf(d[tt][bi][3], tb, fmaf(d[tt][bi][2], tb, acc[4 * tt + 2 + r]));
+              }
             }
           }
         }
@@ -691,7 +727,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       __syncwarp();
       if (lane == 0) mbar_arrive(&C.empty[st]);
       ++it;
-      hand_off(acc);
+      hand_off(acc, true);
     };
 
     // ---- phase 1: once every CTA's logits are in, routing; then the shared
@@ -802,7 +838,7 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
           dst[part * 32] = (uint8_t)f32x2_to_e4m3x2(q, 0.f);
           r -= q;
         }
-        if (lane == 0) ws.hf[unit] = exp2i(6 - sig);
+        if (lane == 0) ws.hf[unit] = exp2i(6 - sig) * 256.0f;  // 2^-sig and the E5M2 weights' 2^-14
       }
       // every CTA's parts are written before any down item reads them
       consumer_bar_sync();
@@ -813,11 +849,19 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
       }
       consumer_bar_sync();
     }
+    // B fragments are loaded once per slot (the CTA's items are consecutive
+    // tiles), one item ahead of the first item that needs them
+    const int q2 = items.p2_begin(C.nslots);
     HFrag nxt;
-    if (n2 > 0) load_h(c / geo.n_tiles, nxt);
+    int nslot = n2 > 0 ? q2 / geo.n_tiles : -1;
+    if (n2 > 0) load_h(nslot, nxt);
     for (int j = 0; j < n2; ++j) {
       const HFrag cur = nxt;
-      if (j + 1 < n2) load_h((c + (j + 1) * G) / geo.n_tiles, nxt);
+      if (j + 1 < n2) {
+        const int s1 = (q2 + j + 1) / geo.n_tiles;
+        if (s1 != nslot) load_h(s1, nxt);
+        nslot = s1;
+      }
       down_item(cur);
     }
     // ---- combine: out = sum over slots, in slot order, of w * partial.  One

@@ -16,7 +16,11 @@
 // permuted: unit c of row r is stored at position c ^ (r & mask), mask =
 // min(8, largest power of two dividing the units per row) - 1.  The kernel's
 // eight rows g = 0..7 that one instruction reads then fall on distinct
-// shared-memory banks.  Packing moves bytes only; no value changes.
+// shared-memory banks.  Within each data byte the two E2M1 codes are
+// re-placed bit by bit (nibble_relayout): element 2j's sign|e1 e0 m go to
+// bits 7|3 2 1 and element 2j+1's to bits 0|6 5 4.  Then a mask alone turns
+// the four even elements of a word into E5M2 codes, and a shift pair the odd
+// ones (see moe_fused.cu).  Packing moves bits only; no value changes.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -24,6 +28,15 @@
 
 namespace moe {
 namespace {
+
+// Four data bytes: E2M1 pair (low nibble = element 2j, high = 2j+1) -> the
+// packed bit placement described above.
+__device__ __forceinline__ uint32_t nibble_relayout(uint32_t w) {
+  return ((w & 0x08080808u) << 4) | ((w & 0x07070707u) << 1) | ((w & 0x80808080u) >> 7) | (w & 0x70707070u);
+}
+__device__ __forceinline__ uint4 nibble_relayout(uint4 v) {
+  return make_uint4(nibble_relayout(v.x), nibble_relayout(v.y), nibble_relayout(v.z), nibble_relayout(v.w));
+}
 
 // One thread per 16-byte unit of the output.
 __global__ void pack_gateup_kernel(const uint8_t* __restrict__ gate_d, const uint8_t* __restrict__ gate_s,
@@ -44,7 +57,7 @@ __global__ void pack_gateup_kernel(const uint8_t* __restrict__ gate_d, const uin
       const int r = j / nb, p = j - r * nb;
       const int c = p ^ (r & mask);           // stored at p, read from unit c of the source row
       const uint8_t* src = (r < 8 ? gate_d : up_d) + ((e * I + q * 8 + (r & 7)) * (int64_t)(H / 2)) + c * 16;
-      v = *reinterpret_cast<const uint4*>(src);
+      v = nibble_relayout(*reinterpret_cast<const uint4*>(src));
     } else {
       const int b = (j - 16 * nb) * 16;       // byte offset in the 16 scale rows (8 gate, then 8 up)
       const uint8_t* src = (b < 8 * nb ? gate_s + b : up_s + (b - 8 * nb)) + (e * I + q * 8) * (int64_t)nb;
@@ -70,7 +83,7 @@ __global__ void pack_down_kernel(const uint8_t* __restrict__ down_d, const uint8
     if (j < 32 * nb) {
       const int r = j / nb, p = j - r * nb;
       const int c = p ^ (r & mask);
-      v = *reinterpret_cast<const uint4*>(down_d + ((e * H + t * 32 + r) * (int64_t)(I / 2)) + c * 16);
+      v = nibble_relayout(*reinterpret_cast<const uint4*>(down_d + ((e * H + t * 32 + r) * (int64_t)(I / 2)) + c * 16));
     } else {
       const int b = (j - 32 * nb) * 16;
       v = *reinterpret_cast<const uint4*>(down_s + (e * H + t * 32) * (int64_t)nb + b);

@@ -47,7 +47,32 @@ __global__ void embed_gather_kernel(const uint16_t* __restrict__ table, int64_t 
   for (int j = threadIdx.x; j < H / 8; j += blockDim.x) dst[j] = ok ? src[j] : make_uint4(0, 0, 0, 0);
 }
 
+// Measurement aid: every thread streams 16-byte words with non-allocating
+// loads (grid-stride) and folds them into one XOR, one atomic per warp.
+__global__ void stream_read_kernel(const uint4* __restrict__ src, size_t n, uint32_t* __restrict__ sink) {
+  uint32_t acc = 0;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n; i += 4 * stride) {  // four independent loads in flight per thread
+    const uint4 a = ld_stream_u4(src + i), b = ld_stream_u4(src + i + stride);
+    const uint4 c = ld_stream_u4(src + i + 2 * stride), d = ld_stream_u4(src + i + 3 * stride);
+    acc ^= a.x ^ a.y ^ a.z ^ a.w ^ b.x ^ b.y ^ b.z ^ b.w ^ c.x ^ c.y ^ c.z ^ c.w ^ d.x ^ d.y ^ d.z ^ d.w;
+  }
+  for (; i < n; i += stride) {
+    const uint4 v = ld_stream_u4(src + i);
+    acc ^= v.x ^ v.y ^ v.z ^ v.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc ^= __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) atomicXor(sink, acc);
+}
+
 }  // namespace
+
+cudaError_t launch_stream_read(const void* src, size_t bytes, uint32_t* sink, int sms, cudaStream_t st) {
+  stream_read_kernel<<<4 * sms, 256, 0, st>>>(static_cast<const uint4*>(src), bytes / 16, sink);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_rmsnorm_bf16(const float* y, int M, int H, float eps, uint16_t* out, cudaStream_t st) {
   rmsnorm_bf16_kernel<<<M, 256, 0, st>>>(y, H, eps, out);

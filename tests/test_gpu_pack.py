@@ -1,6 +1,6 @@
 """The packed expert-bank layout, byte for byte, against a numpy statement of
 the layout that moe_gemv.h documents for moe_packed_bank (packing moves
-bytes only, so the comparison is exact)."""
+bytes and bits only, so the comparison is exact)."""
 import numpy as np
 import pytest
 import torch
@@ -23,6 +23,15 @@ def swizzle_mask(units):
     return min(8, low) - 1
 
 
+def relayout(b):
+    """The documented bit placement of one packed data byte: element 2j (low
+    nibble) sign|e1 e0 m -> bits 7|3 2 1, element 2j+1 (high nibble) -> 0|6 5 4."""
+    b = b.astype(np.uint8)
+    lo, hi = b & 0xF, b >> 4
+    out = ((lo >> 3) << 7) | ((lo & 7) << 1) | (hi >> 3) | ((hi & 7) << 4)
+    return out.astype(np.uint8)
+
+
 def expected_packed(gate, up, down):
     """numpy: (data, scales) pairs of the canonical banks -> (gateup, down) bytes."""
     (gd, gs), (ud, us), (dd, ds) = gate, up, down
@@ -37,7 +46,7 @@ def expected_packed(gate, up, down):
             units = rows.reshape(16, nbH, 16)
             # unit c of row r is stored at position c ^ (r & mask): position p holds unit p ^ (r & mask)
             perm = np.stack([units[r, np.arange(nbH) ^ (r & mH)] for r in range(16)])
-            gu.append(perm.reshape(-1))
+            gu.append(relayout(perm.reshape(-1)))
             gu.append(gs[e, 8 * q:8 * q + 8].reshape(-1))
             gu.append(us[e, 8 * q:8 * q + 8].reshape(-1))
     dn = []
@@ -45,7 +54,7 @@ def expected_packed(gate, up, down):
         for t in range(H // 32):
             units = dd[e, 32 * t:32 * t + 32].reshape(32, nbI, 16)
             perm = np.stack([units[r, np.arange(nbI) ^ (r & mI)] for r in range(32)])
-            dn.append(perm.reshape(-1))
+            dn.append(relayout(perm.reshape(-1)))
             dn.append(ds[e, 32 * t:32 * t + 32].reshape(-1))
     return np.concatenate(gu), np.concatenate(dn)
 
