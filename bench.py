@@ -639,7 +639,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": m1["per_step_us"] / 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic", "config": workload_config(),
-        "roofline": {"bound": "hbm", "kernel": "lmhead_topk_kernel (FP8 LM head, M=1)", "achieved": achieved,
+        "roofline": {"bound": "hbm", "kernel": "lmhead_fp8_tiled_kernel (FP8 LM head, M=1)", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": profiled_traffic(), "algorithmic_bytes_per_launch": head_bytes},
         "breakdown_m1": {"moe_us_mean": m1["moe_us_mean"], "moe_us_median": m1["moe_us_median"],

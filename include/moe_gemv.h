@@ -87,7 +87,8 @@ typedef enum {
     MOE_FMT_BF16 = 1,
     MOE_FMT_MXFP4_E2M1_E8M0_32 = 2,
     MOE_FMT_FP8_E4M3_ROWSCALE_F32 = 3,
-    MOE_FMT_MXFP4_MOE_PACKED = 4
+    MOE_FMT_MXFP4_MOE_PACKED = 4,
+    MOE_FMT_FP8_E4M3_TILED = 5
 } moe_format;
 
 /* A stack of `count` MXFP4 matrices, each [rows][K]:
@@ -137,8 +138,14 @@ typedef struct {
     uint8_t* down;
 } moe_packed_bank;
 
-/* The online-FP8 LM head: q [vocab][hidden] E4M3 and row_scale [vocab] fp32.
- * fmt must be MOE_FMT_FP8_E4M3_ROWSCALE_F32.                                   */
+/* The online-FP8 LM head: q E4M3 and row_scale [vocab] fp32.
+ *   fmt MOE_FMT_FP8_E4M3_ROWSCALE_F32 (lmhead_quantize_fp8): q [vocab][hidden].
+ *   fmt MOE_FMT_FP8_E4M3_TILED (lmhead_tile_fp8; what lmhead_decode reads):
+ *     the same bytes in whole 16-row tiles (zero rows past vocab), tile T of
+ *     16 * hidden bytes; for each 64-byte K slice s, 1,024 bytes ordered
+ *     [half h][lane l][16 bytes] = row 16T + (l >> 2) + 8h, K bytes
+ *     64s + 16(l & 3) .. +15.  One 512-byte run is then one warp's A
+ *     fragments of an mma.sync m16n8k32 pair.  Values are unchanged.       */
 typedef struct {
     int32_t fmt;
     int64_t vocab;
@@ -184,6 +191,16 @@ MOE_API moe_status moe_pack_experts(const moe_expert_bank* src, moe_packed_bank*
  * quantising only this layer to FP8 at load time.                           */
 MOE_API moe_status lmhead_quantize_fp8(const uint16_t* w_bf16, moe_fp8_head* out, void* stream);
 
+/* Bytes of the tiled FP8 head for these sizes (0 if unsupported).            */
+MOE_API size_t lmhead_tiled_bytes(int64_t vocab, int64_t hidden);
+
+/* Re-lay a quantised head (fmt MOE_FMT_FP8_E4M3_ROWSCALE_F32) into the tiled
+ * layout lmhead_decode streams.  The caller fills dst->vocab, hidden (equal
+ * to src's), q (lmhead_tiled_bytes bytes, 16-byte aligned) and row_scale
+ * (an array holding src's row scales -- src->row_scale itself serves; this
+ * call does not touch it).  Enqueued on `stream`; on success sets dst->fmt. */
+MOE_API moe_status lmhead_tile_fp8(const moe_fp8_head* src, moe_fp8_head* dst, void* stream);
+
 /* ---- decode --------------------------------------------------------------- */
 
 /* Bytes of workspace moe_decode needs for these sizes (0 if unsupported).    */
@@ -213,7 +230,7 @@ MOE_API moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w
 MOE_API size_t lmhead_workspace_bytes(int32_t M, int32_t top_k, int64_t vocab, int64_t hidden);
 
 /* FP8 LM head for M tokens (1 <= M <= 4), fused with top-k:
- *   hidden   [M][H] bf16;  head: the quantised head (tag checked)
+ *   hidden   [M][H] bf16;  head: the tiled head (fmt MOE_FMT_FP8_E4M3_TILED)
  *   topk_ids [M][top_k] int32, topk_vals [M][top_k] fp32: the top_k largest
  *            logits, descending, ties to the lower token id (top_k = 1 is the
  *            greedy argmax); 1 <= top_k <= 64

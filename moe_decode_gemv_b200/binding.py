@@ -37,6 +37,7 @@ class Format(enum.IntEnum):
     MXFP4_E2M1_E8M0_32 = 2
     FP8_E4M3_ROWSCALE_F32 = 3
     MXFP4_MOE_PACKED = 4
+    FP8_E4M3_TILED = 5
 
 
 class MoEError(RuntimeError):
@@ -78,6 +79,8 @@ def _load() -> ctypes.CDLL:
     sig = {
         "moe_quantize_mxfp4": ([P, ctypes.POINTER(_Mxfp4), P], I32),
         "lmhead_quantize_fp8": ([P, ctypes.POINTER(_Fp8Head), P], I32),
+        "lmhead_tiled_bytes": ([I64, I64], SZ),
+        "lmhead_tile_fp8": ([ctypes.POINTER(_Fp8Head), ctypes.POINTER(_Fp8Head), P], I32),
         "moe_workspace_bytes": ([I32, I32, I32, I32, I32], SZ),
         "moe_packed_gateup_bytes": ([I32, I32, I32], SZ),
         "moe_packed_down_bytes": ([I32, I32, I32], SZ),
@@ -181,13 +184,20 @@ class PackedBank:
 
 @dataclass
 class FP8Head:
-    """The online-FP8 LM head: q [V, H] uint8 (E4M3) and row_scale [V] fp32."""
+    """The online-FP8 LM head: q uint8 (E4M3) -- [V, H] as quantised, or the
+    flat tiled bytes lmhead_decode reads -- and row_scale [V] fp32."""
     q: torch.Tensor
     row_scale: torch.Tensor
     fmt: int = Format.NONE
+    vocab: int = 0
+    hidden: int = 0
+
+    def __post_init__(self):
+        if self.q.dim() == 2 and not self.vocab:
+            self.vocab, self.hidden = self.q.shape
 
     def _c(self) -> _Fp8Head:
-        return _Fp8Head(int(self.fmt), self.q.shape[0], self.q.shape[1], self.q.data_ptr(), self.row_scale.data_ptr())
+        return _Fp8Head(int(self.fmt), self.vocab, self.hidden, self.q.data_ptr(), self.row_scale.data_ptr())
 
 
 def alloc_fp8_head(vocab: int, hidden: int, device="cuda") -> FP8Head:
@@ -232,12 +242,29 @@ def moe_pack_experts(bank: tuple[MXFP4Bank, MXFP4Bank, MXFP4Bank], stream=None) 
     return out
 
 
-def lmhead_quantize_fp8(w_bf16: torch.Tensor, out: FP8Head | None = None, stream=None) -> FP8Head:
+def lmhead_quantize_fp8(w_bf16: torch.Tensor, out: FP8Head | None = None, stream=None,
+                        tiled: bool = True) -> FP8Head:
+    """bf16 [V, H] -> the FP8 head; tiled (the default) re-lays it for
+    lmhead_decode by lmhead_tile_fp8, else it stays [V, H]."""
     assert w_bf16.dtype == torch.bfloat16 and w_bf16.is_cuda and w_bf16.is_contiguous()
     if out is None:
         out = alloc_fp8_head(w_bf16.shape[0], w_bf16.shape[1], device=w_bf16.device)
     c = out._c()
     _check(library.lmhead_quantize_fp8(_ptr(w_bf16), ctypes.byref(c), _stream(stream)), "lmhead_quantize_fp8")
+    out.fmt = c.fmt
+    return lmhead_tile_fp8(out, stream=stream) if tiled else out
+
+
+def lmhead_tile_fp8(head: FP8Head, stream=None) -> FP8Head:
+    """A quantised [V, H] head -> the tiled head lmhead_decode reads (its row
+    scales are shared with `head`)."""
+    nbytes = int(library.lmhead_tiled_bytes(head.vocab, head.hidden))
+    if nbytes == 0:
+        raise MoEError(Status.UNSUPPORTED_SHAPE, "lmhead_tile_fp8")
+    out = FP8Head(torch.empty((nbytes,), dtype=torch.uint8, device=head.q.device), head.row_scale,
+                  vocab=head.vocab, hidden=head.hidden)
+    src, c = head._c(), out._c()
+    _check(library.lmhead_tile_fp8(ctypes.byref(src), ctypes.byref(c), _stream(stream)), "lmhead_tile_fp8")
     out.fmt = c.fmt
     return out
 
@@ -278,7 +305,7 @@ def lmhead_decode(hidden: torch.Tensor, head: FP8Head, top_k: int, topk_ids: tor
                   logits: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
     M = hidden.shape[0]
     if workspace is None:
-        workspace = new_workspace(lmhead_workspace_bytes(M, top_k, head.q.shape[0], head.q.shape[1]),
+        workspace = new_workspace(lmhead_workspace_bytes(M, top_k, head.vocab, head.hidden),
                                   hidden.device, stream)
     c = head._c()
     st = library.lmhead_decode(_ptr(hidden), ctypes.byref(c), M, top_k, _ptr(topk_ids), _ptr(topk_vals), _ptr(logits),

@@ -121,6 +121,23 @@ moe_status lmhead_quantize_fp8(const uint16_t* w_bf16, moe_fp8_head* out, void* 
   return MOE_OK;
 }
 
+size_t lmhead_tiled_bytes(int64_t vocab, int64_t hidden) {
+  return head_shape_ok(vocab, hidden, 1) ? moe::lmhead_tiled_bytes(vocab, (int)hidden) : 0;
+}
+
+moe_status lmhead_tile_fp8(const moe_fp8_head* src, moe_fp8_head* dst, void* stream) {
+  if (!src || !dst || !src->q || !dst->q || !dst->row_scale) return MOE_ERR_INVALID_ARG;
+  if (src->fmt != MOE_FMT_FP8_E4M3_ROWSCALE_F32) return MOE_ERR_FORMAT_MISMATCH;
+  if (dst->vocab != src->vocab || dst->hidden != src->hidden) return MOE_ERR_INVALID_ARG;
+  if (!head_shape_ok(src->vocab, src->hidden, 1)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(src->q) || !aligned16(dst->q) || !aligned16(dst->row_scale)) return MOE_ERR_MISALIGNED;
+  const cudaError_t e = moe::launch_tile_fp8_head(src->q, src->vocab, (int)src->hidden, dst->q,
+                                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  dst->fmt = MOE_FMT_FP8_E4M3_TILED;
+  return MOE_OK;
+}
+
 size_t moe_packed_gateup_bytes(int32_t count, int32_t hidden, int32_t inter) {
   return pack_shape_ok(count, hidden, inter) ? moe::packed_gateup_bytes(count, hidden, inter) : 0;
 }
@@ -196,7 +213,7 @@ moe_status lmhead_decode(const uint16_t* hidden_bf16, const moe_fp8_head* head, 
                          int32_t* topk_ids, float* topk_vals, float* logits, void* workspace, size_t workspace_bytes,
                          void* stream) {
   if (!head) return MOE_ERR_INVALID_ARG;
-  if (head->fmt != MOE_FMT_FP8_E4M3_ROWSCALE_F32) return MOE_ERR_FORMAT_MISMATCH;
+  if (head->fmt != MOE_FMT_FP8_E4M3_TILED) return MOE_ERR_FORMAT_MISMATCH;
   if (!head->q || !head->row_scale) return MOE_ERR_INVALID_ARG;
   return launch_head_common(hidden_bf16, head->q, head->row_scale, true, head->vocab, head->hidden, M, top_k,
                             topk_ids, topk_vals, logits, workspace, workspace_bytes, stream);
@@ -258,7 +275,7 @@ moe_status moe_query_path(char* buf, size_t n) {
       "sm_100a; moe: one cooperative persistent kernel (router fp32 GEMV, top-k softmax routing, "
       "MXFP4 E2M1/E8M0-32 gate/up + SiLU and down over packed banks, one bulk copy per work item, "
       "E2M1->E5M2 by bit moves into mma.sync m16n8k32 e5m2 x e4m3, output rows summed over slots in order); "
-      "lm-head: online-FP8 E4M3 per-row-scale GEMV (bulk-copy ring, mma.sync m16n8k32 e4m3) fused top-k "
+      "lm-head: online-FP8 E4M3 per-row-scale GEMV over the fragment-tiled head (coalesced 16-byte loads into registers, mma.sync m16n8k32 e4m3) fused top-k "
       "with temperature/top-p sampling; comparator: BF16 head GEMV";
   std::snprintf(buf, n, "%s", desc);
   return std::strlen(desc) < n ? MOE_OK : MOE_ERR_INVALID_ARG;

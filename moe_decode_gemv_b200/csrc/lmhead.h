@@ -10,12 +10,17 @@
 namespace moe {
 
 int lmhead_max_slices();
-// Ring depth and shared memory of one launch; false if the shape does not fit
-// in one CTA's shared memory (the CTA keeps its rows' logits there).
+// Ring depth (0 for the tiled FP8 kernel) and shared memory of one launch;
+// false if the shape does not fit in one CTA's shared memory (the CTA keeps
+// its rows' logits there).
 bool lmhead_plan(int H, int elem_bytes, int M, int top_k, int64_t V, int grid, int* stages, size_t* smem);
 size_t lmhead_cand_bytes(int grid, int M, int top_k);
+// Bytes of the fragment-tiled FP8 head (whole 16-row tiles, zero rows past V).
+size_t lmhead_tiled_bytes(int64_t V, int H);
+cudaError_t launch_tile_fp8_head(const uint8_t* q, int64_t V, int H, uint8_t* out, cudaStream_t st);
 
-cudaError_t launch_lmhead_fp8(const uint16_t* x, const uint8_t* q, const float* s, int64_t V, int H, int M,
+// FP8 head over the tiled layout (qt: lmhead_tiled_bytes bytes).
+cudaError_t launch_lmhead_fp8(const uint16_t* x, const uint8_t* qt, const float* s, int64_t V, int H, int M,
                               int top_k, float* logits, int32_t* ids, float* vals, WsHeader* hdr, void* cand,
                               int grid, cudaStream_t st);
 cudaError_t launch_lmhead_bf16(const uint16_t* x, const uint16_t* w, int64_t V, int H, int M, int top_k,

@@ -51,7 +51,7 @@ extern "C" moe_status lmhead_decode_noalloc(const uint16_t* hidden_bf16, const m
                                             void* stream) {
   // the same argument checks as lmhead_decode, before any CUDA call
   if (!head) return MOE_ERR_INVALID_ARG;
-  if (head->fmt != MOE_FMT_FP8_E4M3_ROWSCALE_F32) return MOE_ERR_FORMAT_MISMATCH;
+  if (head->fmt != MOE_FMT_FP8_E4M3_TILED) return MOE_ERR_FORMAT_MISMATCH;
   if (!head->q || !head->row_scale || !hidden_bf16 || !topk_ids || !topk_vals) return MOE_ERR_INVALID_ARG;
   const int64_t V = head->vocab, H = head->hidden;
   if (M < 1 || M > 4 || top_k < 1 || top_k > 64 || top_k > V) return MOE_ERR_INVALID_ARG;

@@ -184,7 +184,7 @@ def head_weights(seed: int, shape: I.HeadShape) -> torch.Tensor:
 
 def run_head_gpu(B, head, x_dev, k, with_logits=True, bf16_w=None):
     M = x_dev.shape[0]
-    V = bf16_w.shape[0] if bf16_w is not None else head.q.shape[0]
+    V = bf16_w.shape[0] if bf16_w is not None else head.vocab
     ids = torch.empty((M, k), dtype=torch.int32, device="cuda")
     vals = torch.empty((M, k), dtype=torch.float32, device="cuda")
     logits = torch.empty((M, V), dtype=torch.float32, device="cuda") if with_logits else None

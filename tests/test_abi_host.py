@@ -129,20 +129,38 @@ def test_lmhead_rejects_bad_arguments(lib):
     def call(head, M=1, k=1, ids=A, ws_bytes=1 << 22, fn=L.lmhead_decode):
         return fn(A, ctypes.byref(head), M, k, ids, A, None, A, ws_bytes, None)
 
-    fp8 = lib._Fp8Head(3, 4096, 256, A, A)
+    fp8 = lib._Fp8Head(5, 4096, 256, A, A)
     # an FP8 head handed to the BF16 path, and a BF16-tagged head handed to the
-    # FP8 path, are both refused instead of being read with the wrong format
+    # FP8 path, are both refused instead of being read with the wrong format;
+    # so is an FP8 head that was quantised but not tiled
     assert call(lib._Fp8Head(1, 4096, 256, A, A)) == S.FORMAT_MISMATCH
     assert call(lib._Bf16Head(3, 4096, 256, A), fn=L.lmhead_decode_bf16) == S.FORMAT_MISMATCH
     assert call(lib._Fp8Head(0, 4096, 256, A, A)) == S.FORMAT_MISMATCH
+    assert call(lib._Fp8Head(3, 4096, 256, A, A)) == S.FORMAT_MISMATCH
+    assert L.lmhead_decode_noalloc(A, ctypes.byref(lib._Fp8Head(3, 4096, 256, A, A)), 1, 1, A, A, None,
+                                   None) == S.FORMAT_MISMATCH
     assert call(fp8, M=0) == S.INVALID_ARG
     assert call(fp8, k=65) == S.INVALID_ARG
     assert call(fp8, ids=0) == S.INVALID_ARG
     assert call(fp8, ids=U) == S.MISALIGNED
     assert call(fp8, ws_bytes=10) == S.WORKSPACE
-    assert call(lib._Fp8Head(3, 4096, 100, A, A)) == S.UNSUPPORTED_SHAPE
-    assert call(lib._Fp8Head(3, 4096, 8192, A, A)) == S.UNSUPPORTED_SHAPE
-    assert call(lib._Fp8Head(3, 0, 256, A, A)) == S.UNSUPPORTED_SHAPE or call(lib._Fp8Head(3, 0, 256, A, A)) == S.INVALID_ARG
+    assert call(lib._Fp8Head(5, 4096, 100, A, A)) == S.UNSUPPORTED_SHAPE
+    assert call(lib._Fp8Head(5, 4096, 8192, A, A)) == S.UNSUPPORTED_SHAPE
+    assert call(lib._Fp8Head(5, 0, 256, A, A)) in (S.UNSUPPORTED_SHAPE, S.INVALID_ARG)
+
+
+def test_head_tiling_sizes_and_arguments(lib):
+    S, L = lib.Status, lib.library
+    # whole 16-row tiles: 157,184 rows are 9,824 tiles; 4,100 rows round up to 4,112
+    assert L.lmhead_tiled_bytes(157184, 2560) == 157184 * 2560
+    assert L.lmhead_tiled_bytes(4100, 256) == 4112 * 256
+    assert L.lmhead_tiled_bytes(4096, 100) == 0 and L.lmhead_tiled_bytes(0, 256) == 0
+    src, dst = lib._Fp8Head(3, 4096, 256, A, A), lib._Fp8Head(0, 4096, 256, A, A)
+    tile = lambda a, b: L.lmhead_tile_fp8(ctypes.byref(a), ctypes.byref(b), None)
+    assert tile(lib._Fp8Head(5, 4096, 256, A, A), dst) == S.FORMAT_MISMATCH      # already tiled
+    assert tile(src, lib._Fp8Head(0, 4095, 256, A, A)) == S.INVALID_ARG         # sizes differ
+    assert tile(src, lib._Fp8Head(0, 4096, 256, U, A)) == S.MISALIGNED
+    assert tile(src, lib._Fp8Head(0, 4096, 256, 0, A)) == S.INVALID_ARG
 
 
 def test_quantizers_reject_bad_arguments(lib):

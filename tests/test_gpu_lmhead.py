@@ -28,10 +28,11 @@ def O():
 
 def _head(B, O, seed, shape):
     w = I.lmhead_weight(seed, shape)
-    head = B.lmhead_quantize_fp8(w.cuda())
+    canon = B.lmhead_quantize_fp8(w.cuda(), tiled=False)
     q, s = O.fp8_rowquant(u16(w))
     torch.cuda.synchronize()
-    assert np.array_equal(head.q.cpu().numpy(), q)
+    assert np.array_equal(canon.q.cpu().numpy(), q)
+    head = B.lmhead_tile_fp8(canon)
     return w, head, q, s
 
 

@@ -84,3 +84,28 @@ def test_pack_of_ling_shared_expert(B):
     want_gu, want_dn = expected_packed(*canon)
     assert np.array_equal(packed.gateup.cpu().numpy(), want_gu)
     assert np.array_equal(packed.down.cpu().numpy(), want_dn)
+
+
+def expected_tiled_head(q):
+    """numpy: the [V][H] E4M3 head -> the tiled bytes moe_gemv.h documents for
+    MOE_FMT_FP8_E4M3_TILED (whole 16-row tiles, zero rows past V; per 64-byte
+    K slice, [half][lane][16 bytes] = row (lane >> 2) + 8 half, bytes
+    64 s + 16 (lane & 3) ...)."""
+    V, H = q.shape
+    T = (V + 15) // 16
+    padded = np.zeros((T * 16, H), dtype=np.uint8)
+    padded[:V] = q
+    t = padded.reshape(T, 2, 8, H // 64, 4, 16)          # [tile][half][g][slice][tq][16]
+    return t.transpose(0, 3, 1, 2, 4, 5).reshape(-1)     # [tile][slice][half][g][tq][16]
+
+
+@pytest.mark.parametrize("V,H", [(4100, 320), (157184 // 16, 2560)])
+def test_fp8_head_tiles_match_documented_layout(B, V, H):
+    g = torch.Generator().manual_seed(V + H)
+    w = (torch.randn((V, H), generator=g) * 0.02).to(torch.bfloat16)
+    canon = B.lmhead_quantize_fp8(w.cuda(), tiled=False)
+    tiled = B.lmhead_tile_fp8(canon)
+    torch.cuda.synchronize()
+    assert tiled.fmt == B.Format.FP8_E4M3_TILED and (tiled.vocab, tiled.hidden) == (V, H)
+    assert tiled.row_scale.data_ptr() == canon.row_scale.data_ptr()
+    assert np.array_equal(tiled.q.cpu().numpy(), expected_tiled_head(canon.q.cpu().numpy()))

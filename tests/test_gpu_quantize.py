@@ -100,7 +100,7 @@ def test_fp8_rowquant_random_and_adversarial(B, O):
     w[4, :] = torch.linspace(-3, 3, 320)
     w[5, :] = 448.0 * 3                # amax / 448 exactly representable
     wb = w.to(torch.bfloat16)
-    head = B.lmhead_quantize_fp8(wb.cuda())
+    head = B.lmhead_quantize_fp8(wb.cuda(), tiled=False)
     torch.cuda.synchronize()
     q_ref, s_ref = O.fp8_rowquant(u16(wb))
     assert head.fmt == B.Format.FP8_E4M3_ROWSCALE_F32
@@ -112,7 +112,7 @@ def test_fp8_rowquant_random_and_adversarial(B, O):
 def test_fp8_rowquant_full_head(B, O):
     """The 157,184 x 2,560 head: every scale and every byte against the oracle."""
     w = I.lmhead_weight(0, I.LING_HEAD)
-    head = B.lmhead_quantize_fp8(w.cuda())
+    head = B.lmhead_quantize_fp8(w.cuda(), tiled=False)
     torch.cuda.synchronize()
     q_ref, s_ref = O.fp8_rowquant(u16(w))
     assert np.array_equal(head.row_scale.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
