@@ -168,12 +168,20 @@ __device__ void warp_topk_rows(const float* vals, int n, int64_t row0, int k, in
   // 1. group maxima: value i is in group i mod 64 (lane i mod 32, row (i / 32) mod 2)
   float m0 = -FLT_MAX, m1 = -FLT_MAX;
   int32_t j0 = INT32_MAX, j1 = INT32_MAX;
-  for (int b = 0; b < n; b += 64) {  // 2 loads in flight per step
-    const int i0 = b + lane, i1 = b + 32 + lane;
-    const float v0 = i0 < n ? vals[i0] : -FLT_MAX, v1 = i1 < n ? vals[i1] : -FLT_MAX;
-    const int32_t id0 = (int32_t)(row0 + i0), id1 = (int32_t)(row0 + i1);
-    if (i0 < n && better(v0, id0, m0, j0)) { m0 = v0; j0 = id0; }
-    if (i1 < n && better(v1, id1, m1, j1)) { m1 = v1; j1 = id1; }
+  for (int b = 0; b < n; b += 256) {  // 8 loads in flight per step
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = b + 32 * u + lane;
+      v[u] = i < n ? vals[i] : -FLT_MAX;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u += 2) {
+      const int i0 = b + 32 * u + lane, i1 = i0 + 32;
+      const int32_t id0 = (int32_t)(row0 + i0), id1 = (int32_t)(row0 + i1);
+      if (i0 < n && better(v[u], id0, m0, j0)) { m0 = v[u]; j0 = id0; }
+      if (i1 < n && better(v[u + 1], id1, m1, j1)) { m1 = v[u + 1]; j1 = id1; }
+    }
   }
   // 2. L = the k-th best group maximum
   int r0 = 0, r1 = 0;
@@ -200,15 +208,23 @@ __device__ void warp_topk_rows(const float* vals, int n, int64_t row0, int k, in
   // 3. candidates: admissible values not worse than L, gathered in one pass
   //    (a ballot per 32 values gives each its slot)
   int nc = 0;
-  for (int b = 0; b < n; b += 32) {
-    const int i = b + lane;
-    const float v = i < n ? vals[i] : -FLT_MAX;
-    const int32_t id = (int32_t)(row0 + i);
-    const bool keep = i < n && v >= -FLT_MAX && !better(Lv, Li, v, id);
-    const uint32_t bal = __ballot_sync(kFull, keep);
-    const int pos = nc + __popc(bal & ((1u << lane) - 1u));
-    if (keep && pos < kCandCap) scratch[pos] = Cand{v, id};
-    nc += __popc(bal);
+  for (int b = 0; b < n; b += 256) {  // 8 loads in flight per step
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = b + 32 * u + lane;
+      v[u] = i < n ? vals[i] : -FLT_MAX;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = b + 32 * u + lane;
+      const int32_t id = (int32_t)(row0 + i);
+      const bool keep = i < n && v[u] >= -FLT_MAX && !better(Lv, Li, v[u], id);
+      const uint32_t bal = __ballot_sync(kFull, keep);
+      const int pos = nc + __popc(bal & ((1u << lane) - 1u));
+      if (keep && pos < kCandCap) scratch[pos] = Cand{v[u], id};
+      nc += __popc(bal);
+    }
   }
   __syncwarp();
   if (nc <= kCandCap) {
@@ -216,8 +232,11 @@ __device__ void warp_topk_rows(const float* vals, int n, int64_t row0, int k, in
     for (int q = lane; q < nc; q += 32) {
       const Cand e = scratch[q];
       int r = 0;
-#pragma unroll 4
-      for (int o = 0; o < nc; ++o) r += better(scratch[o].v, scratch[o].id, e.v, e.id);
+#pragma unroll 8
+      for (int o = 0; o < nc; ++o) {
+        const Cand f = scratch[o];
+        r += better(f.v, f.id, e.v, e.id);
+      }
       if (r < k) out[r] = e;
     }
     for (int j = nc + lane; j < k; j += 32) out[j] = Cand{-FLT_MAX, INT32_MAX};
@@ -248,10 +267,10 @@ __device__ void head_tail(const float* cvals, int n_cap, Cand* warp_scratch, int
     const int n_local = (int)((t_end * kTileRows < V ? t_end * kTileRows : V) - row0);
     warp_topk_rows(cvals + (size_t)warp * n_cap, n_local, row0, top_k, lane,
                    warp_scratch + warp * kCandCap, cand + ((size_t)blockIdx.x * M + warp) * top_k);
+    __threadfence();  // this list, before the CTA counts itself done (only the lists are read by the merge)
   }
 
   // ------------------------- all lists written? ----------------------------
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
     const uint32_t tk = atomicAdd(&hdr->ticket, 1u);
@@ -292,7 +311,11 @@ __device__ void head_tail(const float* cvals, int n_cap, Cand* warp_scratch, int
     for (int c = threadIdx.x; c < G; c += blockDim.x) {
       const Cand h = heads[c];
       int rank = 0;
-      for (int o = 0; o < G; ++o) rank += better(heads[o].v, heads[o].id, h.v, h.id);
+#pragma unroll 8
+      for (int o = 0; o < G; ++o) {
+        const Cand e = heads[o];
+        rank += better(e.v, e.id, h.v, h.id);
+      }
       if (rank == top_k - 1) *s_bound = h;
     }
     __syncthreads();
@@ -315,7 +338,11 @@ __device__ void head_tail(const float* cvals, int n_cap, Cand* warp_scratch, int
     for (int i = threadIdx.x; i < ns; i += blockDim.x) {
       const Cand e = surv[i];
       int rank = 0;
-      for (int o = 0; o < ns; ++o) rank += better(surv[o].v, surv[o].id, e.v, e.id);
+#pragma unroll 8
+      for (int o = 0; o < ns; ++o) {
+        const Cand f = surv[o];
+        rank += better(f.v, f.id, e.v, e.id);
+      }
       if (rank < top_k) {
         out_ids[m * top_k + rank] = e.id;
         out_vals[m * top_k + rank] = e.v;
