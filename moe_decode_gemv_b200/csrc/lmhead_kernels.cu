@@ -652,9 +652,10 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
 // loads straight into registers (no shared-memory staging), which reaches a
 // higher rate on this part than a ring of bulk copies.
 // ---------------------------------------------------------------------------
-constexpr int kTiledConsumers = 20;  // 40 slices of the 2,560-wide head: 2 per warp
+constexpr int kTiledConsumers = 10;  // 40 slices of the 2,560-wide head: 4 per warp
+constexpr int kTilesInFlight = 3;    // tiles whose loads a consumer warp keeps outstanding
 constexpr int kTiledThreads = (kTiledConsumers + kEpilogueWarps) * 32;
-constexpr int kTiledMaxSlices = 4;   // slices per warp: H <= 4 * 20 * 64 = 5120
+constexpr int kTiledMaxSlices = 80 / kTiledConsumers;  // slices per warp: H <= 80 * 64 = 5120
 
 __global__ void tile_fp8_head_kernel(const uint8_t* __restrict__ q, int64_t V, int H, uint8_t* __restrict__ out) {
   const int64_t ntiles = (V + kTileRows - 1) / kTileRows;
@@ -776,7 +777,7 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
       }
     }
     // A fragments straight from HBM: the next tile's loads are issued before
-    // this tile's MMAs (two tiles in flight per warp, ~80 KB per SM).  Warp 0
+    // this tile's MMAs (three tiles in flight per warp, ~120 KB per SM).  Warp 0
     // also loads the tile's row scales.
     struct TileRegs {
       uint4 a[kSlices], b[kSlices];  // rows g and g + 8
@@ -817,7 +818,23 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
       if (lane == 0) mbar_arrive(&red_full[r]);
     };
     int64_t it = 0;
-    if constexpr (kSlices <= 2) {
+    if constexpr (kTilesInFlight == 3 && kSlices <= 4) {
+      TileRegs R0, R1, R2;
+      int64_t t = t_begin;
+      if (t < t_end) load_tile(t, R0);
+      if (t + 1 < t_end) load_tile(t + 1, R1);
+      while (t < t_end) {
+        if (t + 2 < t_end) load_tile(t + 2, R2);
+        compute(R0, it++);
+        if (++t >= t_end) break;
+        if (t + 2 < t_end) load_tile(t + 2, R0);
+        compute(R1, it++);
+        if (++t >= t_end) break;
+        if (t + 2 < t_end) load_tile(t + 2, R1);
+        compute(R2, it++);
+        ++t;
+      }
+    } else if constexpr (kSlices <= 2 * (20 / kTiledConsumers)) {
       TileRegs R0, R1;
       int64_t t = t_begin;
       if (t < t_end) load_tile(t, R0);
@@ -829,7 +846,7 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
         compute(R1, it++);
         ++t;
       }
-    } else {  // wider rows: one tile in flight per warp (registers)
+    } else {  // wide rows: one tile in flight per warp (registers)
       TileRegs R0;
       for (int64_t t = t_begin; t < t_end; ++t) {
         load_tile(t, R0);
@@ -838,7 +855,7 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
     }
   } else {
     // ------------------------------ epilogue ------------------------------
-    // Two epilogue warps take alternate tiles: sum the 20 partials, apply the
+    // Two epilogue warps take alternate tiles: sum the consumers' partials, apply the
     // row scale and 2^-sigma_m, write logits when asked, and keep each value
     // in shared memory for this CTA's top-k, taken after the stream.
     const int ew = warp - kTiledConsumers;  // 0 or 1
@@ -995,13 +1012,14 @@ cudaError_t launch_lmhead_fp8(const uint16_t* x, const uint8_t* qt, const float*
   int stages = 0;
   size_t smem = 0;
   if (!lmhead_plan(H, 1, M, top_k, V, grid, &stages, &smem)) return cudaErrorInvalidConfiguration;
-  switch ((H / 64 + kTiledConsumers - 1) / kTiledConsumers) {
-    case 1: return launch_tiled_t<1>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
-    case 2: return launch_tiled_t<2>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
-    case 3: return launch_tiled_t<3>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
-    case 4: return launch_tiled_t<4>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
-    default: return cudaErrorInvalidValue;
-  }
+  const int need = (H / 64 + kTiledConsumers - 1) / kTiledConsumers;
+  if (need <= 1) return launch_tiled_t<1>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
+  if (need <= 2) return launch_tiled_t<2>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
+  if (need <= kTiledMaxSlices / 2)
+    return launch_tiled_t<kTiledMaxSlices / 2>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
+  if (need <= kTiledMaxSlices)
+    return launch_tiled_t<kTiledMaxSlices>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_lmhead_bf16(const uint16_t* x, const uint16_t* w, int64_t V, int H, int M, int top_k,
