@@ -419,6 +419,7 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
   // per-token power-of-two scale for the f16 activations (fp8 head only)
   if (warp < M) {
     float amax = 0.f;
+#pragma unroll 8
     for (int j = lane; j < H; j += 32) amax = fmaxf(amax, fabsf(bf16_bits_to_f32(x[(size_t)warp * H + j])));
     amax = warp_max(amax);
     if (lane == 0) {
@@ -702,6 +703,35 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t_begin = ntiles * blockIdx.x / gridDim.x;
   const int64_t t_end = ntiles * (blockIdx.x + 1) / gridDim.x;
+  const int g = lane >> 2, tq = lane & 3;
+
+  // A fragments straight from HBM: the next tile's loads are issued before
+  // this tile's MMAs (three tiles in flight per warp, ~120 KB per SM).  Warp 0
+  // also loads the tile's row scales.
+  struct TileRegs {
+    uint4 a[kSlices], b[kSlices];  // rows g and g + 8
+    float sc;
+  };
+  auto load_tile = [&](int64_t t, TileRegs& R) {
+    const uint8_t* tb = qt + (size_t)t * kTileRows * H + lane * 16;
+#pragma unroll
+    for (int si = 0; si < kSlices; ++si) {
+      const int slice = warp + si * kTiledConsumers;
+      const bool in = slice < nsl;
+      R.a[si] = in ? ld_stream_u4(tb + (size_t)slice * 1024) : make_uint4(0u, 0u, 0u, 0u);
+      R.b[si] = in ? ld_stream_u4(tb + (size_t)slice * 1024 + 512) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const int64_t row = t * kTileRows + lane;
+    R.sc = (warp == 0 && lane < kTileRows && row < V) ? __ldg(row_scale + row) : 1.0f;
+  };
+  // Tiles whose loads go out before anything else (they do not depend on the
+  // activations): the consumers' first tiles are in flight during the prologue.
+  constexpr int kPre = (kTilesInFlight == 3 && kSlices <= 4) ? 2 : (kSlices <= 2 * (20 / kTiledConsumers) ? 1 : 0);
+  TileRegs R0, R1, R2;
+  if (warp < kTiledConsumers) {
+    if (kPre >= 1 && t_begin < t_end) load_tile(t_begin, R0);
+    if (kPre >= 2 && t_begin + 1 < t_end) load_tile(t_begin + 1, R1);
+  }
 
   if (threadIdx.x == 0) {
     for (int r = 0; r < kRed; ++r) {
@@ -713,6 +743,7 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
   }
   if (warp < M) {  // per-token power of two: max |x * 2^sigma| in [2^7, 2^8), inside E4M3's normal range
     float amax = 0.f;
+#pragma unroll 8
     for (int j = lane; j < H; j += 32) amax = fmaxf(amax, fabsf(bf16_bits_to_f32(x[(size_t)warp * H + j])));
     amax = warp_max(amax);
     if (lane == 0) {
@@ -742,7 +773,6 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
 
   if (warp < kTiledConsumers) {
     // ------------------------------ consumers -----------------------------
-    const int g = lane >> 2, tq = lane & 3;
     // B fragments, resident for the whole kernel: column n is part n & 1 of
     // token n >> 1 -- the token, scaled by 2^sigma, split into two E4M3 parts
     // x' = hi + lo, exact for every element above E4M3's subnormal range
@@ -776,25 +806,6 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
         }
       }
     }
-    // A fragments straight from HBM: the next tile's loads are issued before
-    // this tile's MMAs (three tiles in flight per warp, ~120 KB per SM).  Warp 0
-    // also loads the tile's row scales.
-    struct TileRegs {
-      uint4 a[kSlices], b[kSlices];  // rows g and g + 8
-      float sc;
-    };
-    auto load_tile = [&](int64_t t, TileRegs& R) {
-      const uint8_t* tb = qt + (size_t)t * kTileRows * H + lane * 16;
-#pragma unroll
-      for (int si = 0; si < kSlices; ++si) {
-        const int slice = warp + si * kTiledConsumers;
-        const bool in = slice < nsl;
-        R.a[si] = in ? ld_stream_u4(tb + (size_t)slice * 1024) : make_uint4(0u, 0u, 0u, 0u);
-        R.b[si] = in ? ld_stream_u4(tb + (size_t)slice * 1024 + 512) : make_uint4(0u, 0u, 0u, 0u);
-      }
-      const int64_t row = t * kTileRows + lane;
-      R.sc = (warp == 0 && lane < kTileRows && row < V) ? __ldg(row_scale + row) : 1.0f;
-    };
     auto compute = [&](const TileRegs& R, int64_t it) {
       float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
@@ -818,11 +829,8 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
       if (lane == 0) mbar_arrive(&red_full[r]);
     };
     int64_t it = 0;
-    if constexpr (kTilesInFlight == 3 && kSlices <= 4) {
-      TileRegs R0, R1, R2;
+    if constexpr (kPre == 2) {  // R0, R1 hold the first two tiles
       int64_t t = t_begin;
-      if (t < t_end) load_tile(t, R0);
-      if (t + 1 < t_end) load_tile(t + 1, R1);
       while (t < t_end) {
         if (t + 2 < t_end) load_tile(t + 2, R2);
         compute(R0, it++);
@@ -834,10 +842,8 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
         compute(R2, it++);
         ++t;
       }
-    } else if constexpr (kSlices <= 2 * (20 / kTiledConsumers)) {
-      TileRegs R0, R1;
+    } else if constexpr (kPre == 1) {  // R0 holds the first tile
       int64_t t = t_begin;
-      if (t < t_end) load_tile(t, R0);
       while (t < t_end) {
         if (t + 1 < t_end) load_tile(t + 1, R1);
         compute(R0, it++);
@@ -847,7 +853,6 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
         ++t;
       }
     } else {  // wide rows: one tile in flight per warp (registers)
-      TileRegs R0;
       for (int64_t t = t_begin; t < t_end; ++t) {
         load_tile(t, R0);
         compute(R0, it++);
