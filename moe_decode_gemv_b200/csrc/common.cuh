@@ -1,10 +1,10 @@
 // common.cuh -- device helpers shared by the sm_100a kernels of this library.
 //
 // Number formats (OCP Microscaling Formats v1.0; OCP 8-bit Floating Point
-// Specification): E2M1 and E4M3 codes are widened with the hardware
-// conversions of sm_100a (cvt.rn.f16x2.e2m1x2 / .e4m3x2), which are exact
-// because every E2M1 and E4M3 value is an f16 value.  E8M0 scales become
-// fp32 by placing the code in the exponent field.
+// Specification): E4M3 codes are widened with the hardware conversion of
+// sm_100a (cvt.rn.f16x2.e4m3x2), exact because every E4M3 value is an f16
+// value; E2M1 codes of the packed expert banks become E5M2 codes by moving
+// bits; E8M0 scales become fp32 by placing the code in the exponent field.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -65,26 +65,11 @@ __device__ __forceinline__ bool bounded_spin(F ready, uint32_t backoff_ns = 64) 
 // Format conversions.
 // ---------------------------------------------------------------------------
 
-// Two E2M1 codes (low nibble = element 2j, high nibble = element 2j+1) -> f16x2
-// with element 2j in the low half.
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "r"(byte));
-  return r;
-}
-
 // Two E4M3 codes (low byte = lower-index element) -> f16x2, low byte in the low half.
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
   uint32_t r;
   asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "r"(two_bytes));
   return r;
-}
-
-// E8M0 code -> fp32 scale 2^(code - 127).  Code 0 is 2^-127 (a subnormal),
-// code 255 is NaN.
-__device__ __forceinline__ float e8m0_to_f32(uint32_t code) {
-  uint32_t bits = code == 0u ? 0x00400000u : (code == 255u ? 0x7fc00000u : code << 23);
-  return __uint_as_float(bits);
 }
 
 // Two fp32 values -> two E4M3 codes, round to nearest even, saturating to
@@ -105,19 +90,6 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
-
-// Eight E2M1 codes (one word, element i in nibble i) -> eight E4M3 codes by
-// moving bits only: E2M1 s|e1 e0|m becomes E4M3 s|0 0 e1 e0|m 0 0, whose
-// value is the E2M1 value times 2^-6 for every code (the E2M1 subnormal 0.5
-// becomes the E4M3 subnormal 2^-7).  `even` gets elements 0, 2, 4, 6 in bytes
-// 0..3 and `odd` elements 1, 3, 5, 7; a caller pairs them with activations
-// permuted the same way.
-__device__ __forceinline__ uint32_t e2m1x8_even_to_e4m3x4(uint32_t w) {
-  return ((w << 2) & 0x1c1c1c1cu) | ((w << 4) & 0x80808080u);
-}
-__device__ __forceinline__ uint32_t e2m1x8_odd_to_e4m3x4(uint32_t w) {
-  return ((w >> 2) & 0x1c1c1c1cu) | (w & 0x80808080u);
-}
 
 // The packed expert banks (pack_kernels.cu) place the two E2M1 codes of a
 // byte as element 2j: sign|e1 e0 m at bits 7|3 2 1 and element 2j+1 at bits
@@ -197,16 +169,6 @@ __device__ __forceinline__ float warp_max(float v) {
 // Branch-free: evaluated with predicates, never a jump.
 __device__ __forceinline__ bool better(float va, int32_t ia, float vb, int32_t ib) {
   return (va > vb) | ((va == vb) & (ia < ib));
-}
-
-// Warp-wide best (value, index) under `better`; every lane gets the result.
-__device__ __forceinline__ void warp_best(float& v, int32_t& i) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    float ov = __shfl_xor_sync(0xffffffffu, v, o);
-    int32_t oi = __shfl_xor_sync(0xffffffffu, i, o);
-    if (better(ov, oi, v, i)) { v = ov; i = oi; }
-  }
 }
 
 // ---------------------------------------------------------------------------
