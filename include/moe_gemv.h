@@ -290,7 +290,8 @@ MOE_API moe_status moe_mtp_accept(const int32_t* draft_ids, const int32_t* verif
  * address (cudaGetSymbolAddress) and should come before any stream capture.
  * Each call clears the array's header on `stream` before its kernel.  All
  * calls share the array, so calls that overlap on the GPU (different
- * streams, or different threads) race: serialise them.  Allocates nothing.  */
+ * streams, or different threads) race: serialise them.  Allocates nothing.
+ * The head is the tiled one, as for lmhead_decode.                         */
 #define MOE_LMHEAD_NOALLOC_SCRATCH_BYTES (256u * 1024u)
 MOE_API moe_status lmhead_decode_noalloc(const uint16_t* hidden_bf16, const moe_fp8_head* head,
                                          int32_t M, int32_t top_k, int32_t* topk_ids, float* topk_vals,
