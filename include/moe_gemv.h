@@ -219,8 +219,13 @@ MOE_API size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts
  *               zeroed once (moe_workspace_reset) before its first use.
  * Supported: H and I multiples of 64, H <= 4096, I <= 1024, E <= 1024,
  * 1 <= top_k <= 8 and top_k <= E.  The call is one cooperative launch
- * (one CTA per SM, all resident).  Each distinct routed expert is streamed once per call, however
- * many of the M tokens chose it.                                             */
+ * (one CTA per SM, all resident).  Each distinct routed expert is streamed
+ * once per call, however many of the M tokens chose it.
+ * E8M0 scales are decoded by one multiply into the fp32 exponent: code 0
+ * contributes 0 instead of 2^-127 times its elements (below 2^-116 of any
+ * product), and code 255 acts as +inf, so a non-finite block as
+ * moe_quantize_mxfp4 writes it (scale 0xFF, zero elements) still turns the
+ * rows that read it into NaN.                                                */
 MOE_API moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const float* router_bias,
                       const moe_packed_bank* experts, const moe_packed_bank* shared,
                       int32_t M, int32_t top_k, float* out, int32_t* topk_ids, float* topk_w,
