@@ -23,9 +23,10 @@
 //    byte far below what the HBM stream allows, at M = 1 and M = 4 alike.
 //  * Activations: each bf16 token is scaled by 2^sigma_m (max |x| into
 //    [2^7, 2^8)) and split into two E4M3 parts hi + lo, which represent the
-//    bf16 value exactly (8 significand bits = 4 + 4) for every element above
-//    E4M3's subnormal range; the two parts take two MMAs.  The logit is
-//    acc * s_v * 2^-sigma_m.
+//    bf16 value exactly (8 significand bits = 4 + 4) when its scaled
+//    magnitude is at least 2^-2 (2^-10 of the token's largest or more); below
+//    that lo is rounded to E4M3's subnormal step, an error under 2^-17 of the
+//    largest.  The logit is acc * s_v * 2^-sigma_m.
 //  * Epilogue: two warps take alternate tiles.  A tile's 16 row scales ride
 //    in its ring stage (one more bulk copy) and reach the epilogue with the
 //    consumers' partial sums, so no global load sits on the epilogue's path.
@@ -480,9 +481,9 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
     const int g = lane >> 2, tq = lane & 3;
     // B fragments: token n = g, this warp's K slices, resident for the whole kernel.
     // FP8 head: the token, scaled by 2^sigma, is split into two E4M3 parts,
-    // x' = hi + lo, exact for every element whose magnitude is above E4M3's
-    // subnormal range (more than 2^-14 of the token's largest).  Each part
-    // takes its own MMA; the weights enter the MMA as raw E4M3 bytes.
+    // x' = hi + lo, exact for every element of scaled magnitude 2^-2 or more
+    // (the rest within 2^-17 of the token's largest).  Each part takes its own
+    // MMA; the weights enter the MMA as raw E4M3 bytes.
     uint32_t bfrag[kSlices][T::kMmasPerSlice][2];
     {
       const bool live = g < M;
@@ -775,9 +776,9 @@ lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
     // ------------------------------ consumers -----------------------------
     // B fragments, resident for the whole kernel: column n is part n & 1 of
     // token n >> 1 -- the token, scaled by 2^sigma, split into two E4M3 parts
-    // x' = hi + lo, exact for every element above E4M3's subnormal range
-    // (more than 2^-14 of the token's largest) -- so one MMA covers both
-    // parts of four tokens.
+    // x' = hi + lo, exact for every element of scaled magnitude 2^-2 or more
+    // (the rest within 2^-17 of the token's largest) -- so one MMA covers
+    // both parts of four tokens.
     uint32_t bfrag[kSlices][2][2];  // [slice][mma][b0, b1]
     {
       const int m = g >> 1, part = g & 1;

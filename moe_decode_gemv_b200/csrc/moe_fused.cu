@@ -43,7 +43,8 @@
 // places each E2M1 code's bits so that a mask (even elements) or two shifts
 // (odd ones) give the E5M2 code of its value times 2^-14.  Activations are
 // scaled by a per-token power of two that puts their largest magnitude in
-// [2^7, 2^8); bf16 x is then carried exactly by two E4M3 parts, which ride in
+// [2^7, 2^8); bf16 x is then carried by two E4M3 parts (exactly for scaled
+// magnitudes of 2^-2 and up, within 2^-17 of the largest below), which ride in
 // two columns of the same MMA.  h is scaled per 32-element block and token
 // (largest magnitude into [2^7, 2^8)) and carried by three E4M3 parts (12
 // significant bits) in three columns; one MMA covers two tokens.
@@ -552,7 +553,8 @@ __global__ void __launch_bounds__(kThreadsAll, 1) moe_fused_kernel(FusedArgs a) 
 
     // x as E4M3 B fragments for this warp's K blocks of the gate/up GEMV.
     // Column n of B is part n & 1 of token n >> 1: each token, scaled by
-    // 2^sigma, is carried exactly by two E4M3 parts (hi, lo), and the two
+    // 2^sigma, is carried by two E4M3 parts (hi, lo; exact for scaled
+    // magnitudes of 2^-2 and up, within 2^-17 of the largest below), and the two
     // parts ride in two columns of ONE MMA (their sum is taken after it).
     // Within a 32-element block, lane (g, tq) covers elements 8tq..8tq+7 of
     // column g: the even ones fill k-slots 4tq..4tq+3 (b0), the odd ones

@@ -1,0 +1,94 @@
+"""Format facts the GPU kernels rely on, checked on the host against an
+independent decoder (ml_dtypes) -- not against the kernels' own code.
+
+* The packed expert banks place element 2j's E2M1 sign|e1 e0 m at bits
+  7|3 2 1 of the byte and element 2j+1's at bits 0|6 5 4.  A mask (even
+  element) or two shifts (odd element) then give a byte that, read as E5M2,
+  is the E2M1 value times 2^-14 -- for all 16 codes, subnormal and zeros
+  included.
+* E8M0 code c placed in the fp32 exponent field (c << 23) is 2^(c-127) for
+  c = 1..254; code 0 gives +0 and code 255 gives +inf (the kernels' documented
+  departure from the spec's 2^-127 and NaN).
+* An E4M3 hi/lo split carries a bf16 value (the token scaled so that its
+  largest magnitude is in [2^7, 2^8)) exactly when the scaled magnitude is
+  at least 2^-2, and within 2^-10 below that.
+"""
+import itertools
+
+import ml_dtypes
+import numpy as np
+import pytest
+
+
+def e2m1(code):
+    return float(np.array([code], np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)[0])
+
+
+def e5m2(byte):
+    return float(np.array([byte], np.uint8).view(ml_dtypes.float8_e5m2).astype(np.float64)[0])
+
+
+def relayout(lo, hi):
+    """The packer's bit placement of one byte (lo = element 2j, hi = 2j+1)."""
+    return ((lo >> 3) << 7) | ((lo & 7) << 1) | (hi >> 3) | ((hi & 7) << 4)
+
+
+def even_e5m2(byte):
+    return byte & 0x8E
+
+
+def odd_e5m2(byte):
+    return ((byte >> 3) & 0x0E) | ((byte << 7) & 0x80)
+
+
+@pytest.mark.parametrize("lo,hi", list(itertools.product(range(16), range(16))))
+def test_packed_nibbles_unpack_to_e5m2(lo, hi):
+    b = relayout(lo, hi)
+    assert 0 <= b < 256
+    # the placement is a bijection on bytes: both codes are recoverable
+    assert e5m2(even_e5m2(b)) == e2m1(lo) * 2.0 ** -14
+    assert e5m2(odd_e5m2(b)) == e2m1(hi) * 2.0 ** -14
+
+
+def test_word_level_unpack_keeps_bytes_apart():
+    """The 32-bit forms act byte by byte: no bit crosses into a neighbour."""
+    rng = np.random.default_rng(0)
+    for _ in range(2000):
+        codes = rng.integers(0, 16, size=8)
+        w = 0
+        for j in range(4):
+            w |= relayout(int(codes[2 * j]), int(codes[2 * j + 1])) << (8 * j)
+        even = w & 0x8E8E8E8E
+        odd = ((w >> 3) & 0x0E0E0E0E) | ((w << 7) & 0x80808080)
+        for j in range(4):
+            assert e5m2((even >> (8 * j)) & 0xFF) == e2m1(int(codes[2 * j])) * 2.0 ** -14
+            assert e5m2((odd >> (8 * j)) & 0xFF) == e2m1(int(codes[2 * j + 1])) * 2.0 ** -14
+
+
+def test_e8m0_by_exponent_placement():
+    bits = (np.arange(256, dtype=np.uint64) << 23).astype(np.uint32)
+    f = bits.view(np.float32).astype(np.float64)
+    for c in range(1, 255):
+        assert f[c] == 2.0 ** (c - 127)
+    assert f[0] == 0.0 and np.isposinf(f[255])
+    # the spec values the kernels depart from: 2^-127 and NaN
+    spec = np.array([0, 255], np.uint8).view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    assert spec[0] == 2.0 ** -127 and np.isnan(spec[1])
+
+
+def test_bf16_is_carried_by_two_e4m3_parts():
+    """A bf16 value v, scaled so that the token's largest magnitude is in
+    [2^7, 2^8), equals hi + lo (hi = rne_e4m3(v), lo = rne_e4m3(v - hi)) when
+    |v| >= 2^-2: 8 significant bits = 4 + 4 with lo's last bit at or above
+    E4M3's subnormal step 2^-9.  Below 2^-2 the error is at most half that
+    step, 2^-10, under 2^-17 of the token's largest."""
+    e4m3 = ml_dtypes.float8_e4m3fn
+    vals = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16).view(ml_dtypes.bfloat16).astype(np.float64)
+    vals = vals[np.isfinite(vals) & (np.abs(vals) < 2.0 ** 8)]
+    hi = vals.astype(np.float32).astype(e4m3).astype(np.float64)
+    lo = (vals - hi).astype(np.float32).astype(e4m3).astype(np.float64)
+    big = np.abs(vals) >= 2.0 ** -2
+    assert np.array_equal((hi + lo)[big], vals[big])
+    assert np.abs((hi + lo) - vals)[~big].max() <= 2.0 ** -10
+    # the bound is tight: some value just below 2^-2 is not carried exactly
+    assert (np.abs((hi + lo) - vals)[~big] > 0).any()
