@@ -142,6 +142,7 @@ def test_ling_layer(B, O, ling, M):
         x = I.hidden_states(seed, M, I.LING_MOE.hidden, tag=f"ling{M}")
         y, ids, w = ling.run_gpu(x.cuda())
         rep = check_moe(ling, O, x, y, ids, w)
+        print(f"ling layer M={M} seed={seed}: rel-L2 {rep['rel_l2']:.2e}, max-abs {rep['max_abs']:.2e}")
         assert rep["skipped_tokens"] == 0, rep
         if M == 4:
             assert len(set(ids.reshape(-1).tolist())) <= 32
