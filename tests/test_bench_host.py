@@ -92,7 +92,7 @@ def test_traffic_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch)
     assert bench.profiled_traffic() is None
 
 
-def test_workload_config_names_the_configs():
+def test_workload_config_names_the_workload():
     bench = _bench()
     cfg = bench.workload_config()
     assert cfg["hidden"] == 2560 and cfg["expert_inter"] == 768 and cfg["experts"] == 512
