@@ -114,28 +114,35 @@ typedef struct {
 } moe_expert_bank;
 
 /* An expert bank re-laid out for moe_decode (moe_pack_experts): the same
- * MXFP4 bytes, grouped so that each unit of the kernel's work is one
- * contiguous run that a single bulk copy moves.
- *   gateup [count][I/8][16 * (H/2 + H/32) bytes]: for each 8-row chunk q of an
- *          expert, gate rows 8q..8q+7 then up rows 8q..8q+7 (H/2 bytes each),
- *          then the 8 gate scale rows and the 8 up scale rows (H/32 bytes each);
- *   down   [count][H/32][32 * (I/2 + I/32) bytes]: for each 32-row tile t,
- *          down rows 32t..32t+31 (I/2 bytes each), then their 32 scale rows.
- * Within a data row, the 16-byte unit c (one 32-element block) of row r is
- * stored at position c ^ (r & mask), mask = min(8, largest power of two
- * dividing the units per row) - 1, so that eight consecutive rows read
- * together hit distinct shared-memory banks.  Within every data byte the
- * bits of its two E2M1 codes are re-placed: element 2j's sign, e1, e0, m go
- * to bits 7, 3, 2, 1 and element 2j+1's to bits 0, 6, 5, 4 (scale bytes are
- * unchanged).  fmt must be MOE_FMT_MXFP4_MOE_PACKED.  The pages have no
- * counterpart for this layout; it moves bits, never changes a value.          */
+ * MXFP4 bytes, grouped by the kernel's work items.  An item (e, j) is 16 rows
+ * of expert e's intermediate dimension: gate and up rows 16j .. 16j+15 and
+ * down columns 16j .. 16j+15.
+ *   units   [count][inter/16][25 * hidden bytes]: item (e, j)'s bytes, one
+ *           contiguous run in the order of the kernel's MMA fragments:
+ *     A (hidden/32 blocks x 512 B): for K block b and lane l = 4g + t
+ *       (g = l >> 2, t = l & 3), 16 bytes = the 4-byte words t of block b of
+ *       gate row 16j+g, up row 16j+g, gate row 16j+8+g and up row 16j+8+g
+ *       (word t of a block holds elements 32b + 8t .. 32b + 8t + 7);
+ *     B (hidden/32 x 32 B): for block b and g, the E8M0 scales of block b of
+ *       those four rows, in the same order;
+ *     C (hidden/32 groups x 256 B): for 32-row group G and lane l = 4g + t,
+ *       8 bytes = 2 bytes (columns 16j + 4t .. 16j + 4t + 3) of each of down
+ *       rows 32G + g, 32G + 8 + g, 32G + 16 + g and 32G + 24 + g;
+ *   dscales [count][inter/32][hidden]: the down scales of each 32-column
+ *           pair p (shared by items 2p and 2p+1); byte 32G + 4g + r is the
+ *           scale of down row 32G + 8r + g, block p.
+ * Within every data byte the bits of its two E2M1 codes are re-placed:
+ * element 2j's sign, e1, e0, m go to bits 7, 3, 2, 1 and element 2j+1's to
+ * bits 0, 6, 5, 4 (scale bytes are unchanged).  fmt must be
+ * MOE_FMT_MXFP4_MOE_PACKED.  The pages have no counterpart for this layout;
+ * it moves bits, never changes a value.                                      */
 typedef struct {
     int32_t fmt;
     int32_t count;
     int32_t hidden;
     int32_t inter;
-    uint8_t* gateup;
-    uint8_t* down;
+    uint8_t* units;
+    uint8_t* dscales;
 } moe_packed_bank;
 
 /* The online-FP8 LM head: q E4M3 and row_scale [vocab] fp32.
@@ -173,13 +180,14 @@ typedef struct {
 MOE_API moe_status moe_quantize_mxfp4(const uint16_t* w_bf16, moe_mxfp4_tensor* out, void* stream);
 
 /* Bytes of the two packed arrays of a bank with `count` experts (0 if the
- * sizes are unsupported: hidden and inter multiples of 64).                  */
-MOE_API size_t moe_packed_gateup_bytes(int32_t count, int32_t hidden, int32_t inter);
-MOE_API size_t moe_packed_down_bytes(int32_t count, int32_t hidden, int32_t inter);
+ * sizes are unsupported: hidden and inter multiples of 32).                  */
+MOE_API size_t moe_packed_units_bytes(int32_t count, int32_t hidden, int32_t inter);
+MOE_API size_t moe_packed_dscales_bytes(int32_t count, int32_t hidden, int32_t inter);
 
 /* Re-lay out a quantised bank (`src`: gate and up count x [I][H], down
  * count x [H][I], all tagged MXFP4) into `dst`, whose caller fills count,
- * hidden, inter and the two device arrays (sizes above, 16-byte aligned).
+ * hidden, inter and the two device arrays (units, dscales: sizes above,
+ * 16-byte aligned).
  * Enqueued on `stream`; on success sets dst->fmt.  The source is not needed
  * by moe_decode afterwards.                                                  */
 MOE_API moe_status moe_pack_experts(const moe_expert_bank* src, moe_packed_bank* dst, void* stream);
@@ -217,10 +225,19 @@ MOE_API size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts
  *   topk_w      [M][top_k] fp32 or NULL:  renormalised softmax weights
  *   workspace   device buffer of at least moe_workspace_bytes(...) bytes,
  *               zeroed once (moe_workspace_reset) before its first use.
- * Supported: H and I multiples of 64, H <= 4096, I <= 1024, E <= 1024,
- * 1 <= top_k <= 8 and top_k <= E.  The call is one cooperative launch
- * (one CTA per SM, all resident).  Each distinct routed expert is streamed
- * once per call, however many of the M tokens chose it.
+ * Supported: H and I multiples of 32, 32 <= H <= 4096, 32 <= I <= 65536,
+ * E <= 1024, 1 <= top_k <= 8 and top_k <= E.  The call is one cooperative
+ * launch (one CTA per SM, all resident).  Each distinct routed expert is
+ * streamed once per call, however many of the M tokens chose it.  The
+ * output is the same on every call with the same inputs (a fixed summation
+ * order on a given GPU).
+ * Arithmetic: fp32 sums of exact products of the E2M1 weights with parts
+ * of the activations.  x, per token and 32-element block scaled by a power
+ * of two, is split into two E4M3 parts: exact for bf16 values down to 2^-10
+ * of the block's largest magnitude, within 2^-17 of it below.  h, per token
+ * and 16 values scaled likewise, is split into two f16 parts (about 22
+ * significant bits).  Activations and h must stay below 2^120 in magnitude;
+ * every smaller bf16 value, subnormals included, is carried as above.
  * E8M0 scales are decoded by one multiply into the fp32 exponent: code 0
  * contributes 0 instead of 2^-127 times its elements (below 2^-116 of any
  * product), and code 255 acts as +inf, so a non-finite block as

@@ -22,7 +22,7 @@ _BINDING_NAMES = {
     "moe_decode", "lmhead_decode", "lmhead_decode_bf16", "lmhead_decode_noalloc",
     "lmhead_sample", "moe_mtp_accept", "moe_rmsnorm_bf16", "moe_embed_gather", "moe_stream_read",
     "moe_workspace_bytes", "lmhead_workspace_bytes", "new_workspace", "moe_workspace_status",
-    "moe_query_path", "moe_get_device_status", "MXFP4Bank", "PackedBank", "FP8Head",
+    "moe_query_path", "MXFP4Bank", "PackedBank", "FP8Head",
     "alloc_mxfp4_bank", "alloc_fp8_head",
 }
 

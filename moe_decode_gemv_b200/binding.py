@@ -57,7 +57,7 @@ class _Bank(ctypes.Structure):
 
 class _Packed(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("count", ctypes.c_int32), ("hidden", ctypes.c_int32),
-                ("inter", ctypes.c_int32), ("gateup", ctypes.c_void_p), ("down", ctypes.c_void_p)]
+                ("inter", ctypes.c_int32), ("units", ctypes.c_void_p), ("dscales", ctypes.c_void_p)]
 
 
 class _Fp8Head(ctypes.Structure):
@@ -82,8 +82,8 @@ def _load() -> ctypes.CDLL:
         "lmhead_tiled_bytes": ([I64, I64], SZ),
         "lmhead_tile_fp8": ([ctypes.POINTER(_Fp8Head), ctypes.POINTER(_Fp8Head), P], I32),
         "moe_workspace_bytes": ([I32, I32, I32, I32, I32], SZ),
-        "moe_packed_gateup_bytes": ([I32, I32, I32], SZ),
-        "moe_packed_down_bytes": ([I32, I32, I32], SZ),
+        "moe_packed_units_bytes": ([I32, I32, I32], SZ),
+        "moe_packed_dscales_bytes": ([I32, I32, I32], SZ),
         "moe_pack_experts": ([ctypes.POINTER(_Bank), ctypes.POINTER(_Packed), P], I32),
         "moe_decode": ([P, P, P, ctypes.POINTER(_Packed), ctypes.POINTER(_Packed), I32, I32, P, P, P, P, SZ, P], I32),
         "lmhead_workspace_bytes": ([I32, I32, I64, I64], SZ),
@@ -164,22 +164,22 @@ def alloc_mxfp4_bank(count: int, rows: int, K: int, device="cuda") -> MXFP4Bank:
 
 @dataclass
 class PackedBank:
-    """An expert bank laid out for moe_decode (moe_pack_experts): gateup
-    [count * I/8 * 16 (H/2 + H/32)] and down [count * H/32 * 32 (I/2 + I/32)]
-    uint8, the MXFP4 bytes grouped into one contiguous run per unit of the
-    kernel's work."""
-    gateup: torch.Tensor
-    down: torch.Tensor
+    """An expert bank laid out for moe_decode (moe_pack_experts): units
+    [count * I/16 * 25 H] uint8 (one contiguous run per 16-row work item) and
+    dscales [count * I/32 * H] uint8 (the down scales of each 32-column pair)."""
+    units: torch.Tensor
+    dscales: torch.Tensor
     count: int
     hidden: int
     inter: int
     fmt: int = Format.NONE
 
     def _c(self) -> _Packed:
-        return _Packed(int(self.fmt), self.count, self.hidden, self.inter, self.gateup.data_ptr(), self.down.data_ptr())
+        return _Packed(int(self.fmt), self.count, self.hidden, self.inter, self.units.data_ptr(),
+                       self.dscales.data_ptr())
 
     def nbytes(self) -> int:
-        return self.gateup.numel() + self.down.numel()
+        return self.units.numel() + self.dscales.numel()
 
 
 @dataclass
@@ -229,8 +229,8 @@ def moe_pack_experts(bank: tuple[MXFP4Bank, MXFP4Bank, MXFP4Bank], stream=None) 
     """(gate, up, down) quantised banks -> the packed bank moe_decode reads."""
     gate, up, down = bank
     E, H, I = gate.count, gate.K, gate.rows
-    gb = int(library.moe_packed_gateup_bytes(E, H, I))
-    db = int(library.moe_packed_down_bytes(E, H, I))
+    gb = int(library.moe_packed_units_bytes(E, H, I))
+    db = int(library.moe_packed_dscales_bytes(E, H, I))
     if gb == 0 or db == 0:
         raise MoEError(Status.UNSUPPORTED_SHAPE, "moe_pack_experts")
     dev = gate.data.device
@@ -400,7 +400,3 @@ def moe_query_path() -> str:
     buf = ctypes.create_string_buffer(1024)
     _check(library.moe_query_path(buf, len(buf)), "moe_query_path")
     return buf.value.decode()
-
-
-def moe_get_device_status(workspace: torch.Tensor, stream=None) -> Status:
-    return moe_workspace_status(workspace, stream)

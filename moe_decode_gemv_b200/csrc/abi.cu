@@ -41,15 +41,15 @@ moe_status check_bank(const moe_expert_bank* b, int64_t count, int64_t H, int64_
 }
 
 bool pack_shape_ok(int64_t count, int64_t H, int64_t I) {
-  return count >= 1 && count <= (int64_t(1) << 20) && H >= 64 && I >= 64 && H % 64 == 0 && I % 64 == 0 &&
+  return count >= 1 && count <= (int64_t(1) << 20) && H >= 32 && I >= 32 && H % 32 == 0 && I % 32 == 0 &&
          H <= 65536 && I <= 65536;
 }
 
 moe_status check_packed(const moe_packed_bank* b, int64_t count, int64_t H, int64_t I) {
   if (b->fmt != MOE_FMT_MXFP4_MOE_PACKED) return MOE_ERR_FORMAT_MISMATCH;
-  if (!b->gateup || !b->down) return MOE_ERR_INVALID_ARG;
+  if (!b->units || !b->dscales) return MOE_ERR_INVALID_ARG;
   if (b->count != count || b->hidden != H || b->inter != I) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(b->gateup) || !aligned16(b->down)) return MOE_ERR_MISALIGNED;
+  if (!aligned16(b->units) || !aligned16(b->dscales)) return MOE_ERR_MISALIGNED;
   return MOE_OK;
 }
 
@@ -138,16 +138,16 @@ moe_status lmhead_tile_fp8(const moe_fp8_head* src, moe_fp8_head* dst, void* str
   return MOE_OK;
 }
 
-size_t moe_packed_gateup_bytes(int32_t count, int32_t hidden, int32_t inter) {
-  return pack_shape_ok(count, hidden, inter) ? moe::packed_gateup_bytes(count, hidden, inter) : 0;
+size_t moe_packed_units_bytes(int32_t count, int32_t hidden, int32_t inter) {
+  return pack_shape_ok(count, hidden, inter) ? moe::packed_units_bytes(count, hidden, inter) : 0;
 }
 
-size_t moe_packed_down_bytes(int32_t count, int32_t hidden, int32_t inter) {
-  return pack_shape_ok(count, hidden, inter) ? moe::packed_down_bytes(count, hidden, inter) : 0;
+size_t moe_packed_dscales_bytes(int32_t count, int32_t hidden, int32_t inter) {
+  return pack_shape_ok(count, hidden, inter) ? moe::packed_dscales_bytes(count, hidden, inter) : 0;
 }
 
 moe_status moe_pack_experts(const moe_expert_bank* src, moe_packed_bank* dst, void* stream) {
-  if (!src || !dst || !dst->gateup || !dst->down) return MOE_ERR_INVALID_ARG;
+  if (!src || !dst || !dst->units || !dst->dscales) return MOE_ERR_INVALID_ARG;
   for (const moe_mxfp4_tensor* t : {&src->gate, &src->up, &src->down})
     if (t->fmt != MOE_FMT_MXFP4_E2M1_E8M0_32) return MOE_ERR_FORMAT_MISMATCH;
   const int64_t E = src->gate.count, H = src->gate.K, I = src->gate.rows;
@@ -155,10 +155,10 @@ moe_status moe_pack_experts(const moe_expert_bank* src, moe_packed_bank* dst, vo
     return MOE_ERR_UNSUPPORTED_SHAPE;
   moe_status s;
   if ((s = check_bank(src, E, H, I)) != MOE_OK) return s;
-  if (!aligned16(dst->gateup) || !aligned16(dst->down)) return MOE_ERR_MISALIGNED;
+  if (!aligned16(dst->units) || !aligned16(dst->dscales)) return MOE_ERR_MISALIGNED;
   cudaError_t e = moe::launch_pack_experts(src->gate.data, src->gate.scales, src->up.data, src->up.scales,
-                                           src->down.data, src->down.scales, E, (int)H, (int)I, dst->gateup,
-                                           dst->down, static_cast<cudaStream_t>(stream));
+                                           src->down.data, src->down.scales, E, (int)H, (int)I, dst->units,
+                                           dst->dscales, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   dst->fmt = MOE_FMT_MXFP4_MOE_PACKED;
   return MOE_OK;
@@ -166,8 +166,8 @@ moe_status moe_pack_experts(const moe_expert_bank* src, moe_packed_bank* dst, vo
 
 size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts, int32_t hidden, int32_t inter) {
   if (M < 1 || M > 4 || top_k < 1 || top_k > 8 || num_experts < 1 || num_experts > 1024) return 0;
-  if (hidden < 64 || inter < 64 || !moe::moe_fused_supported(hidden, inter)) return 0;
-  return moe::moe_ws_bytes(M, top_k, num_experts, hidden, inter);
+  if (!moe::moe_layer_supported(hidden, inter)) return 0;
+  return moe::moe_ws_bytes(num_experts, hidden);
 }
 
 moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const float* router_bias,
@@ -181,7 +181,7 @@ moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const 
     return MOE_ERR_FORMAT_MISMATCH;
   const int64_t E = experts->count, H = experts->hidden, I = experts->inter;
   if (E < 1 || E > 1024 || top_k > E) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (H < 64 || I < 64 || !moe::moe_fused_supported((int)H, (int)I)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!moe::moe_layer_supported((int)H, (int)I)) return MOE_ERR_UNSUPPORTED_SHAPE;
   moe_status s;
   if ((s = check_packed(experts, E, H, I)) != MOE_OK) return s;
   if ((s = check_packed(shared, 1, H, I)) != MOE_OK) return s;
@@ -195,12 +195,12 @@ moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const 
   a.x = hidden_bf16;
   a.router_w = router_w;
   a.router_bias = router_bias;
-  a.bank = moe::MoeBank{experts->gateup, experts->down};
-  a.shared = moe::MoeBank{shared->gateup, shared->down};
+  a.bank = moe::MoeBank{experts->units, experts->dscales};
+  a.shared = moe::MoeBank{shared->units, shared->dscales};
   a.M = M; a.top_k = top_k; a.E = (int)E; a.H = (int)H; a.I = (int)I;
   a.out = out; a.ids_out = topk_ids; a.w_out = topk_w;
-  a.ws = moe::MoeWs::carve(workspace, (int)E, (int)H, (int)I);
-  return cuda_status(moe::launch_moe_fused(a, static_cast<cudaStream_t>(stream)));
+  a.ws = moe::MoeWs::carve(workspace, (int)E, (int)H);
+  return cuda_status(moe::launch_moe_layer(a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t lmhead_workspace_bytes(int32_t M, int32_t top_k, int64_t vocab, int64_t hidden) {
@@ -272,9 +272,10 @@ moe_status moe_workspace_status(void* workspace, void* stream) {
 moe_status moe_query_path(char* buf, size_t n) {
   if (!buf || n == 0) return MOE_ERR_INVALID_ARG;
   const char* desc =
-      "sm_100a; moe: one cooperative persistent kernel (router fp32 GEMV, top-k softmax routing, "
-      "MXFP4 E2M1/E8M0-32 gate/up + SiLU and down over packed banks, one bulk copy per work item, "
-      "E2M1->E5M2 by bit moves into mma.sync m16n8k32 e5m2 x e4m3, output rows summed over slots in order); "
+      "sm_100a; moe: one cooperative persistent kernel (router fp32 GEMV with epoch-tagged logits, "
+      "bitonic top-k softmax routing in every CTA, split-K over the intermediate: 16-row slices of MXFP4 "
+      "E2M1/E8M0-32 gate/up + SiLU + down per work item, cp.async ring, E2M1->E5M2 by bit moves into "
+      "mma.sync m16n8k32 e5m2 x e4m3 with per-block activation scales, one grid barrier, fixed-order combine); "
       "lm-head: online-FP8 E4M3 per-row-scale GEMV over the fragment-tiled head (coalesced 16-byte loads into registers, mma.sync m16n8k32 e4m3) fused top-k "
       "with temperature/top-p sampling; comparator: BF16 head GEMV";
   std::snprintf(buf, n, "%s", desc);

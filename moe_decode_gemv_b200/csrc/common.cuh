@@ -22,8 +22,9 @@ namespace moe {
 struct WsHeader {
   int32_t status;     // 0, or the first moe_status a kernel reported
   uint32_t ticket;    // last-block-done counter (returns to 0 after each use)
-  uint32_t barrier;   // grid barrier word (sense-reversing; see grid_barrier)
-  uint32_t pad[13];   // keeps what follows on a 64-byte boundary
+  uint32_t barrier;   // grid barrier word (sense-reversing; see grid_arrive)
+  uint32_t epoch;     // calls completed on this workspace (tags published values; see moe_layer.cu)
+  uint32_t pad[12];   // keeps what follows on a 64-byte boundary
 };
 static_assert(sizeof(WsHeader) == 64, "workspace header is 64 bytes");
 
@@ -115,6 +116,14 @@ __device__ __forceinline__ float e8m0_to_f32_fast(uint32_t code) { return __uint
 __device__ __forceinline__ void mma_e5m2_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                               uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k32.row.col.f32.e5m2.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// f16 x f16 -> fp32 tensor-core MMA, m16n8k16 (A row-major 16x16, B 16x8).
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
@@ -233,6 +242,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// An L2 cache policy that evicts last: for small inputs every CTA reads.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 

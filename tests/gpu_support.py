@@ -93,8 +93,14 @@ class Layer:
 
     KINDS = ("gate", "up", "down")
 
-    def __init__(self, B, seed: int, shape: I.MoEShape, layer: int = 0, skewed: bool = False):
+    def __init__(self, B, seed: int, shape: I.MoEShape, layer: int = 0, skewed: bool = False,
+                 wfn=None, sfn=None):
+        """wfn(kind, expert, w_bf16) -> w_bf16 changes an expert's weights before
+        quantisation; sfn(kind, scales_uint8) -> scales_uint8 patches the E8M0
+        codes after it.  Both sides (GPU and oracle) apply the same hooks."""
         self.B, self.seed, self.shape, self.layer = B, seed, shape, layer
+        self.wfn = wfn or (lambda kind, e, w: w)
+        self.sfn = sfn or (lambda kind, sc: sc)
         self.router_w = I.router_weight(seed, shape.experts, shape.hidden, layer)
         self.router_bias = I.router_bias(seed, shape.experts, layer) if skewed else None
         self.router_w_dev = self.router_w.cuda()
@@ -111,10 +117,17 @@ class Layer:
         experts = list(experts)
         staging = torch.empty((len(experts), rows, cols), dtype=torch.bfloat16, device="cuda")
         for i, e in enumerate(experts):
-            staging[i].copy_(I.expert_matrix(self.seed, s, e, kind, self.layer), non_blocking=False)
+            staging[i].copy_(self.wfn(kind, e, I.expert_matrix(self.seed, s, e, kind, self.layer)), non_blocking=False)
         bank = self.B.moe_quantize_mxfp4(staging)
         del staging
+        patched = self.sfn(kind, bank.scales.cpu().numpy())
+        bank.scales.copy_(torch.from_numpy(np.ascontiguousarray(patched)))
         return bank
+
+    def _oracle_quantize(self, kind, e):
+        w = self.wfn(kind, e, I.expert_matrix(self.seed, self.shape, e, kind, self.layer))
+        d, sc = oracle.load().mxfp4_quantize(u16(w))
+        return d, self.sfn(kind, sc)
 
     def oracle_banks(self, O, experts):
         """Stacked numpy banks holding the oracle's own quantisation of the
@@ -126,10 +139,9 @@ class Layer:
             d = np.zeros((s.experts, rows, cols // 2), np.uint8)
             sc = np.zeros((s.experts, rows, cols // 32), np.uint8)
             for e in sorted(set(int(v) for v in experts)):
-                d[e], sc[e] = O.mxfp4_quantize(u16(I.expert_matrix(self.seed, s, e, kind, self.layer)))
+                d[e], sc[e] = self._oracle_quantize(kind, e)
             out[kind] = (d, sc)
-        shared = {k: O.mxfp4_quantize(u16(I.expert_matrix(self.seed, s, "shared", k, self.layer)))
-                  for k in self.KINDS}
+        shared = {k: self._oracle_quantize(k, "shared") for k in self.KINDS}
         shared = {k: (v[0][None], v[1][None]) for k, v in shared.items()}
         return out, shared
 

@@ -54,8 +54,11 @@ def test_workspace_sizes(lib):
     assert lib.moe_workspace_bytes(4, 8, 512, 2560, 768) > 0
     assert lib.moe_workspace_bytes(5, 8, 512, 2560, 768) == 0          # M > 4
     assert lib.moe_workspace_bytes(1, 9, 512, 2560, 768) == 0          # top_k > 8
-    assert lib.moe_workspace_bytes(1, 8, 512, 2561, 768) == 0          # H not a multiple of 64
-    assert lib.moe_workspace_bytes(1, 8, 512, 2560, 96) == 0           # I not a multiple of 64
+    assert lib.moe_workspace_bytes(1, 8, 512, 2561, 768) == 0          # H not a multiple of 32
+    assert lib.moe_workspace_bytes(1, 8, 512, 2560, 80) == 0           # I not a multiple of 32
+    assert lib.moe_workspace_bytes(1, 8, 512, 4128, 768) == 0          # H above 4096
+    assert lib.moe_workspace_bytes(1, 8, 1025, 2560, 768) == 0         # more than 1024 experts
+    assert lib.moe_workspace_bytes(1, 8, 512, 96, 32) > 0              # the smallest odd sizes
     assert lib.lmhead_workspace_bytes(1, 29, 157184, 2560) > 0
     assert lib.lmhead_workspace_bytes(1, 65, 157184, 2560) == 0
     assert lib.lmhead_workspace_bytes(1, 8, 4, 256) == 0                # top_k > vocab
@@ -75,8 +78,8 @@ def _bank(lib, fmt=2, E=16, H=256, I=64):
     return lib._Bank(_mx(lib, fmt, E, I, H), _mx(lib, fmt, E, I, H), _mx(lib, fmt, E, H, I))
 
 
-def _packed(lib, fmt=4, E=16, H=256, I=64, gateup=A, down=A):
-    return lib._Packed(fmt, E, H, I, gateup, down)
+def _packed(lib, fmt=4, E=16, H=256, I=64, units=A, dscales=A):
+    return lib._Packed(fmt, E, H, I, units, dscales)
 
 
 def _decode(lib, experts, shared, M=1, top_k=2, x=A, ws=A, ws_bytes=1 << 24):
@@ -100,25 +103,26 @@ def test_moe_decode_rejects_bad_arguments(lib):
     assert _decode(lib, _packed(lib, H=250), _packed(lib, E=1, H=250)) == S.UNSUPPORTED_SHAPE
     assert _decode(lib, ok_bank, _packed(lib, E=2)) == S.UNSUPPORTED_SHAPE          # shared count != 1
     assert _decode(lib, ok_bank, _packed(lib, E=1, I=128)) == S.UNSUPPORTED_SHAPE   # shared width differs
-    assert _decode(lib, _packed(lib, gateup=U), ok_shared) == S.MISALIGNED
-    assert _decode(lib, _packed(lib, down=0), ok_shared) == S.INVALID_ARG
+    assert _decode(lib, _packed(lib, units=U), ok_shared) == S.MISALIGNED
+    assert _decode(lib, _packed(lib, dscales=0), ok_shared) == S.INVALID_ARG
 
 
 def test_pack_rejects_bad_arguments_and_sizes(lib):
     S, L = lib.Status, lib.library
-    # sizes: one gate/up chunk is 16 (H/2 + H/32) bytes per 8 rows, one down tile 32 (I/2 + I/32) per 32 rows
-    assert L.moe_packed_gateup_bytes(512, 2560, 768) == 512 * 96 * 16 * (1280 + 80)
-    assert L.moe_packed_down_bytes(512, 2560, 768) == 512 * 80 * 32 * (384 + 24)
-    assert L.moe_packed_gateup_bytes(512, 2560, 768) + L.moe_packed_down_bytes(512, 2560, 768) == 512 * 3133440
-    assert L.moe_packed_gateup_bytes(1, 250, 64) == 0 and L.moe_packed_down_bytes(1, 256, 96) == 0
+    # sizes: one 16-row item is 32 gate/up rows of H/2 + H/32 bytes and 16 down
+    # columns of H rows (8 bytes each); the down scales are H bytes per 32 columns
+    assert L.moe_packed_units_bytes(512, 2560, 768) == 512 * 48 * (32 * (1280 + 80) + 2560 * 8)
+    assert L.moe_packed_dscales_bytes(512, 2560, 768) == 512 * 24 * 2560
+    assert L.moe_packed_units_bytes(512, 2560, 768) + L.moe_packed_dscales_bytes(512, 2560, 768) == 512 * 3133440
+    assert L.moe_packed_units_bytes(1, 250, 64) == 0 and L.moe_packed_dscales_bytes(1, 256, 80) == 0
 
     def pack(src, dst):
         return L.moe_pack_experts(ctypes.byref(src), ctypes.byref(dst), None)
 
     assert pack(_bank(lib, fmt=1), _packed(lib, fmt=0)) == S.FORMAT_MISMATCH
     assert pack(_bank(lib), _packed(lib, fmt=0, E=8)) == S.UNSUPPORTED_SHAPE        # dst count differs
-    assert pack(_bank(lib), _packed(lib, fmt=0, gateup=U)) == S.MISALIGNED
-    assert pack(_bank(lib), _packed(lib, fmt=0, down=0)) == S.INVALID_ARG
+    assert pack(_bank(lib), _packed(lib, fmt=0, units=U)) == S.MISALIGNED
+    assert pack(_bank(lib), _packed(lib, fmt=0, dscales=0)) == S.INVALID_ARG
     bad_down = lib._Bank(_mx(lib, 2, 16, 64, 256), _mx(lib, 2, 16, 64, 256), _mx(lib, 2, 16, 64, 256))
     assert pack(bad_down, _packed(lib, fmt=0)) == S.UNSUPPORTED_SHAPE               # down not [H][I]
 

@@ -136,3 +136,24 @@ def test_repeat_calls_identical(B, tiny):
     assert B.moe_workspace_status(ws) == B.Status.OK
     for o in outs[1:]:
         assert np.array_equal(o[0], outs[0][0]) and np.array_equal(o[1], outs[0][1])
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_ling_head_outlier_tokens(B, O, ling, M):
+    """A token with one element at 1e3 among 1e-3 values (and, at M = 4, a
+    plain token, a negative outlier and a scaled token beside it)."""
+    w, head, q, s = ling
+    base = I.hidden_states(0, 4, I.LING_HEAD.hidden, tag="outlier").float()
+    x = torch.empty((4, I.LING_HEAD.hidden))
+    x[0] = base[0] * 1e-3
+    x[0, 1234] = 1e3
+    x[1] = base[1]
+    x[2] = base[2] * 1e-3
+    x[2, 77] = -1e3
+    x[3] = base[3] * 8
+    x = x[:M].to(torch.bfloat16)
+    ids, vals, logits = run_head_gpu(B, head, x.cuda(), 29)
+    ref = O.lmhead_fp8(u16(x), q, s)
+    near = check_head(ids, vals, logits, ref)
+    err = max(float(np.abs(logits[m] - ref[m]).max()) for m in range(M))
+    print(f"head outlier tokens M={M}: max-abs {err:.2e}, near ties {near}")

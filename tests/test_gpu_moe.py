@@ -104,12 +104,13 @@ def test_every_expert_selected_and_top1(B, O):
     check_moe(layer, O, x, y, ids, w)
 
 
-def test_odd_sizes(B, O):
-    """H and I multiples of 64 that are not powers of two, E not a multiple of
-    the CTA count, top_k = 3."""
-    s = I.MoEShape(hidden=192, inter=192, experts=24, top_k=3)
+@pytest.mark.parametrize("H,Inter,E,k,M", [(192, 192, 24, 3, 3), (96, 32, 5, 2, 4), (32, 96, 9, 8, 2)])
+def test_odd_sizes(B, O, H, Inter, E, k, M):
+    """H and I multiples of 32 that are not powers of two (down to one K block
+    and one pair of 16-row slices), E not a multiple of the CTA count."""
+    s = I.MoEShape(hidden=H, inter=Inter, experts=E, top_k=k)
     layer = Layer(B, 6, s)
-    x = I.hidden_states(6, 3, 192)
+    x = I.hidden_states(6, M, H)
     y, ids, w = layer.run_gpu(x.cuda())
     check_moe(layer, O, x, y, ids, w)
 
@@ -154,3 +155,87 @@ def test_ling_layer_skewed_m4(B, O, ling_skewed):
     y, ids, w = ling_skewed.run_gpu(x.cuda())
     check_moe(ling_skewed, O, x, y, ids, w)
     assert len(set(ids.reshape(-1).tolist())) < 32
+
+
+# ---------------------------------------------------------------------------
+# Inputs that stress the GPU path's own number handling: activations are
+# carried as E4M3 parts per 32-element block (x) and as f16 parts per
+# 16-value slice (h), and E8M0 scales are decoded by exponent placement.
+# The bar is the same as everywhere: rel-L2 <= 2e-3, max-abs <= 1e-2 against
+# the fp64 oracle on the same quantised bytes, ids exact outside the margin.
+# ---------------------------------------------------------------------------
+
+def outlier_tokens(M, H, seed=0):
+    """Token 0: one element at 1e3, the rest 1e-3 N(0, 1); token 1: N(0, 1);
+    token 2: one element at -1e3 among 1e-3 N(0, 1); token 3: 8 N(0, 1)."""
+    base = I.hidden_states(seed, 4, H, tag="outlier").float()
+    x = torch.empty((4, H))
+    x[0] = base[0] * 1e-3
+    x[0, 1234 % H] = 1e3
+    x[1] = base[1]
+    x[2] = base[2] * 1e-3
+    x[2, 77 % H] = -1e3
+    x[3] = base[3] * 8
+    return x[:M].to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_ling_layer_outlier_tokens(B, O, ling, M):
+    """A token with one 1e3 element among 1e-3 values: the block holding the
+    outlier spans 2^20, the other blocks are tiny."""
+    x = outlier_tokens(M, I.LING_MOE.hidden)
+    y, ids, w = ling.run_gpu(x.cuda())
+    rep = check_moe(ling, O, x, y, ids, w)
+    print(f"outlier tokens M={M}: rel-L2 {rep['rel_l2']:.2e}, max-abs {rep['max_abs']:.2e}, "
+          f"|y|max {np.abs(y).max():.1f}")
+    assert rep["skipped_tokens"] == 0, rep
+
+
+LING_WIDTH = I.MoEShape(hidden=2560, inter=768, experts=64, top_k=8)
+
+
+def test_ling_width_h_spans_2_20_per_slice(B, O):
+    """Gate and up rows 16j of every expert scaled by 2^4, the other rows by
+    2^-6: within each 16-row slice h spans about 2^20."""
+    def wfn(kind, e, w):
+        if kind == "down":
+            return w
+        f = torch.full((w.shape[0], 1), 2.0 ** -6)
+        f[::16] = 2.0 ** 4
+        return (w.float() * f).to(torch.bfloat16)
+
+    layer = Layer(B, 12, LING_WIDTH, wfn=wfn)
+    for M in (1, 3):
+        x = I.hidden_states(12, M, LING_WIDTH.hidden, tag="hrange")
+        y, ids, w = layer.run_gpu(x.cuda())
+        rep = check_moe(layer, O, x, y, ids, w)
+        print(f"h range M={M}: rel-L2 {rep['rel_l2']:.2e}, max-abs {rep['max_abs']:.2e}")
+        assert rep["skipped_tokens"] == 0, rep
+
+
+def test_ling_width_e8m0_extremes(B, O):
+    """Every gate and up row's block 0 carries E8M0 code 254 (2^127) and block
+    1 code 1 (2^-126); the activations' block 0 is bf16-subnormal (about
+    2^-128) and block 1 about 2^118, so the products stay finite.  The router
+    ignores block 1 (its columns are zero)."""
+    def sfn(kind, sc):
+        if kind != "down":
+            sc = sc.copy()
+            sc[..., 0] = 254
+            sc[..., 1] = 1
+        return sc
+
+    layer = Layer(B, 13, LING_WIDTH, sfn=sfn)
+    layer.router_w[:, 32:64] = 0.0
+    layer.router_w_dev = layer.router_w.cuda()
+    M = 2
+    x = I.hidden_states(13, M, LING_WIDTH.hidden, tag="e8m0").float()
+    x[:, :32] *= 2.0 ** -128
+    x[:, 32:64] *= 2.0 ** 118
+    x = x.to(torch.bfloat16)
+    assert (x[:, :32].float().abs() < 2.0 ** -126).any()  # subnormal bf16 values are present
+    y, ids, w = layer.run_gpu(x.cuda())
+    assert np.isfinite(y).all()
+    rep = check_moe(layer, O, x, y, ids, w)
+    print(f"E8M0 extremes: rel-L2 {rep['rel_l2']:.2e}, max-abs {rep['max_abs']:.2e}, |y|max {np.abs(y).max():.1f}")
+    assert rep["skipped_tokens"] == 0, rep

@@ -1,4 +1,4 @@
-"""The packed expert-bank layout, byte for byte, against a numpy statement of
+"""The sliced expert-bank layout, byte for byte, against a numpy statement of
 the layout that moe_gemv.h documents for moe_packed_bank (packing moves
 bytes and bits only, so the comparison is exact)."""
 import numpy as np
@@ -18,11 +18,6 @@ def B():
     return binding
 
 
-def swizzle_mask(units):
-    low = units & -units
-    return min(8, low) - 1
-
-
 def relayout(b):
     """The documented bit placement of one packed data byte: element 2j (low
     nibble) sign|e1 e0 m -> bits 7|3 2 1, element 2j+1 (high nibble) -> 0|6 5 4."""
@@ -33,33 +28,35 @@ def relayout(b):
 
 
 def expected_packed(gate, up, down):
-    """numpy: (data, scales) pairs of the canonical banks -> (gateup, down) bytes."""
+    """numpy: (data, scales) pairs of the canonical banks -> (units, dscales)
+    bytes of the sliced layout moe_gemv.h documents for moe_packed_bank."""
     (gd, gs), (ud, us), (dd, ds) = gate, up, down
     E, I, Hh = gd.shape
     H = 2 * Hh
-    nbH, nbI = H // 32, I // 32
-    mH, mI = swizzle_mask(nbH), swizzle_mask(nbI)
-    gu = []
+    nb = H // 32
+    units, dsc = [], []
     for e in range(E):
-        for q in range(I // 8):
-            rows = np.concatenate([gd[e, 8 * q:8 * q + 8], ud[e, 8 * q:8 * q + 8]])  # [16][H/2]
-            units = rows.reshape(16, nbH, 16)
-            # unit c of row r is stored at position c ^ (r & mask): position p holds unit p ^ (r & mask)
-            perm = np.stack([units[r, np.arange(nbH) ^ (r & mH)] for r in range(16)])
-            gu.append(relayout(perm.reshape(-1)))
-            gu.append(gs[e, 8 * q:8 * q + 8].reshape(-1))
-            gu.append(us[e, 8 * q:8 * q + 8].reshape(-1))
-    dn = []
-    for e in range(E):
-        for t in range(H // 32):
-            units = dd[e, 32 * t:32 * t + 32].reshape(32, nbI, 16)
-            perm = np.stack([units[r, np.arange(nbI) ^ (r & mI)] for r in range(32)])
-            dn.append(relayout(perm.reshape(-1)))
-            dn.append(ds[e, 32 * t:32 * t + 32].reshape(-1))
-    return np.concatenate(gu), np.concatenate(dn)
+        for j in range(I // 16):
+            # A: [block][g][t][gate g, up g, gate 8+g, up 8+g][4 bytes]
+            g2 = gd[e, 16 * j:16 * j + 16].reshape(2, 8, nb, 4, 4).transpose(0, 2, 1, 3, 4)  # [half][b][g][t][4]
+            u2 = ud[e, 16 * j:16 * j + 16].reshape(2, 8, nb, 4, 4).transpose(0, 2, 1, 3, 4)
+            a = np.stack([g2[0], u2[0], g2[1], u2[1]], axis=3)  # [b][g][t][w][4]
+            units.append(relayout(a.reshape(-1)))
+            # B: [block][g][gate g, up g, gate 8+g, up 8+g]
+            gs2 = gs[e, 16 * j:16 * j + 16].reshape(2, 8, nb).transpose(0, 2, 1)  # [half][b][g]
+            us2 = us[e, 16 * j:16 * j + 16].reshape(2, 8, nb).transpose(0, 2, 1)
+            units.append(np.stack([gs2[0], us2[0], gs2[1], us2[1]], axis=2).reshape(-1))
+            # C: [group][g][t][r][2 bytes] = columns 16j + 4t .. +3 of down row 32G + 8r + g
+            cols = dd[e][:, 8 * j:8 * j + 8].reshape(H // 32, 4, 8, 4, 2)  # [G][r][g][t][2]
+            c = cols.transpose(0, 2, 3, 1, 4)  # [G][g][t][r][2]
+            units.append(relayout(c.reshape(-1)))
+        for p in range(I // 32):
+            # byte 32G + 4g + t = scale of down row 32G + 8t + g
+            dsc.append(ds[e][:, p].reshape(H // 32, 4, 8).transpose(0, 2, 1).reshape(-1))
+    return np.concatenate(units), np.concatenate(dsc)
 
 
-@pytest.mark.parametrize("E,H,Inter", [(3, 256, 64), (2, 192, 192), (2, 2560, 768)])
+@pytest.mark.parametrize("E,H,Inter", [(3, 256, 64), (2, 192, 192), (2, 96, 32), (2, 2560, 768)])
 def test_pack_matches_documented_layout(B, E, H, Inter):
     g = torch.Generator().manual_seed(E * 1000 + H + Inter)
     banks = []
@@ -70,9 +67,9 @@ def test_pack_matches_documented_layout(B, E, H, Inter):
     torch.cuda.synchronize()
     assert packed.fmt == B.Format.MXFP4_MOE_PACKED
     canon = [(b.data.cpu().numpy(), b.scales.cpu().numpy()) for b in banks]
-    want_gu, want_dn = expected_packed(*canon)
-    assert np.array_equal(packed.gateup.cpu().numpy(), want_gu)
-    assert np.array_equal(packed.down.cpu().numpy(), want_dn)
+    want_u, want_d = expected_packed(*canon)
+    assert np.array_equal(packed.units.cpu().numpy(), want_u)
+    assert np.array_equal(packed.dscales.cpu().numpy(), want_d)
     assert packed.nbytes() == sum(b.nbytes() for b in banks)  # same bytes, regrouped
 
 
@@ -81,9 +78,9 @@ def test_pack_of_ling_shared_expert(B):
     banks = tuple(B.moe_quantize_mxfp4(I.expert_matrix(0, s, "shared", k).cuda()) for k in ("gate", "up", "down"))
     packed = B.moe_pack_experts(banks)
     canon = [(b.data.cpu().numpy(), b.scales.cpu().numpy()) for b in banks]
-    want_gu, want_dn = expected_packed(*canon)
-    assert np.array_equal(packed.gateup.cpu().numpy(), want_gu)
-    assert np.array_equal(packed.down.cpu().numpy(), want_dn)
+    want_u, want_d = expected_packed(*canon)
+    assert np.array_equal(packed.units.cpu().numpy(), want_u)
+    assert np.array_equal(packed.dscales.cpu().numpy(), want_d)
 
 
 def expected_tiled_head(q):
