@@ -1,4 +1,5 @@
-// lmhead.h -- internal interface of the LM-head kernels (lmhead_kernels.cu).
+// lmhead.h -- internal interface of the LM-head kernels: the FP8 head
+// (lmhead_fp8.cu) and the BF16 comparator head (lmhead_kernels.cu).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -10,10 +11,11 @@
 namespace moe {
 
 int lmhead_max_slices();
-// Ring depth (0 for the tiled FP8 kernel) and shared memory of one launch;
-// false if the shape does not fit in one CTA's shared memory (the CTA keeps
-// its rows' logits there).
+// Ring depth and shared memory of one launch (elem_bytes 1: the FP8 head, 2:
+// the BF16 head); false if the shape does not fit in one CTA's shared memory
+// (the CTA keeps its rows' logits there).
 bool lmhead_plan(int H, int elem_bytes, int M, int top_k, int64_t V, int grid, int* stages, size_t* smem);
+bool lmhead_fp8_plan(int H, int M, int top_k, int64_t V, int grid, int* stages, size_t* smem);
 size_t lmhead_cand_bytes(int grid, int M, int top_k);
 // Bytes of the fragment-tiled FP8 head (whole 16-row tiles, zero rows past V).
 size_t lmhead_tiled_bytes(int64_t V, int H);

@@ -1,11 +1,12 @@
-// lmhead_kernels.cu -- the online-FP8 LM head (and its BF16 comparator):
-// one pass over the [V][H] head for all M tokens, fused with the per-row
-// scale, an optional logits write and a top-k reduction.
+// lmhead_kernels.cu -- the BF16 comparator head: the same GEMV + per-row
+// scale-free top-k as the FP8 head (lmhead_fp8.cu) over the unquantised BF16
+// [V][H] head, which the FP8 head halves in bytes.  One pass over the head
+// for all M tokens, fused with an optional logits write and a top-k.
 //
-// The pages: every generated token reads the whole 157,184 x 2,560 head, and
-// quantising only this layer to FP8 at load time halves those reads
-// (ncijnetwork.com summary, "What are the 3 optimizations?", item 2;
-// generativeaipub.com blog, "2. Compressing the Output Head").
+// The pages: quantising only the vocabulary projection to FP8 at load time
+// halves the bytes each token reads (ncijnetwork.com summary, "What are the 3
+// optimizations?", item 2; generativeaipub.com blog, "2. Compressing the
+// Output Head"); this kernel is the BF16 side of that comparison.
 //
 // Design (sm_100a, one GPU):
 //  * One CTA per SM, persistent over a contiguous range of 16-row tiles.
@@ -13,27 +14,13 @@
 //    (cp.async.bulk, no multicast) into a ring of stages guarded by
 //    mbarriers; rows are copied one by one into a padded stride so that the
 //    consumers' 16-byte shared loads are free of bank conflicts.
-//  * Eight consumer warps split K.  Each computes 16 rows x 8 token columns
-//    with mma.sync m16n8k32 (E4M3 x E4M3 -> fp32): the weight bytes from
-//    shared memory ARE the A fragments -- no conversion instruction per
-//    weight -- and the B fragments hold the token activations, resident in
-//    registers for the whole kernel.  This is a GEMV: the tensor-core
-//    instruction is used because it retires 4,096 multiply-adds per issue and
-//    needs no per-weight decode, which keeps the instruction count per weight
-//    byte far below what the HBM stream allows, at M = 1 and M = 4 alike.
-//  * Activations: each bf16 token is scaled by 2^sigma_m (max |x| into
-//    [2^7, 2^8)) and split into two E4M3 parts hi + lo, which represent the
-//    bf16 value exactly (8 significand bits = 4 + 4) when its scaled
-//    magnitude is at least 2^-2 (2^-10 of the token's largest or more); below
-//    that lo is rounded to E4M3's subnormal step, an error under 2^-17 of the
-//    largest.  The logit is acc * s_v * 2^-sigma_m.
-//  * Epilogue: two warps take alternate tiles.  A tile's 16 row scales ride
-//    in its ring stage (one more bulk copy) and reach the epilogue with the
-//    consumers' partial sums, so no global load sits on the epilogue's path.
-//    The epilogue sums the partials, applies the row scale and 2^-sigma_m,
-//    writes logits when asked, and offers the 16 values to a per-token sorted
-//    top-k list held in its registers (ties to the lower id).  The last CTA to
-//    finish merges all CTAs' lists.
+//  * Eight consumer warps split K, each computing 16 rows x 8 token columns
+//    with mma.sync m16n8k16 (bf16 x bf16 -> fp32); the B fragments hold the
+//    tokens and stay in registers for the whole kernel.
+//  * An epilogue warp sums the consumers' partials, writes logits when asked
+//    and keeps each value in shared memory; after the stream one warp per
+//    token takes the CTA's top-k, and the last CTA to finish merges all
+//    CTAs' lists (ties to the lower id).
 #include <cuda_runtime.h>
 
 #include <cfloat>
@@ -643,268 +630,6 @@ lmhead_topk_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
 }
 
 
-// ---------------------------------------------------------------------------
-// The FP8 head over the fragment-tiled layout (lmhead_tile_fp8).
-//
-// Tile T (rows 16T .. 16T+15, zero rows past V) is 16 * H bytes: for each
-// 64-byte K slice s, 1,024 bytes = [half h][lane l][16 bytes], the 16 bytes
-// of row 16T + (l >> 2) + 8h at K bytes 64s + 16 (l & 3) ...  So the A
-// fragments of one mma.sync m16n8k32 pair are one 512-byte contiguous read
-// per warp and half: the weights stream with plain, fully coalesced 16-byte
-// loads straight into registers (no shared-memory staging), which reaches a
-// higher rate on this part than a ring of bulk copies.
-// ---------------------------------------------------------------------------
-constexpr int kTiledConsumers = 10;  // 40 slices of the 2,560-wide head: 4 per warp
-constexpr int kTilesInFlight = 3;    // tiles whose loads a consumer warp keeps outstanding
-constexpr int kTiledThreads = (kTiledConsumers + kEpilogueWarps) * 32;
-constexpr int kTiledMaxSlices = 80 / kTiledConsumers;  // slices per warp: H <= 80 * 64 = 5120
-
-__global__ void tile_fp8_head_kernel(const uint8_t* __restrict__ q, int64_t V, int H, uint8_t* __restrict__ out) {
-  const int64_t ntiles = (V + kTileRows - 1) / kTileRows;
-  const int64_t units = ntiles * H;  // 16-byte units: 16 * H bytes per tile
-  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < units; u += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = u / H;
-    const int j = (int)(u - t * H);
-    const int s = j >> 6, h = (j >> 5) & 1, l = j & 31;
-    const int64_t row = t * kTileRows + (l >> 2) + 8 * h;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (row < V) v = *reinterpret_cast<const uint4*>(q + row * H + 64 * s + 16 * (l & 3));
-    *reinterpret_cast<uint4*>(out + u * 16) = v;
-  }
-}
-
-template <int kSlices>
-__global__ void __launch_bounds__(kTiledThreads, 1)
-lmhead_fp8_tiled_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
-                        const uint8_t* __restrict__ qt,       // tiled E4M3 head
-                        const float* __restrict__ row_scale,  // [V]
-                        int64_t V, int H, int M, int top_k,
-                        float* __restrict__ logits,           // [M][V] or nullptr
-                        int32_t* __restrict__ out_ids,        // [M][top_k]
-                        float* __restrict__ out_vals,         // [M][top_k]
-                        WsHeader* __restrict__ hdr,
-                        Cand* __restrict__ cand)              // [gridDim][M][top_k]
-{
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int64_t ntiles = (V + kTileRows - 1) / kTileRows;
-  const int n_cap = (int)((ntiles + gridDim.x - 1) / gridDim.x) * kTileRows;  // rows of the largest CTA range
-  const int nsl = H / 64;                                                      // 64-byte K slices
-
-  // shared memory: [top-k scratch][reduce buffers][row scales][logits of this CTA's rows][barriers][scalars]
-  Cand* warp_scratch = reinterpret_cast<Cand*>(smem);                          // [4][kCandCap]
-  float* red = reinterpret_cast<float*>(warp_scratch + 4 * kCandCap);          // [kRed][20][16][4]
-  float* rsc = red + kRed * kTiledConsumers * kTileRows * 4;                   // [kRed][16] row scales
-  float* cvals = rsc + kRed * kTileRows;                                       // [M][n_cap]
-  uint64_t* red_full = reinterpret_cast<uint64_t*>(cvals + (size_t)M * ((n_cap + 1) & ~1));
-  uint64_t* red_empty = red_full + kRed;
-  int* s_sigma = reinterpret_cast<int*>(red_empty + kRed);  // [4]
-  int* s_poison = s_sigma + 4;  // set once any bounded wait ran out
-  int* s_last = s_sigma + 5;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t_begin = ntiles * blockIdx.x / gridDim.x;
-  const int64_t t_end = ntiles * (blockIdx.x + 1) / gridDim.x;
-  const int g = lane >> 2, tq = lane & 3;
-
-  // A fragments straight from HBM: the next tile's loads are issued before
-  // this tile's MMAs (three tiles in flight per warp, ~120 KB per SM).  Warp 0
-  // also loads the tile's row scales.
-  struct TileRegs {
-    uint4 a[kSlices], b[kSlices];  // rows g and g + 8
-    float sc;
-  };
-  auto load_tile = [&](int64_t t, TileRegs& R) {
-    const uint8_t* tb = qt + (size_t)t * kTileRows * H + lane * 16;
-#pragma unroll
-    for (int si = 0; si < kSlices; ++si) {
-      const int slice = warp + si * kTiledConsumers;
-      const bool in = slice < nsl;
-      R.a[si] = in ? ld_stream_u4(tb + (size_t)slice * 1024) : make_uint4(0u, 0u, 0u, 0u);
-      R.b[si] = in ? ld_stream_u4(tb + (size_t)slice * 1024 + 512) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    const int64_t row = t * kTileRows + lane;
-    R.sc = (warp == 0 && lane < kTileRows && row < V) ? __ldg(row_scale + row) : 1.0f;
-  };
-  // Tiles whose loads go out before anything else (they do not depend on the
-  // activations): the consumers' first tiles are in flight during the prologue.
-  constexpr int kPre = (kTilesInFlight == 3 && kSlices <= 4) ? 2 : (kSlices <= 2 * (20 / kTiledConsumers) ? 1 : 0);
-  TileRegs R0, R1, R2;
-  if (warp < kTiledConsumers) {
-    if (kPre >= 1 && t_begin < t_end) load_tile(t_begin, R0);
-    if (kPre >= 2 && t_begin + 1 < t_end) load_tile(t_begin + 1, R1);
-  }
-
-  if (threadIdx.x == 0) {
-    for (int r = 0; r < kRed; ++r) {
-      mbar_init(&red_full[r], kTiledConsumers);
-      mbar_init(&red_empty[r], 1);
-    }
-    fence_mbar_init();
-    *s_poison = 0;
-  }
-  if (warp < M) {  // per-token power of two: max |x * 2^sigma| in [2^7, 2^8), inside E4M3's normal range
-    float amax = 0.f;
-#pragma unroll 8
-    for (int j = lane; j < H; j += 32) amax = fmaxf(amax, fabsf(bf16_bits_to_f32(x[(size_t)warp * H + j])));
-    amax = warp_max(amax);
-    if (lane == 0) {
-      int sigma = 0;
-      if (amax > 0.f) {
-        const int e = (int)((__float_as_uint(amax) >> 23) & 0xff);
-        const int fl = e ? e - 127 : (31 - __clz(__float_as_uint(amax) & 0x7fffff)) - 149;
-        sigma = 7 - fl;
-        sigma = sigma > 126 ? 126 : (sigma < -126 ? -126 : sigma);
-      }
-      s_sigma[warp] = sigma;
-    }
-  }
-  __syncthreads();
-
-  // bounded wait shared by all roles: lane 0 polls, the warp agrees on the result
-  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-    bool ok = !*(volatile int*)s_poison;
-    if (ok && lane == 0) ok = mbar_wait(bar, parity);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok && lane == 0 && !*(volatile int*)s_poison) {
-      report(hdr, MOE_ERR_TIMEOUT);
-      atomicExch(s_poison, 1);
-    }
-    return ok;
-  };
-
-  if (warp < kTiledConsumers) {
-    // ------------------------------ consumers -----------------------------
-    // B fragments, resident for the whole kernel: column n is part n & 1 of
-    // token n >> 1 -- the token, scaled by 2^sigma, split into two E4M3 parts
-    // x' = hi + lo, exact for every element of scaled magnitude 2^-2 or more
-    // (the rest within 2^-17 of the token's largest) -- so one MMA covers
-    // both parts of four tokens.
-    uint32_t bfrag[kSlices][2][2];  // [slice][mma][b0, b1]
-    {
-      const int m = g >> 1, part = g & 1;
-      const bool live = m < M;
-      const float scl = live ? __uint_as_float((uint32_t)(127 + s_sigma[m]) << 23) : 0.f;
-#pragma unroll
-      for (int si = 0; si < kSlices; ++si) {
-        const int slice = warp + si * kTiledConsumers;
-        const bool in = live && slice < nsl;
-        const int e0 = slice * 64 + tq * 16;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {  // four groups of 4 elements: mma (q / 2), register (q % 2)
-          uint32_t hw = 0u, lw = 0u;
-          if (in) {
-            const uint2 p = *reinterpret_cast<const uint2*>(x + (size_t)m * H + e0 + 4 * q);
-            const float v0 = bf16_bits_to_f32(p.x & 0xffffu) * scl, v1 = bf16_bits_to_f32(p.x >> 16) * scl;
-            const float v2 = bf16_bits_to_f32(p.y & 0xffffu) * scl, v3 = bf16_bits_to_f32(p.y >> 16) * scl;
-            const uint32_t h01 = f32x2_to_e4m3x2(v0, v1), h23 = f32x2_to_e4m3x2(v2, v3);
-            const uint32_t f01 = e4m3x2_to_f16x2(h01), f23 = e4m3x2_to_f16x2(h23);
-            const float2 r01 = __half22float2(*reinterpret_cast<const __half2*>(&f01));
-            const float2 r23 = __half22float2(*reinterpret_cast<const __half2*>(&f23));
-            hw = h01 | (h23 << 16);
-            lw = f32x2_to_e4m3x2(v0 - r01.x, v1 - r01.y) | (f32x2_to_e4m3x2(v2 - r23.x, v3 - r23.y) << 16);
-          }
-          bfrag[si][q / 2][q % 2] = part ? lw : hw;
-        }
-      }
-    }
-    auto compute = [&](const TileRegs& R, int64_t it) {
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-      for (int si = 0; si < kSlices; ++si) {
-        if (warp + si * kTiledConsumers < nsl) {
-          // rows g and g+8, 16 bytes each: words 0,1 feed MMA 0 and words 2,3 MMA 1
-          mma_e4m3(acc[0], R.a[si].x, R.b[si].x, R.a[si].y, R.b[si].y, bfrag[si][0][0], bfrag[si][0][1]);
-          mma_e4m3(acc[1], R.a[si].z, R.b[si].z, R.a[si].w, R.b[si].w, bfrag[si][1][0], bfrag[si][1][1]);
-        }
-      }
-      // columns 2tq, 2tq+1 hold the two parts of token tq
-      const float row_g = acc[0][0] + acc[0][1] + acc[1][0] + acc[1][1];
-      const float row_g8 = acc[0][2] + acc[0][3] + acc[1][2] + acc[1][3];
-      const int r = (int)(it % kRed);
-      if (it >= kRed) wait_all(&red_empty[r], (uint32_t)(((it / kRed) & 1) ^ 1));
-      float* rb = red + (size_t)r * kTiledConsumers * kTileRows * 4;
-      if (warp == 0 && lane < kTileRows) rsc[r * kTileRows + lane] = R.sc;
-      rb[(warp * kTileRows + g) * 4 + tq] = row_g;
-      rb[(warp * kTileRows + g + 8) * 4 + tq] = row_g8;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&red_full[r]);
-    };
-    int64_t it = 0;
-    if constexpr (kPre == 2) {  // R0, R1 hold the first two tiles
-      int64_t t = t_begin;
-      while (t < t_end) {
-        if (t + 2 < t_end) load_tile(t + 2, R2);
-        compute(R0, it++);
-        if (++t >= t_end) break;
-        if (t + 2 < t_end) load_tile(t + 2, R0);
-        compute(R1, it++);
-        if (++t >= t_end) break;
-        if (t + 2 < t_end) load_tile(t + 2, R1);
-        compute(R2, it++);
-        ++t;
-      }
-    } else if constexpr (kPre == 1) {  // R0 holds the first tile
-      int64_t t = t_begin;
-      while (t < t_end) {
-        if (t + 1 < t_end) load_tile(t + 1, R1);
-        compute(R0, it++);
-        if (++t >= t_end) break;
-        if (t + 1 < t_end) load_tile(t + 1, R0);
-        compute(R1, it++);
-        ++t;
-      }
-    } else {  // wide rows: one tile in flight per warp (registers)
-      for (int64_t t = t_begin; t < t_end; ++t) {
-        load_tile(t, R0);
-        compute(R0, it++);
-      }
-    }
-  } else {
-    // ------------------------------ epilogue ------------------------------
-    // Two epilogue warps take alternate tiles: sum the consumers' partials, apply the
-    // row scale and 2^-sigma_m, write logits when asked, and keep each value
-    // in shared memory for this CTA's top-k, taken after the stream.
-    const int ew = warp - kTiledConsumers;  // 0 or 1
-    float inv[4];  // 2^-sigma_m
-#pragma unroll
-    for (int m = 0; m < 4; ++m) inv[m] = __uint_as_float((uint32_t)(127 - (m < M ? s_sigma[m] : 0)) << 23);
-    int64_t it = ew;
-    for (int64_t t = t_begin + ew; t < t_end; t += kEpilogueWarps, it += kEpilogueWarps) {
-      const int r = (int)(it % kRed);
-      const int64_t row = t * kTileRows + lane;
-      const int nrows = (int)(V - t * kTileRows < kTileRows ? V - t * kTileRows : kTileRows);
-      const bool valid = lane < nrows;
-      const bool ok = wait_all(&red_full[r], (uint32_t)((it / kRed) & 1));
-      const float* rb = red + (size_t)r * kTiledConsumers * kTileRows * 4;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      float rs = 1.0f;
-      if (valid && ok) {
-#pragma unroll
-        for (int ww = 0; ww < kTiledConsumers; ++ww) {
-          const float4 p = *reinterpret_cast<const float4*>(rb + (ww * kTileRows + lane) * 4);
-          acc[0] += p.x; acc[1] += p.y; acc[2] += p.z; acc[3] += p.w;
-        }
-        rs = rsc[r * kTileRows + lane];
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&red_empty[r]);
-      if (valid) {
-        const int local = (int)((t - t_begin) * kTileRows) + lane;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          if (m < M) {
-            const float v = acc[m] * rs * inv[m];
-            if (logits) logits[(size_t)m * V + row] = v;
-            cvals[(size_t)m * n_cap + local] = v;
-          }
-        }
-      }
-    }
-  }
-  head_tail(cvals, n_cap, warp_scratch, t_begin, t_end, V, M, top_k, warp, lane, hdr, cand, smem, s_last, out_ids,
-            out_vals);
-}
-
 }  // namespace
 
 // ----------------------------------------------------------------------------
@@ -927,29 +652,10 @@ static size_t stream_smem_bytes(int H, int elem_bytes, int stages, int M, int64_
   return bytes;
 }
 
-static size_t tiled_smem_bytes(int M, int64_t V, int grid) {
-  const int64_t ntiles = (V + kTileRows - 1) / kTileRows;
-  const int64_t n_cap = (ntiles + grid - 1) / grid * kTileRows;
-  size_t bytes = 4 * kCandCap * sizeof(Cand);                           // per-token top-k scratch
-  bytes += kRed * kTiledConsumers * kTileRows * 4 * sizeof(float);      // reduce buffers
-  bytes += kRed * kTileRows * sizeof(float);                            // row scales
-  bytes += (size_t)M * ((n_cap + 1) & ~1) * sizeof(float);              // this CTA's logits
-  bytes += 2 * kRed * sizeof(uint64_t) + 8 * sizeof(int);
-  return bytes;
-}
-
-// elem_bytes 1: the tiled FP8 kernel (stages = 0: no ring); 2: the BF16 ring kernel.
+// elem_bytes 1: the FP8 head kernel (lmhead_fp8.cu); 2: the BF16 ring kernel.
 bool lmhead_plan(int H, int elem_bytes, int M, int top_k, int64_t V, int grid, int* stages, size_t* smem) {
+  if (elem_bytes == 1) return lmhead_fp8_plan(H, M, top_k, V, grid, stages, smem);
   const size_t merge = merge_smem_bytes(grid, top_k);  // the final merge reuses the whole dynamic buffer
-  if (elem_bytes == 1) {
-    size_t b = tiled_smem_bytes(M, V, grid);
-    if (merge > b) b = merge;
-    if (H % 64 != 0 || (H / 64 + kTiledConsumers - 1) / kTiledConsumers > kTiledMaxSlices || b > kMaxSmem)
-      return false;
-    *stages = 0;
-    *smem = b;
-    return true;
-  }
   for (int st = 4; st >= 2; --st) {
     size_t b = stream_smem_bytes(H, elem_bytes, st, M, V, grid);
     if (merge > b) b = merge;
@@ -961,15 +667,6 @@ bool lmhead_plan(int H, int elem_bytes, int M, int top_k, int64_t V, int grid, i
   }
   return false;
 }
-
-size_t lmhead_tiled_bytes(int64_t V, int H) { return (size_t)((V + kTileRows - 1) / kTileRows) * kTileRows * H; }
-
-cudaError_t launch_tile_fp8_head(const uint8_t* q, int64_t V, int H, uint8_t* out, cudaStream_t st) {
-  tile_fp8_head_kernel<<<4 * 148, 256, 0, st>>>(q, V, H, out);
-  return cudaGetLastError();
-}
-
-size_t lmhead_cand_bytes(int grid, int M, int top_k) { return (size_t)grid * M * top_k * sizeof(Cand); }
 
 template <typename W, int kSlices>
 static cudaError_t launch_head_t(const uint16_t* x, const W* w, const float* s, int64_t V, int H, int M, int top_k,
@@ -999,33 +696,6 @@ static cudaError_t launch_head(const uint16_t* x, const W* w, const float* s, in
 #undef MOE_CASE
     default: return cudaErrorInvalidValue;
   }
-}
-
-template <int kS>
-static cudaError_t launch_tiled_t(const uint16_t* x, const uint8_t* qt, const float* s, int64_t V, int H, int M,
-                                  int top_k, float* logits, int32_t* ids, float* vals, WsHeader* hdr, void* cand,
-                                  int grid, size_t smem, cudaStream_t st) {
-  cudaError_t e = ensure_smem_optin<lmhead_fp8_tiled_kernel<kS>>();
-  if (e != cudaSuccess) return e;
-  lmhead_fp8_tiled_kernel<kS><<<grid, kTiledThreads, smem, st>>>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr,
-                                                                  reinterpret_cast<Cand*>(cand));
-  return cudaGetLastError();
-}
-
-cudaError_t launch_lmhead_fp8(const uint16_t* x, const uint8_t* qt, const float* s, int64_t V, int H, int M,
-                              int top_k, float* logits, int32_t* ids, float* vals, WsHeader* hdr, void* cand,
-                              int grid, cudaStream_t st) {
-  int stages = 0;
-  size_t smem = 0;
-  if (!lmhead_plan(H, 1, M, top_k, V, grid, &stages, &smem)) return cudaErrorInvalidConfiguration;
-  const int need = (H / 64 + kTiledConsumers - 1) / kTiledConsumers;
-  if (need <= 1) return launch_tiled_t<1>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
-  if (need <= 2) return launch_tiled_t<2>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
-  if (need <= kTiledMaxSlices / 2)
-    return launch_tiled_t<kTiledMaxSlices / 2>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
-  if (need <= kTiledMaxSlices)
-    return launch_tiled_t<kTiledMaxSlices>(x, qt, s, V, H, M, top_k, logits, ids, vals, hdr, cand, grid, smem, st);
-  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_lmhead_bf16(const uint16_t* x, const uint16_t* w, int64_t V, int H, int M, int top_k,

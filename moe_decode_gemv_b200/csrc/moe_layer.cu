@@ -27,9 +27,9 @@
 //    | value), so that readers need no barrier: every CTA polls the words
 //    until all carry this call's tag, then takes the same top-k and builds
 //    the same slot table (slot 0 = shared expert, then each distinct routed
-//    expert once).  Top-k: the k-th best of 16 group maxima bounds the k-th
-//    best logit from below, and the few logits not worse than that bound are
-//    ranked by counting.
+//    expert once).  Top-k, one warp per token: the k-th best of the 32 lane
+//    maxima bounds the k-th best logit from below, and the few logits not
+//    worse than that bound are ranked by counting.
 //  * Each lane owns a fixed set of output rows and accumulates its CTA's
 //    weighted contributions in registers across items.  After the last item
 //    the CTAs write these partial outputs, meet at one grid barrier, and sum
@@ -85,18 +85,13 @@ struct Geo {
   }
 };
 
-constexpr int kCandCap = 512;  // routing candidates per token: at most top_k groups of E/16 logits
+constexpr int kCandCap = 256;  // routing candidates per token: at most top_k lanes' E/32 logits
 
 struct Ctl {
   uint64_t full[kMaxStages];                 // one phase per item copied into the stage
   uint64_t xbar;                             // the tokens' copy into shared memory
   float router_part[kWarps][4];
   int32_t sigma_x[4][kMaxBlocksPerWarp * kWarps];
-  float gmax_v[4][16];                       // routing: the 16 group maxima of each token
-  int32_t gmax_i[4][16];
-  float bound_v[4];                          // routing: the k-th best group maximum
-  int32_t bound_i[4];
-  int ncand[4];
   uint16_t cand[4][kCandCap];                // routing: candidate experts of each token
   int32_t ids[4][8];
   float topv[4][8];
@@ -476,105 +471,102 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   auto route = [&]() {
     float* lg = reinterpret_cast<float*>(scratch);  // [M][E]
     {
-      const uint64_t start = global_ns();
-      bool ok = !poisoned();
-      for (int i = threadIdx.x; i < M * E; i += kThreads) {
-        uint64_t v = 0;
-        for (;;) {
-          v = ld_relaxed_u64(&ws.logits[i]);
-          if ((uint32_t)(v >> 32) == tag || !ok) break;
-          if (global_ns() - start > kWaitLimitNs) {
-            ok = false;
-            break;
-          }
-          __nanosleep(32);
+      // this thread's words (at most 8: M * E <= 4096), all read at once;
+      // only stale ones are read again
+      constexpr int kPer = 4 * kMaxE / kThreads;
+      uint64_t v[kPer];
+      uint32_t stale = 0u;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int i = threadIdx.x + u * kThreads;
+        if (i < M * E) {
+          v[u] = ld_relaxed_u64(&ws.logits[i]);
+          if ((uint32_t)(v[u] >> 32) != tag) stale |= 1u << u;
         }
-        const float x = __uint_as_float((uint32_t)v);
-        lg[i] = x > -FLT_MAX ? x : -FLT_MAX;  // NaN and -inf rank as -FLT_MAX
       }
-      if (!ok) fail();
+      const uint64_t start = global_ns();
+      while (stale && !poisoned()) {
+        if (global_ns() - start > kWaitLimitNs) {
+          fail();
+          break;
+        }
+        __nanosleep(32);
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          if (stale >> u & 1u) {
+            v[u] = ld_relaxed_u64(&ws.logits[threadIdx.x + u * kThreads]);
+            if ((uint32_t)(v[u] >> 32) == tag) stale &= ~(1u << u);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int i = threadIdx.x + u * kThreads;
+        if (i < M * E) {
+          const float x = __uint_as_float((uint32_t)v[u]);
+          lg[i] = x > -FLT_MAX ? x : -FLT_MAX;  // NaN and -inf rank as -FLT_MAX
+        }
+      }
     }
-    // Token m's logits go to nthr threads; thread l holds experts l, l + nthr, ...
-    // The threads form 16 groups of gs consecutive lanes.
-    const int wpt = M == 1 ? 16 : (M == 2 ? 8 : 4);
-    const int nthr = 32 * wpt, gs = 2 * wpt;
-    const int m = warp / wpt, tl = threadIdx.x - m * nthr;
-    const bool tok = m < M;
-    if (threadIdx.x < 4) C.ncand[threadIdx.x] = 0;
     __syncthreads();
-    // 1. group maxima
-    if (tok) {
+    // One warp per token: lane l holds experts l, l + 32, ...  The k-th best
+    // of the 32 lane maxima bounds the k-th best logit from below (those are k
+    // real logits), so only logits not worse than it are candidates; they are
+    // ranked by counting (ids are distinct, so ranks are).
+    if (warp < M) {
+      const int m = warp;
+      const float* lm = lg + m * E;
       VI b = pad_entry(0);
-      for (int e = tl; e < E; e += nthr) {
-        const float v = lg[m * E + e];
-        if (better(v, e, b.v, b.i)) b = VI{v, e};
-      }
-      for (int o = gs >> 1; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(kFull, b.v, o);
-        const int32_t oi = __shfl_xor_sync(kFull, b.i, o);
-        if (better(ov, oi, b.v, b.i)) b = VI{ov, oi};
-      }
-      if (tl % gs == 0) {
-        C.gmax_v[m][tl / gs] = b.v;
-        C.gmax_i[m][tl / gs] = b.i;
-      }
-    }
-    __syncthreads();
-    // 2. the bound: the top_k-th best group maximum (if top_k groups hold an expert)
-    if (tok && tl < 32) {
-      const VI mine = tl < 16 ? VI{C.gmax_v[m][tl], C.gmax_i[m][tl]} : pad_entry(tl);
+#pragma unroll 8
+      for (int e = lane; e < E; e += 32)
+        if (better(lm[e], e, b.v, b.i)) b = VI{lm[e], e};
       int rank = 0;
-      for (int o = 0; o < 16; ++o) rank += better(C.gmax_v[m][o], C.gmax_i[m][o], mine.v, mine.i);
-      const uint32_t hit = __ballot_sync(kFull, tl < 16 && rank == a.top_k - 1 && mine.i < E);
-      if (tl == 0) {
-        const int src = hit ? __ffs(hit) - 1 : -1;
-        C.bound_v[m] = src >= 0 ? C.gmax_v[m][src] : -FLT_MAX;
-        C.bound_i[m] = src >= 0 ? C.gmax_i[m][src] : 0x7fffffff;
+#pragma unroll
+      for (int o = 0; o < 32; ++o) {
+        const float ov = __shfl_sync(kFull, b.v, o);
+        const int32_t oi = __shfl_sync(kFull, b.i, o);
+        rank += better(ov, oi, b.v, b.i);
       }
-    }
-    __syncthreads();
-    // 3. candidates: experts not worse than the bound
-    if (tok) {
-      const float bv = C.bound_v[m];
-      const int32_t bi = C.bound_i[m];
-      for (int e0 = 0; e0 < E; e0 += nthr) {
-        const int e = e0 + tl;
-        const bool keep = e < E && !better(bv, bi, lg[m * E + e], e);
+      const uint32_t hit = __ballot_sync(kFull, rank == a.top_k - 1 && b.i < E);
+      VI bound = pad_entry(0);  // none: fewer than k lanes hold an expert, every expert is a candidate
+      if (hit) {
+        bound.v = __shfl_sync(kFull, b.v, __ffs(hit) - 1);
+        bound.i = __shfl_sync(kFull, b.i, __ffs(hit) - 1);
+      }
+      int nc = 0;
+#pragma unroll 4
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const bool keep = e < E && !better(bound.v, bound.i, lm[e], e);
         const uint32_t bal = __ballot_sync(kFull, keep);
-        int base = 0;
-        if (lane == 0 && bal) base = atomicAdd(&C.ncand[m], __popc(bal));
-        base = __shfl_sync(kFull, base, 0);
-        const int pos = base + __popc(bal & ((1u << lane) - 1u));
-        if (keep && pos < kCandCap) C.cand[m][pos] = (uint16_t)e;  // never more: see kCandCap
+        const int pos = nc + __popc(bal & ((1u << lane) - 1u));
+        if (keep && pos < kCandCap) C.cand[m][pos] = (uint16_t)e;  // never more: k lanes' experts at most
+        nc += __popc(bal);
       }
-    }
-    __syncthreads();
-    // 4. rank the candidates by counting (ranks are distinct: ids are)
-    if (tok) {
-      const int nc = min(C.ncand[m], kCandCap);
-      for (int q = tl; q < nc; q += nthr) {
+      __syncwarp();
+      nc = min(nc, kCandCap);
+      for (int q = lane; q < nc; q += 32) {
         const int e = C.cand[m][q];
-        const float v = lg[m * E + e];
-        int rank = 0;
+        const float v = lm[e];
+        int r = 0;
+#pragma unroll 8
         for (int o = 0; o < nc; ++o) {
           const int f = C.cand[m][o];
-          rank += better(lg[m * E + f], f, v, e);
+          r += better(lm[f], f, v, e);
         }
-        if (rank < a.top_k) {
-          C.ids[m][rank] = e;
-          C.topv[m][rank] = v;
+        if (r < a.top_k) {
+          C.ids[m][r] = e;
+          C.topv[m][r] = v;
         }
       }
-    }
-    __syncthreads();
-    if (warp < M) {  // softmax over the selected k, renormalised
-      const int mm = warp;
-      const float v0 = C.topv[mm][0];
-      const float ex = lane < a.top_k ? expf(C.topv[mm][lane] - v0) : 0.f;
+      __syncwarp();
+      // softmax over the selected k, renormalised
+      const float v0 = C.topv[m][0];
+      const float ex = lane < a.top_k ? expf(C.topv[m][lane] - v0) : 0.f;
       float z = ex;
 #pragma unroll
       for (int o = 4; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
-      if (lane < a.top_k) C.wts[mm][lane] = ex / z;
+      if (lane < a.top_k) C.wts[m][lane] = ex / z;
     }
     __syncthreads();
     if (warp == 0) {
