@@ -24,7 +24,8 @@ struct WsHeader {
   uint32_t ticket;    // last-block-done counter (returns to 0 after each use)
   uint32_t barrier;   // grid barrier word (sense-reversing; see grid_arrive)
   uint32_t epoch;     // calls completed on this workspace (tags published values; see moe_layer.cu)
-  uint32_t pad[12];   // keeps what follows on a 64-byte boundary
+  uint32_t tiles;     // next tile handed out by a counter (returns to 0 after each use)
+  uint32_t pad[11];   // keeps what follows on a 64-byte boundary
 };
 static_assert(sizeof(WsHeader) == 64, "workspace header is 64 bytes");
 
@@ -235,8 +236,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Bounded wait on an mbarrier phase.  Returns false if the wait ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;  // the common case reads no timer
   return bounded_spin([&] { return mbar_try_wait(bar, parity); }, 0);
 }
+
+// Orders this thread's view of global memory (made visible to it by an
+// acquire) before its later bulk copies, which read through the async proxy.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async;" ::: "memory"); }
 
 // An L2 cache policy that evicts first: for weights read once per step.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
