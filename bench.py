@@ -103,23 +103,52 @@ REASON_BITS = {
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during a window."""
+    """SM clock, power and clock-event reasons sampled during a window, by
+    read-only NVML queries in a thread (nvidia-smi when NVML is missing).
+    Nothing here changes a setting of the GPU."""
 
-    def __init__(self, gpu_index: int, period_ms: int = 50):
-        self.samples = []
-        self.proc = None
+    def __init__(self, gpu_index: int, period_s: float = 0.02):
+        self.samples = []  # (time, sm_mhz, sm_max_mhz, power_w, reasons bitmask)
         self.window = None
+        self.source = None
+        self._stop = threading.Event()
+        self.proc = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append((time.time(), float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                                             sm_max, pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0, int(reasons(h))))
+                    except Exception:  # a query this driver lacks: stop sampling, report what there is
+                        return
+                    self._stop.wait(period_s)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            self.source = "nvml"
+        except Exception:
+            self._start_smi(gpu_index, int(period_s * 1000))
+
+    def _start_smi(self, gpu_index, period_ms):
         cmd = ["nvidia-smi", "-i", str(gpu_index),
                "--query-gpu=timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
-               "--format=csv,noheader,nounits", "-lms", str(period_ms)]
+               "--format=csv,noheader,nounits", "-lms", str(max(period_ms, 50))]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
+            self.source = "nvidia-smi"
         except (OSError, ValueError):
             self.proc = None
 
-    def _read(self):
+    def _read_smi(self):
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 5:
@@ -135,14 +164,16 @@ class ClockSampler:
         self.window = (t0, t1)
 
     def stop(self):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-        if self.proc is None or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock samples (NVML and nvidia-smi)"],
+                    "source": self.source}
         t0, t1 = self.window if self.window else (0, 1e18)
         inwin = [s for s in self.samples if t0 - 0.05 <= s[0] <= t1 + 0.05] or self.samples[-3:]
         reasons = set()
@@ -151,7 +182,8 @@ class ClockSampler:
                 if s[4] & bit and name != "gpu_idle":
                     reasons.add(name)
         return {"sm_mhz": statistics.median(s[1] for s in inwin), "sm_max_mhz": max(s[2] for s in inwin),
-                "power_w_max": max(s[3] for s in inwin), "samples": len(inwin), "reasons": sorted(reasons)}
+                "power_w_max": max(s[3] for s in inwin), "samples": len(inwin), "reasons": sorted(reasons),
+                "source": self.source}
 
 
 # ---------------------------------------------------------------------------
@@ -164,7 +196,7 @@ class Workload:
         self.B, self.torch = B, torch
         s, h = I.LING_MOE, I.LING_HEAD
         self.s, self.h = s, h
-        self.layers = []
+        self.layers, self.bias = [], []
         for l in range(n_layers):
             router = I.router_weight(seed, s.experts, s.hidden, layer=l, device=device)
             banks, shared = [], []
@@ -177,6 +209,8 @@ class Workload:
                 shared.append(B.moe_quantize_mxfp4(sh))
             # load time: regroup the quantised bytes into the layout moe_decode streams
             self.layers.append((router, B.moe_pack_experts(tuple(banks)), B.moe_pack_experts(tuple(shared))))
+            # the skewed regime: a per-expert logit bias N(0, 2^2), so tokens share experts
+            self.bias.append(I.router_bias(seed, s.experts, layer=l, device=device))
             del banks, shared
         self.head_bf16 = self.head = None
         if head:
@@ -196,7 +230,7 @@ class Workload:
                         for M in (1, 4)}
         torch.cuda.synchronize()
 
-    def step(self, i: int, M: int, ev=None, x_moe=None, x_head=None):
+    def step(self, i: int, M: int, ev=None, x_moe=None, x_head=None, skewed: bool = False):
         """One decode step: MoE layer (layer i mod 8) then the LM head."""
         B = self.B
         xm = self.x[M][i % N_X] if x_moe is None else x_moe
@@ -204,9 +238,10 @@ class Workload:
         if ev is not None:
             ev[0].record()
         if self.layers:
-            router, banks, shared = self.layers[i % len(self.layers)]
-            B.moe_decode(xm, router, None, banks, shared, self.s.top_k, self.out[M], self.ids[M], self.w[M],
-                         workspace=self.moe_ws[M])
+            l = i % len(self.layers)
+            router, banks, shared = self.layers[l]
+            B.moe_decode(xm, router, self.bias[l] if skewed else None, banks, shared, self.s.top_k, self.out[M],
+                         self.ids[M], self.w[M], workspace=self.moe_ws[M])
         if ev is not None:
             ev[1].record()
         if self.head is not None:
@@ -220,39 +255,48 @@ class Workload:
                                   self.logits[M], workspace=self.head_ws[M])
 
 
-def time_steps(wl, M, steps, warmup, dist, device):
-    """Device time of `steps` steps: total, MoE part and head part (us)."""
+def _q(v, f):
+    v = sorted(v)
+    return v[min(len(v) - 1, int(f * len(v)))]
+
+
+def time_steps(wl, M, steps, warmup, dist, device, skewed=False):
+    """Device time of `steps` steps (CUDA events around every step and each
+    half, on the launching stream): total, per-step distribution, MoE and
+    head parts (us)."""
     torch = wl.torch
     for i in range(warmup):
-        wl.step(i, M)
+        wl.step(i, M, skewed=skewed)
     evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     t0 = time.time()
     for i in range(steps):
-        wl.step(warmup + i, M, ev=evs[i])
+        wl.step(warmup + i, M, ev=evs[i], skewed=skewed)
     torch.cuda.synchronize()
     t1 = time.time()
     total_ms = evs[0][0].elapsed_time(evs[-1][2])
+    step = [e[0].elapsed_time(e[2]) * 1e3 for e in evs]
     moe = [e[0].elapsed_time(e[1]) * 1e3 for e in evs]
     head = [e[1].elapsed_time(e[2]) * 1e3 for e in evs]
     total_ms = max_over_ranks(total_ms, dist, device)
-    q = lambda v, f: sorted(v)[min(len(v) - 1, int(f * len(v)))]
+    med = max_over_ranks(statistics.median(step), dist, device)
     return {"total_us": total_ms * 1e3, "per_step_us": total_ms * 1e3 / steps,
+            "step_us_median": med, "step_us_p10": _q(step, 0.1), "step_us_p90": _q(step, 0.9),
             "moe_us_mean": statistics.fmean(moe), "moe_us_median": statistics.median(moe),
-            "moe_us_p10": q(moe, 0.1), "moe_us_p90": q(moe, 0.9),
+            "moe_us_p10": _q(moe, 0.1), "moe_us_p90": _q(moe, 0.9),
             "head_us_mean": statistics.fmean(head), "head_us_median": statistics.median(head),
-            "head_us_p10": q(head, 0.1), "head_us_p90": q(head, 0.9),
+            "head_us_p10": _q(head, 0.1), "head_us_p90": _q(head, 0.9),
             "wall": (t0, t1)}
 
 
-def distinct_experts(wl, M, n):
+def distinct_experts(wl, M, n, skewed=False):
     """|U|, the distinct routed experts one M-token step streams, over n steps."""
     torch = wl.torch
     us = []
     for i in range(n):
-        wl.step(i, M)
+        wl.step(i, M, skewed=skewed)
         torch.cuda.synchronize()
         us.append(len(set(wl.ids[M].cpu().numpy().reshape(-1).tolist())))
     return {"mean": statistics.fmean(us), "min": min(us), "max": max(us), "steps": n}
@@ -431,119 +475,163 @@ def stream_leg(wl, B, I, A, seed, device, steps):
 # CPU oracle (baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 
-class OracleStep:
-    """The oracle on a bounded sample of one decode step: the full router for
-    one token, a 32-row slice of each of the 8 selected experts and of the
-    shared expert, and a slice of the LM head's rows.  The measured time is
-    scaled by the inverse of each slice's fraction of its part of the step."""
+def _run_threads(fn, items, n_threads):
+    """fn over items on n_threads Python threads: the oracle's C calls release
+    the interpreter lock, so the threads run on separate cores."""
+    if n_threads <= 1 or len(items) <= 1:
+        return [fn(it) for it in items]
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=n_threads) as ex:
+        return list(ex.map(fn, items))
 
-    def __init__(self, seed: int, head_rows: int = 1024, expert_rows: int = 32):
+
+class OracleBench:
+    """The oracle (plain C, fp64) on the benchmark's own configurations, on the
+    host's cores: the tiny layer + tiny head in full (C0), the Ling layer at
+    M=1 and M=4 (C1: router, then every selected expert and the shared expert
+    in full), and the full 157,184 x 2,560 FP8 head (C3).  Work is split into
+    independent calls -- experts per (token, expert) pair, head rows in slabs
+    -- that threads run side by side; quantisation is load time, untimed."""
+
+    def __init__(self, seed: int, head_rows: int | None = None):
         import numpy as np
+        import torch
 
         import oracle
         from moe_decode_gemv_b200 import inputs as I
-        self.np, self.O, self.I = np, oracle.load(), I
-        s, h = I.LING_MOE, I.LING_HEAD
-        self.s, self.h = s, h
-        self.expert_rows, self.head_rows = expert_rows, head_rows
-        self.router = I.router_weight(seed, s.experts, s.hidden).numpy()
-        self.x = [I.hidden_states(seed, 1, s.hidden, tag=f"cpu{i}") for i in range(8)]
-        self.xb = [t.view(__import__("torch").int16).numpy().view(np.uint16) for t in self.x]
-        # LM-head slices, quantised by the oracle (load time, untimed)
-        self.head_slices = []
-        for j in range(4):
-            r0 = (j * 37 * 1024) % (h.vocab - head_rows)
-            w = I.normal(seed, f"lmhead/{r0}", (head_rows, h.hidden), I.WEIGHT_STD)
-            wb = w.view(__import__("torch").int16).numpy().view(np.uint16)
-            self.head_slices.append(self.O.fp8_rowquant(wb))
-        self.expert_cache = {}
+        self.np, self.torch, self.O, self.I, self.seed = np, torch, oracle.load(), I, seed
+        self.host_cores = os.cpu_count() or 1
+        self.cache = {}
+        self.router = {s: I.router_weight(seed, s.experts, s.hidden).numpy() for s in (I.TINY_MOE, I.LING_MOE)}
+        self.heads = {}
+        self.head_rows = head_rows  # None: the full head
+        self._head(I.TINY_HEAD, None)
+        self._head(I.LING_HEAD, head_rows)
 
-    def _expert_slice(self, e):
-        """Gate/up rows [0, r) and down columns [0, r) of expert e, quantised."""
-        if e in self.expert_cache:
-            return self.expert_cache[e]
-        np, I, s, r = self.np, self.I, self.s, self.expert_rows
-        import torch
-        q = {}
-        for kind in ("gate", "up", "down"):
-            m = I.expert_matrix(0, s, e, kind)
-            m = m[:r] if kind != "down" else m[:, :r].contiguous()
-            q[kind] = self.O.mxfp4_quantize(m.view(torch.int16).numpy().view(np.uint16))
-        self.expert_cache[e] = q
-        return q
+    def _head(self, h, rows):
+        """The FP8 head quantised by the oracle, slab by slab (all cores)."""
+        I = self.I
+        V = h.vocab if rows is None else min(rows, h.vocab)
+        slab = 8192
+        starts = list(range(0, V, slab))
 
-    def prepare(self, i):
-        _, ids, _ = self.O.router(self.xb[i % 8], self.router, None, self.s.top_k)
-        for e in list(ids[0]) + ["shared"]:
-            self._expert_slice(e if e == "shared" else int(e))
-        return ids
+        def quant(r0):
+            r1 = min(V, r0 + slab)
+            w = I.normal(self.seed, f"lmhead/{r0}", (r1 - r0, h.hidden), I.WEIGHT_STD)
+            return self.O.fp8_rowquant(w)
 
-    def run(self, i) -> float:
-        """Seconds of oracle work scaled to one full step."""
-        O, s, h = self.O, self.s, self.h
-        xb = self.xb[i % 8]
+        parts = _run_threads(quant, starts, self.host_cores)
+        self.heads[h] = (self.np.concatenate([q for q, _ in parts]), self.np.concatenate([sc for _, sc in parts]))
+
+    def _expert(self, s, e):
+        key = (s, e)
+        if key not in self.cache:
+            self.cache[key] = {k: self.O.mxfp4_quantize(self.I.expert_matrix(self.seed, s, e, k))
+                               for k in ("gate", "up", "down")}
+        return self.cache[key]
+
+    def moe_step(self, s, x, n_threads) -> float:
+        """Seconds for one layer step of x [M, H] bf16: router, top-k, the
+        selected experts and the shared expert, weighted combine."""
+        np = self.np
+        M = x.shape[0]
+        _, ids, w = self.O.router(x, self.router[s], None, s.top_k)
+        for e in set(ids.reshape(-1).tolist()) | {"shared"}:
+            self._expert(s, e)  # quantisation is load time: outside the timed region
         t0 = time.perf_counter()
-        _, ids, _ = O.router(xb, self.router, None, s.top_k)
-        t1 = time.perf_counter()
-        for e in list(ids[0]) + ["shared"]:
-            q = self._expert_slice(e if e == "shared" else int(e))
-            O.expert_mlp(xb, q["gate"], q["up"], q["down"])
-        t2 = time.perf_counter()
-        qh, sh = self.head_slices[i % len(self.head_slices)]
-        logits = O.lmhead_fp8(xb, qh, sh)
-        O.topk(logits[0], HEAD_TOPK)
-        t3 = time.perf_counter()
-        return (t1 - t0) + (t2 - t1) * (s.inter / self.expert_rows) + (t3 - t2) * (h.vocab / self.head_rows)
+        _, ids, w = self.O.router(x, self.router[s], None, s.top_k)
+        tasks = [(m, int(ids[m, r]), float(w[m, r])) for m in range(M) for r in range(s.top_k)]
+        tasks += [(m, "shared", 1.0) for m in range(M)]
 
-    def describe(self):
-        return (f"oracle (plain C, fp64, 1 thread) per step: full router for 1 token; gate/up rows and down "
-                f"columns [0,{self.expert_rows}) of the 8 routed + shared experts, scaled x{self.s.inter // self.expert_rows}; "
-                f"LM-head rows slice of {self.head_rows} of {self.h.vocab}, scaled x{self.h.vocab / self.head_rows:.1f}")
+        def run(t):
+            m, e, wt = t
+            q = self._expert(s, e)
+            out, _ = self.O.expert_mlp(x[m:m + 1], q["gate"], q["up"], q["down"])
+            return m, wt * out
+
+        y = np.zeros((M, s.hidden))
+        for m, part in _run_threads(run, tasks, n_threads):
+            y[m] += part
+        return time.perf_counter() - t0
+
+    def head_step(self, h, x, k, n_threads) -> float:
+        """Seconds for the head on x [M, H] bf16: logits over the head's rows
+        (slabs in parallel), then the top-k of each token."""
+        np = self.np
+        q, sc = self.heads[h]
+        V = q.shape[0]
+        slab = max(1024, -(-V // max(n_threads, 1)))
+        t0 = time.perf_counter()
+        parts = _run_threads(lambda r0: self.O.lmhead_fp8(x, q[r0:r0 + slab], sc[r0:r0 + slab]),
+                             list(range(0, V, slab)), n_threads)
+        logits = np.concatenate(parts, axis=1)
+        for m in range(x.shape[0]):
+            self.O.topk(logits[m], k)
+        return time.perf_counter() - t0
+
+    def step_us(self, M: int, n_threads: int, tag: str) -> dict:
+        """One step of the Ling layer + head at M tokens: us for each part."""
+        I = self.I
+        x = I.hidden_states(self.seed, M, I.LING_MOE.hidden, tag=tag)
+        moe = self.moe_step(I.LING_MOE, x, n_threads)
+        head = self.head_step(I.LING_HEAD, x, HEAD_TOPK, n_threads)
+        scale = I.LING_HEAD.vocab / self.heads[I.LING_HEAD][0].shape[0]  # 1 for the full head
+        return {"moe_us": moe * 1e6, "head_us": head * scale * 1e6, "step_us": (moe + head * scale) * 1e6}
+
+    def tiny_us(self, n_threads: int) -> float:
+        I = self.I
+        x = I.hidden_states(self.seed, 1, I.TINY_MOE.hidden, tag="cpu-tiny")
+        return (self.moe_step(I.TINY_MOE, x, n_threads) + self.head_step(I.TINY_HEAD, x, HEAD_TOPK, n_threads)) * 1e6
+
+    def describe(self, n_threads):
+        rows = "all 157,184 rows" if self.head_rows is None else f"the first {self.head_rows} rows, scaled to 157,184"
+        return (f"oracle (plain C, fp64) on {n_threads} thread(s) of {self.host_cores} host cores: Ling layer in full "
+                f"(router, every selected expert and the shared expert, combine) + FP8 head over {rows} + top-{HEAD_TOPK}")
 
 
-def cpu_baseline(seed, budget_s=15.0):
-    st = OracleStep(seed)
-    for i in range(8):
-        st.prepare(i)
-    times = []
-    t_start = time.perf_counter()
-    i = 0
-    while time.perf_counter() - t_start < budget_s or i < 3:
-        times.append(st.run(i))
-        i += 1
-    us = statistics.fmean(times) * 1e6
-    return {"value": us, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": st.describe() + f"; {i} steps"}
+def cpu_baseline(seed, reps=2):
+    """The oracle timed on the host's cores, 1 thread and all of them: C0 in
+    full, C1 (Ling layer) and C3 (Ling head) at M=1 and M=4, `reps` steps
+    each (median)."""
+    ob = OracleBench(seed)
+    T = ob.host_cores
+    detail = {}
+    for n in sorted({1, T}):
+        d = {"C0_tiny_step_us": statistics.median(ob.tiny_us(n) for _ in range(reps))}
+        for M in (1, 4):
+            runs = [ob.step_us(M, n, tag=f"cpu{M}-{r}") for r in range(reps)]
+            d[f"C1_moe_m{M}_us"] = statistics.median(r["moe_us"] for r in runs)
+            d[f"C3_head_m{M}_us"] = statistics.median(r["head_us"] for r in runs)
+            d[f"step_m{M}_us"] = statistics.median(r["step_us"] for r in runs)
+        detail[f"{n}_threads"] = d
+    best = detail[f"{T}_threads"]
+    return {"value": best["step_m1_us"], "unit": UNIT, "cores": T, "host_cores": T, "kind": "oracle",
+            "sample": ob.describe(T) + f"; median of {reps} steps per configuration; 1-thread timings in detail",
+            "detail": detail}
 
 
 def reference_arm(args):
     world, rank, local = dist_env()
     if rank != 0:
         return 0
-    budget = 120.0
-    st = OracleStep(args.seed)
-    for i in range(8):
-        st.prepare(i)
-    # size the sample so that warmup + steps fit the budget
-    probe = [st.run(i) for i in range(2)]
-    t_probe = time.perf_counter()
-    st.run(2)
-    per = time.perf_counter() - t_probe
+    budget = 150.0
+    probe = OracleBench(args.seed, head_rows=8192)
+    T = probe.host_cores
+    per = probe.step_us(1, T, tag="ref-probe")["step_us"] * 1e-6  # the full step, estimated from 8,192 head rows
     total = args.steps + args.warmup
-    if per * total > budget:
-        shrink = max(1, int(per * total / budget) + 1)
-        st.head_rows = max(64, st.head_rows // shrink)
-        st.head_slices = [(q[: st.head_rows], s[: st.head_rows]) for q, s in st.head_slices]
+    rows = None if per * total <= budget else max(8192, int(157184 * budget / (per * total)) // 8192 * 8192)
+    ob = OracleBench(args.seed, head_rows=rows)
     for i in range(args.warmup):
-        st.run(i)
-    times = [st.run(args.warmup + i) for i in range(args.steps)]
-    us = statistics.fmean(times) * 1e6
+        ob.step_us(1, T, tag=f"ref{i}")
+    times = [ob.step_us(1, T, tag=f"ref{args.warmup + i}")["step_us"] for i in range(args.steps)]
+    us = statistics.median(times)
     line = {"impl": "reference", "metric": METRIC, "value": us, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(),
-            "cpu_baseline": {"value": us, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": st.describe()},
+            "cpu_baseline": {"value": us, "unit": UNIT, "cores": T, "host_cores": T, "kind": "oracle",
+                             "sample": ob.describe(T)},
             "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    del probe
     print(json.dumps(line))
     return 0
 
@@ -563,7 +651,7 @@ def measured_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("lmhead_kernels.cu", "common.cuh"):
+    for name in ("lmhead_fp8.cu", "common.cuh"):
         with open(os.path.join(ROOT, "moe_decode_gemv_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -612,9 +700,9 @@ def main():
     from moe_decode_gemv_b200 import binding as B
     from moe_decode_gemv_b200 import inputs as I
 
+    sampler = ClockSampler(local)  # started early: it samples through every timed region below
     n_layers = 0 if args.only == "head" else args.layers
     wl = Workload(B, I, args.seed + rank, device, n_layers=n_layers, head=args.only != "moe")
-    sampler = ClockSampler(local)
     m1 = time_steps(wl, 1, args.steps, args.warmup, dist, device)
     sampler.mark(*m1["wall"])
     clocks = sampler.stop()
@@ -624,42 +712,58 @@ def main():
                           "moe_us_mean": m1["moe_us_mean"], "head_us_mean": m1["head_us_mean"], "clocks": clocks}))
         return 0
     e2e_us, h2d, d2h = time_e2e(wl, 1, args.steps, args.warmup, dist, device)
-    m4 = None if args.no_m4 else time_steps(wl, 4, max(args.steps // 2, 1), args.warmup, dist, device)
+    m4 = {}
+    if not args.no_m4:
+        for regime, skewed in (("uniform", False), ("skewed", True)):
+            m4[regime] = time_steps(wl, 4, max(args.steps // 2, 1), args.warmup, dist, device, skewed=skewed)
+            m4[regime]["distinct_experts"] = distinct_experts(wl, 4, 32, skewed=skewed)
     bf16_head_us = time_bf16_head(wl, 1, 200)
     status = [B.moe_workspace_status(ws) for ws in list(wl.moe_ws.values()) + list(wl.head_ws.values())]
     if any(s != B.Status.OK for s in status):
         raise SystemExit(f"device status not OK: {status}")
 
-    head_bytes = A.lmhead_fp8_bytes(I.LING_HEAD)
-    moe_bytes_m1 = A.moe_layer_bytes(I.LING_MOE, I.LING_MOE.top_k)
+    s, h = I.LING_MOE, I.LING_HEAD
+    head_bytes = A.lmhead_fp8_bytes(h)
+    moe_bytes_m1 = A.moe_layer_bytes(s, s.top_k)
     peak, peak_kind = measured_peaks()
-    achieved = head_bytes / (m1["head_us_mean"] * 1e-6) / 1e9
-    value = m1["total_us"] / (args.steps * world)
+    gbs = lambda nbytes, us: nbytes / (us * 1e-6) / 1e9
+    achieved = gbs(head_bytes, m1["head_us_mean"])
+    # the headline: median device time per M=1 step over all ranks' steps
+    value = m1["step_us_median"] / world
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": m1["per_step_us"] / 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic", "config": workload_config(),
-        "roofline": {"bound": "hbm", "kernel": "lmhead_fp8_tiled_kernel (FP8 LM head, M=1)", "achieved": achieved,
+        "ms_per_step": m1["step_us_median"] / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(),
+        "value_stats": {"median_us": m1["step_us_median"], "p10_us": m1["step_us_p10"], "p90_us": m1["step_us_p90"],
+                        "mean_us": m1["per_step_us"], "steps": args.steps},
+        "arithmetic": "fp32 accumulate; activations carried as two E4M3 parts per block (x) and two f16 parts "
+                      "per 16-value slice (h); weights MXFP4 (experts) and E4M3 + fp32 row scale (head)",
+        "roofline": {"bound": "hbm", "kernel": "lmhead_fp8_kernel (FP8 LM head, M=1)", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": profiled_traffic(), "algorithmic_bytes_per_launch": head_bytes},
         "breakdown_m1": {"moe_us_mean": m1["moe_us_mean"], "moe_us_median": m1["moe_us_median"],
                          "moe_us_p10": m1["moe_us_p10"], "moe_us_p90": m1["moe_us_p90"],
                          "head_us_mean": m1["head_us_mean"], "head_us_median": m1["head_us_median"],
                          "head_us_p10": m1["head_us_p10"], "head_us_p90": m1["head_us_p90"],
-                         "moe_bytes": moe_bytes_m1,
-                         "moe_gbs": moe_bytes_m1 / (m1["moe_us_mean"] * 1e-6) / 1e9,
-                         "head_gbs": achieved},
+                         "moe_bytes": moe_bytes_m1, "moe_gbs": gbs(moe_bytes_m1, m1["moe_us_mean"]),
+                         "moe_frac": gbs(moe_bytes_m1, m1["moe_us_mean"]) / peak,
+                         "head_gbs": achieved, "head_frac": achieved / peak},
         "bf16_head_us": bf16_head_us,
-        "bf16_head_gbs": A.lmhead_bf16_bytes(I.LING_HEAD) / (bf16_head_us * 1e-6) / 1e9,
+        "bf16_head_gbs": gbs(A.lmhead_bf16_bytes(h), bf16_head_us),
         "clocks": clocks,
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,  # one MoE and one LM-head kernel per timed step
         "path": B.moe_query_path(),
     }
-    if m4 is not None:
-        line["m4"] = {"us_per_step": m4["per_step_us"], "moe_us_mean": m4["moe_us_mean"],
-                      "head_us_mean": m4["head_us_mean"], "steps": max(args.steps // 2, 1),
-                      "distinct_experts": distinct_experts(wl, 4, 16)}
+    for regime, r in m4.items():
+        u = r["distinct_experts"]["mean"]
+        mb = A.moe_layer_bytes(s, u)
+        line.setdefault("m4", {})[regime] = {
+            "step_us_median": r["step_us_median"], "step_us_p10": r["step_us_p10"], "step_us_p90": r["step_us_p90"],
+            "moe_us_mean": r["moe_us_mean"], "head_us_mean": r["head_us_mean"], "steps": max(args.steps // 2, 1),
+            "distinct_experts": r["distinct_experts"], "moe_bytes_at_mean_U": mb,
+            "moe_gbs": gbs(mb, r["moe_us_mean"]), "moe_frac": gbs(mb, r["moe_us_mean"]) / peak,
+            "head_gbs": gbs(head_bytes, r["head_us_mean"]), "head_frac": gbs(head_bytes, r["head_us_mean"]) / peak}
     line["read_ceiling"] = read_ceiling(B, wl.head.q)
     if not args.no_stream:
         try:

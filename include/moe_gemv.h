@@ -306,18 +306,28 @@ MOE_API moe_status moe_mtp_accept(const int32_t* draft_ids, const int32_t* verif
  * counterpart on the pages: this is an interface convenience.  The scratch is
  * one fixed device array of MOE_LMHEAD_NOALLOC_SCRATCH_BYTES, held by every
  * GPU that loads the library until the process exits.  It must fit a 64-byte
- * header plus (SM count) x M x top_k x 8 bytes of candidate lists, e.g.
- * M x top_k <= 221 on a 148-SM B200; larger requests return
- * MOE_ERR_WORKSPACE.  The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress) and should come before any stream capture.
- * Each call clears the array's header on `stream` before its kernel.  All
- * calls share the array, so calls that overlap on the GPU (different
- * streams, or different threads) race: serialise them.  Allocates nothing.
- * The head is the tiled one, as for lmhead_decode.                         */
+ * header plus M candidate lists of (SM count) x top_k entries of 8 bytes,
+ * each list rounded up to an even entry count: M x top_k <= 220 on a 148-SM
+ * B200 (e.g. M = 4, top_k <= 55); larger requests return MOE_ERR_WORKSPACE.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and should come before any stream capture.  Each
+ * call resets the header's counters on `stream` before its kernel but keeps
+ * its status word: a device error (a wait that ran out) stays there until
+ * lmhead_noalloc_status reads and clears it.  All calls share the array, so
+ * calls that overlap on the GPU (different streams, or different threads)
+ * race: serialise them.  Allocates nothing.  The head is the tiled one, as
+ * for lmhead_decode.                                                         */
 #define MOE_LMHEAD_NOALLOC_SCRATCH_BYTES (256u * 1024u)
 MOE_API moe_status lmhead_decode_noalloc(const uint16_t* hidden_bf16, const moe_fp8_head* head,
                                          int32_t M, int32_t top_k, int32_t* topk_ids, float* topk_vals,
                                          float* logits, void* stream);
+
+/* The device status of lmhead_decode_noalloc on the current device: waits
+ * for `stream` (cudaStreamSynchronize), writes to *status_out the first
+ * moe_status a no-alloc launch reported since the last read (MOE_OK if none)
+ * and clears it.  Returns MOE_OK, MOE_ERR_INVALID_ARG (status_out NULL) or
+ * MOE_ERR_CUDA.  Allocates nothing; do not call it during stream capture.   */
+MOE_API moe_status lmhead_noalloc_status(int32_t* status_out, void* stream);
 
 /* ---- between the layers of a decode step ---------------------------------- */
 

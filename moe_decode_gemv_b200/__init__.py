@@ -19,7 +19,7 @@ from __future__ import annotations
 _BINDING_NAMES = {
     "Status", "MoEError", "Format", "library", "library_path",
     "moe_quantize_mxfp4", "moe_pack_experts", "lmhead_quantize_fp8", "lmhead_tile_fp8",
-    "moe_decode", "lmhead_decode", "lmhead_decode_bf16", "lmhead_decode_noalloc",
+    "moe_decode", "lmhead_decode", "lmhead_decode_bf16", "lmhead_decode_noalloc", "lmhead_noalloc_status",
     "lmhead_sample", "moe_mtp_accept", "moe_rmsnorm_bf16", "moe_embed_gather", "moe_stream_read",
     "moe_workspace_bytes", "lmhead_workspace_bytes", "new_workspace", "moe_workspace_status",
     "moe_query_path", "MXFP4Bank", "PackedBank", "FP8Head",

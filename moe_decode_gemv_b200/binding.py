@@ -90,6 +90,7 @@ def _load() -> ctypes.CDLL:
         "lmhead_decode": ([P, ctypes.POINTER(_Fp8Head), I32, I32, P, P, P, P, SZ, P], I32),
         "lmhead_decode_bf16": ([P, ctypes.POINTER(_Bf16Head), I32, I32, P, P, P, P, SZ, P], I32),
         "lmhead_decode_noalloc": ([P, ctypes.POINTER(_Fp8Head), I32, I32, P, P, P, P], I32),
+        "lmhead_noalloc_status": ([ctypes.POINTER(I32), P], I32),
         "moe_rmsnorm_bf16": ([P, I32, I32, ctypes.c_float, P, P], I32),
         "moe_embed_gather": ([P, I64, I64, P, I32, I32, P, P], I32),
         "moe_workspace_reset": ([P, SZ, P], I32),
@@ -338,6 +339,16 @@ def lmhead_decode_noalloc(hidden: torch.Tensor, head: FP8Head, top_k: int, topk_
                                        _ptr(topk_vals), _ptr(logits), _stream(stream))
     _check(st, "lmhead_decode_noalloc")
     return topk_ids, topk_vals
+
+
+def lmhead_noalloc_status(stream=None) -> int:
+    """The first device status a lmhead_decode_noalloc launch reported since
+    the last read (Status.OK if none), cleared by the read; waits for
+    `stream`."""
+    out = ctypes.c_int32(0)
+    st = library.lmhead_noalloc_status(ctypes.byref(out), _stream(stream))
+    _check(st, "lmhead_noalloc_status")
+    return int(out.value)
 
 
 def lmhead_sample(topk_ids: torch.Tensor, topk_vals: torch.Tensor, temperature: float, top_p: float,

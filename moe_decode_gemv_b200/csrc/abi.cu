@@ -19,7 +19,7 @@
 
 namespace {
 
-constexpr int kHeadMaxGrid = 1024;  // upper bound on LM-head CTAs (sizes the candidate buffer)
+
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -61,7 +61,7 @@ bool head_shape_ok(int64_t vocab, int64_t hidden, int elem_bytes) {
 }
 
 size_t head_ws_bytes(int32_t M, int32_t top_k) {
-  return sizeof(moe::WsHeader) + moe::lmhead_cand_bytes(kHeadMaxGrid, M, top_k);
+  return sizeof(moe::WsHeader) + moe::lmhead_cand_bytes(moe::kLmheadMaxGrid, M, top_k);
 }
 
 moe_status launch_head_common(const uint16_t* hidden, const void* w, const float* scale, bool fp8, int64_t V,
@@ -77,9 +77,7 @@ moe_status launch_head_common(const uint16_t* hidden, const void* w, const float
 
   int dev = 0, sms = 0;
   if (moe::current_device_sms(&dev, &sms) != cudaSuccess) return MOE_ERR_CUDA;
-  const int64_t ntiles = (V + 15) / 16;
-  int grid = sms < kHeadMaxGrid ? sms : kHeadMaxGrid;
-  if (grid > ntiles) grid = (int)ntiles;
+  const int grid = moe::lmhead_grid(sms, V);
   int stages = 0;
   size_t smem = 0;  // each CTA keeps its rows' logits in shared memory: a limit on vocab / SMs
   if (!moe::lmhead_plan((int)H, fp8 ? 1 : 2, M, top_k, V, grid, &stages, &smem)) return MOE_ERR_UNSUPPORTED_SHAPE;

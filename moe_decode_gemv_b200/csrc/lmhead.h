@@ -17,6 +17,15 @@ int lmhead_max_slices();
 bool lmhead_plan(int H, int elem_bytes, int M, int top_k, int64_t V, int grid, int* stages, size_t* smem);
 bool lmhead_fp8_plan(int H, int M, int top_k, int64_t V, int grid, int* stages, size_t* smem);
 size_t lmhead_cand_bytes(int grid, int M, int top_k);
+// CTAs of one head launch: one per SM, at most one per 16-row tile and at
+// most kLmheadMaxGrid (every entry point launches this many).
+constexpr int kLmheadMaxGrid = 1024;
+inline int lmhead_grid(int sms, int64_t V) {
+  const int64_t ntiles = (V + 15) / 16;
+  int64_t g = sms < kLmheadMaxGrid ? sms : kLmheadMaxGrid;
+  if (g > ntiles) g = ntiles;
+  return (int)g;
+}
 // Bytes of the fragment-tiled FP8 head (whole 16-row tiles, zero rows past V).
 size_t lmhead_tiled_bytes(int64_t V, int H);
 cudaError_t launch_tile_fp8_head(const uint8_t* q, int64_t V, int H, uint8_t* out, cudaStream_t st);

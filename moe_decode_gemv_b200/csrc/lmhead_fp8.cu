@@ -594,7 +594,8 @@ lmhead_fp8_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
       }
     }
     __syncthreads();
-    // 3. rank the survivors; pad when fewer than k values are admissible
+    // 4. rank the survivors by counting; pad when fewer than k values are
+    // admissible
     {
       const int per = kThreadsF / mt, j = t / per, q0 = t - j * per;
       if (j < mt) {
@@ -647,6 +648,7 @@ cudaError_t launch_fp8_t(const uint16_t* x, const uint8_t* qt, const float* s, i
 }  // namespace
 
 bool lmhead_fp8_plan(int H, int M, int top_k, int64_t V, int grid, int* stages, size_t* smem) {
+  if (grid < 1 || grid > kLmheadMaxGrid) return false;
   if (H < 64 || H % 64 != 0 || H > kMaxHF || M < 1 || M > 4 || top_k < 1 || top_k > 64) return false;
   for (int st = kMaxStagesF; st >= 2; --st) {
     const HeadGeo g = head_geo(V, H, M, grid, st, top_k);

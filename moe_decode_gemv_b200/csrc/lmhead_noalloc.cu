@@ -64,8 +64,7 @@ extern "C" moe_status lmhead_decode_noalloc(const uint16_t* hidden_bf16, const m
   // one CTA per SM, as lmhead_decode launches; its candidate lists must fit
   int dev = 0, sms = 0;
   if (moe::current_device_sms(&dev, &sms) != cudaSuccess) return MOE_ERR_CUDA;
-  const int64_t ntiles = (V + 15) / 16;
-  const int grid = (int)(sms < ntiles ? sms : ntiles);
+  const int grid = moe::lmhead_grid(sms, V);
   if (kHeaderBytes + moe::lmhead_cand_bytes(grid, M, top_k) > kScratchBytes) return MOE_ERR_WORKSPACE;
   int stages = 0;
   size_t smem = 0;
@@ -75,11 +74,29 @@ extern "C" moe_status lmhead_decode_noalloc(const uint16_t* hidden_bf16, const m
   const moe_status st = scratch_for_current_device(&scratch);
   if (st != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the ticket must start at zero: clear the header (the lists need no clearing)
-  if (cudaMemsetAsync(scratch, 0, kHeaderBytes, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // the counters must start at zero: clear the header after its status word,
+  // which keeps the first error until lmhead_noalloc_status reads it (the
+  // lists need no clearing)
+  if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + sizeof(int32_t), 0, kHeaderBytes - sizeof(int32_t), s) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
   auto* hdr = static_cast<moe::WsHeader*>(scratch);
   void* cand = static_cast<uint8_t*>(scratch) + kHeaderBytes;
   const cudaError_t e = moe::launch_lmhead_fp8(hidden_bf16, head->q, head->row_scale, V, (int)H, M, top_k, logits,
                                                topk_ids, topk_vals, hdr, cand, grid, s);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" moe_status lmhead_noalloc_status(int32_t* status_out, void* stream) {
+  if (!status_out) return MOE_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  const moe_status st = scratch_for_current_device(&scratch);
+  if (st != MOE_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  auto* hdr = static_cast<moe::WsHeader*>(scratch);
+  int32_t status = 0;
+  if (cudaMemcpy(&status, &hdr->status, sizeof(status), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (status != 0 && cudaMemset(&hdr->status, 0, sizeof(status)) != cudaSuccess) return MOE_ERR_CUDA;
+  *status_out = status;
+  return MOE_OK;
 }

@@ -143,6 +143,7 @@ def test_lmhead_rejects_bad_arguments(lib):
     assert call(lib._Fp8Head(3, 4096, 256, A, A)) == S.FORMAT_MISMATCH
     assert L.lmhead_decode_noalloc(A, ctypes.byref(lib._Fp8Head(3, 4096, 256, A, A)), 1, 1, A, A, None,
                                    None) == S.FORMAT_MISMATCH
+    assert L.lmhead_noalloc_status(None, None) == S.INVALID_ARG  # checked before any CUDA call
     assert call(fp8, M=0) == S.INVALID_ARG
     assert call(fp8, k=65) == S.INVALID_ARG
     assert call(fp8, ids=0) == S.INVALID_ARG

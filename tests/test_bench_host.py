@@ -82,7 +82,7 @@ def test_traffic_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch)
         f"# comment\nkernel_source_sha256_16 = {h}\ndram_bytes_per_launch = 409988352\n")
     src = tmp_path / "moe_decode_gemv_b200" / "csrc"
     src.mkdir(parents=True)
-    for name in ("lmhead_kernels.cu", "common.cuh"):
+    for name in ("lmhead_fp8.cu", "common.cuh"):
         with open(os.path.join(ROOT, "moe_decode_gemv_b200", "csrc", name), "rb") as f:
             (src / name).write_bytes(f.read())
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))

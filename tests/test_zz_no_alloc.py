@@ -46,20 +46,56 @@ def test_matches_workspace_entry_point_twice(B, shape, M, k):
         assert np.abs(v - rv).max() <= MAX_ABS_TOL
         lg, rlg = logits.cpu().numpy(), ref_logits.cpu().numpy()
         assert rel_l2(lg, rlg) <= REL_L2_TOL and np.abs(lg - rlg).max() <= MAX_ABS_TOL
+    assert B.lmhead_noalloc_status() == B.Status.OK  # no device error since the last read
+
+
+def _need(G, M, k):
+    """Scratch bytes of one call: the 64-byte header, then M lists of G x k
+    candidates of 8 bytes, each list rounded up to an even entry count."""
+    return 64 + M * ((G * k + 1) & ~1) * 8
+
+
+def _raw(B, x, head, M, k, ids, vals, logits=None):
+    c = head._c()
+    return B.library.lmhead_decode_noalloc(ctypes.c_void_p(x.data_ptr()), ctypes.byref(c), M, k,
+                                           ctypes.c_void_p(ids.data_ptr()), ctypes.c_void_p(vals.data_ptr()),
+                                           None if logits is None else ctypes.c_void_p(logits.data_ptr()), None)
 
 
 def test_refuses_requests_beyond_its_scratch(B):
     """M x top_k candidate lists for every SM must fit the fixed scratch."""
     head = B.lmhead_quantize_fp8(I.lmhead_weight(0, I.TINY_HEAD).cuda())
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    limit = B.library.lmhead_decode_noalloc  # raw C call: expect a status, not an exception
     M, k = 4, 64
-    need = 64 + min(sms, I.TINY_HEAD.vocab // 16) * M * k * 8
+    need = _need(min(sms, I.TINY_HEAD.vocab // 16), M, k)
     x = I.hidden_states(0, M, I.TINY_HEAD.hidden).cuda()
     ids, vals, _ = _outputs(M, k, I.TINY_HEAD.vocab)
-    c = head._c()
-    st = limit(ctypes.c_void_p(x.data_ptr()), ctypes.byref(c), M, k, ctypes.c_void_p(ids.data_ptr()),
-               ctypes.c_void_p(vals.data_ptr()), None, None)
+    st = _raw(B, x, head, M, k, ids, vals)  # raw C call: expect a status, not an exception
     expected = B.Status.WORKSPACE if need > 256 * 1024 else B.Status.OK
     assert st == expected, (st, need)
     torch.cuda.synchronize()
+    assert B.lmhead_noalloc_status() == B.Status.OK
+
+
+def test_largest_request_that_fits_and_the_next(B):
+    """On the Ling head at M = 4: the largest top_k whose lists fit the scratch
+    runs and matches lmhead_decode; one more is refused with WORKSPACE."""
+    shape, M = I.LING_HEAD, 4
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    G = min(sms, shape.vocab // 16)
+    fits = [k for k in range(1, 65) if _need(G, M, k) <= 256 * 1024]
+    k = max(fits)
+    head = B.lmhead_quantize_fp8(I.lmhead_weight(0, shape).cuda())
+    x = I.hidden_states(5, M, shape.hidden, tag="noalloc-limit").cuda()
+    ref_ids, ref_vals, _ = _outputs(M, k, shape.vocab)
+    B.lmhead_decode(x, head, k, ref_ids, ref_vals)
+    ids, vals, _ = _outputs(M, k, shape.vocab)
+    assert _raw(B, x, head, M, k, ids, vals) == B.Status.OK
+    torch.cuda.synchronize()
+    assert torch.equal(ids, ref_ids)
+    assert np.abs(vals.cpu().numpy() - ref_vals.cpu().numpy()).max() <= MAX_ABS_TOL
+    assert B.lmhead_noalloc_status() == B.Status.OK
+    if k < 64:
+        ids2, vals2, _ = _outputs(M, k + 1, shape.vocab)
+        assert _raw(B, x, head, M, k + 1, ids2, vals2) == B.Status.WORKSPACE
+    print(f"no-alloc limit on {sms} SMs at M={M}: top_k {k} runs, {k + 1} is refused")
