@@ -219,11 +219,20 @@ lmhead_fp8_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
     mbar_init(&C.lbar, 1);
     fence_mbar_init();
     C.poison = 0;
+  }
+  __syncthreads();
+  pdl_launch_dependents();  // the next kernel may launch; its CTAs start as this one's exit
+  if (t == 0) {
+    // The tokens (and, after them, everything this kernel writes) may come
+    // from the previous kernel on the stream: wait for it here, while the
+    // producer already streams weights.  The other threads see its results
+    // through the tokens' barrier; the producer waits on its own before it
+    // takes tiles from the workspace's counter.
+    pdl_wait();
     const uint32_t xbytes = (uint32_t)(M * H * 2);
     mbar_arrive_expect_tx(&C.xbar, xbytes);
     bulk_g2s(work, x, xbytes, &C.xbar, l2_evict_last_policy());
   }
-  __syncthreads();
   auto poisoned = [&]() -> bool { return *(volatile int*)&C.poison != 0; };
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {  // bounded; every lane polls
     if (poisoned()) return false;
@@ -251,6 +260,7 @@ lmhead_fp8_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
           if (it < geo.ps) {
             tile = (int64_t)blockIdx.x * geo.ps + it;
           } else {
+            if (it == geo.ps) pdl_wait();  // the counter belongs to the workspace: after the previous kernel
             if (!have_next) next = atomicAdd(&hdr->tiles, 1u);
             have_next = false;
             tile = geo.dyn0 + next;
@@ -258,6 +268,7 @@ lmhead_fp8_kernel(const uint16_t* __restrict__ x,       // [M][H] bf16
           }
         }
         if (tile >= 0 && it + 1 >= geo.ps && it + 1 < geo.cap) {  // every fetched value is used next
+          if (it + 1 == geo.ps) pdl_wait();
           next = atomicAdd(&hdr->tiles, 1u);
           have_next = true;
         }
@@ -640,9 +651,8 @@ cudaError_t launch_fp8_t(const uint16_t* x, const uint8_t* qt, const float* s, i
                          size_t smem, cudaStream_t st) {
   cudaError_t e = ensure_smem_optin<lmhead_fp8_kernel<kS>>();
   if (e != cudaSuccess) return e;
-  lmhead_fp8_kernel<kS><<<grid, kThreadsF, smem, st>>>(x, qt, s, V, H, M, top_k, stages, logits, ids, vals, hdr,
-                                                      reinterpret_cast<HeadCand*>(cand));
-  return cudaGetLastError();
+  return launch_dependent(lmhead_fp8_kernel<kS>, dim3(grid), dim3(kThreadsF), smem, st, false, x, qt, s, V, H, M,
+                          top_k, stages, logits, ids, vals, hdr, reinterpret_cast<HeadCand*>(cand));
 }
 
 }  // namespace

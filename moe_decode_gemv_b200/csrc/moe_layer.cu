@@ -211,8 +211,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   const int nb = geo.nb, n_sl = geo.n_sl;
   const MoeWs ws = a.ws;
   WsHeader* hdr = ws.hdr;
-  // This call's tag: the epoch advances once per call, after every CTA has read it.
-  const uint32_t tag = ld_relaxed_u32(&hdr->epoch) + 1u;
   const uint64_t policy = l2_evict_first_policy();
   const uint16_t* xs = reinterpret_cast<const uint16_t*>(scratch);  // the tokens, [M][H] bf16
 
@@ -242,11 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
     mbar_init(&C.xbar, 1);
     fence_mbar_init();
     C.poison = 0;
-    // the tokens first (the router needs them), then the shared expert's items
-    const uint32_t xbytes = (uint32_t)(M * H * 2);
-    mbar_arrive_expect_tx(&C.xbar, xbytes);
-    bulk_g2s(scratch, a.x, xbytes, &C.xbar, l2_evict_last_policy());
-    top_up(n_pre);
+    top_up(n_pre);  // the shared expert's items: weights, which no kernel writes
   }
 
   // ---- router loads of this CTA's rows: the first chunk goes out now ----
@@ -276,6 +270,18 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   router_slot(0, r_row, r_f0, r_f1);
   if (R > 0) router_load(r_row, r_f0 + lane, r_f1);
   __syncthreads();  // the barriers are initialised
+  // Everything below may read what the previous kernel on the stream wrote
+  // (the tokens, the workspace): wait for it.  The weight copies and loads
+  // above are already on their way.
+  pdl_wait();
+  pdl_launch_dependents();  // the next kernel may launch; its CTAs start as this one's exit
+  // This call's tag: the epoch advances once per call, after every CTA has read it.
+  const uint32_t tag = ld_relaxed_u32(&hdr->epoch) + 1u;
+  if (threadIdx.x == 0) {
+    const uint32_t xbytes = (uint32_t)(M * H * 2);
+    mbar_arrive_expect_tx(&C.xbar, xbytes);
+    bulk_g2s(scratch, a.x, xbytes, &C.xbar, l2_evict_last_policy());
+  }
 
   auto poisoned = [&]() -> bool { return *(volatile int*)&C.poison != 0; };
   auto fail = [&]() {  // the first wait of this CTA that ran out
@@ -701,18 +707,9 @@ cudaError_t launch_layer_t(const LayerArgs& a, cudaStream_t st) {
   int dev = 0, sms = 0;
   if ((e = current_device_sms(&dev, &sms)) != cudaSuccess) return e;
   const Geo geo(a.H, a.I);
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(sms < MoeWs::kMaxGrid ? sms : MoeWs::kMaxGrid);  // one CTA per SM, all resident
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = (size_t)kCtlBytes + scratch_bytes(a.H) + (size_t)a.stages * geo.stage_bytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, moe_layer_kernel<kB>, a);
-  if (e != cudaSuccess) (void)cudaGetLastError();  // leave no stale error for the next call to find
+  const int grid = sms < MoeWs::kMaxGrid ? sms : MoeWs::kMaxGrid;  // one CTA per SM, all resident
+  const size_t smem = (size_t)kCtlBytes + scratch_bytes(a.H) + (size_t)a.stages * geo.stage_bytes;
+  e = launch_dependent(moe_layer_kernel<kB>, dim3(grid), dim3(kThreads), smem, st, true, a);
   return e;
 }
 

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "device_cache.h"
 #include "stack.h"
 
 namespace moe {
@@ -15,6 +16,8 @@ namespace {
 
 // One CTA per row.
 __global__ void rmsnorm_bf16_kernel(const float* __restrict__ y, int H, float eps, uint16_t* __restrict__ out) {
+  pdl_wait();  // y comes from the previous kernel
+  pdl_launch_dependents();
   const float* row = y + (size_t)blockIdx.x * H;
   float ss = 0.f;
   for (int j = threadIdx.x; j < H; j += blockDim.x) ss = fmaf(row[j], row[j], ss);
@@ -40,6 +43,8 @@ __global__ void rmsnorm_bf16_kernel(const float* __restrict__ y, int H, float ep
 // row (no out-of-bounds read).
 __global__ void embed_gather_kernel(const uint16_t* __restrict__ table, int64_t V, int H,
                                     const int32_t* __restrict__ ids, int ids_stride, uint16_t* __restrict__ out) {
+  pdl_wait();  // ids come from the previous kernel
+  pdl_launch_dependents();
   const int32_t id = ids[(size_t)blockIdx.x * ids_stride];
   const bool ok = id >= 0 && id < V;
   const uint4* src = reinterpret_cast<const uint4*>(table + (size_t)(ok ? id : 0) * H);
@@ -75,14 +80,12 @@ cudaError_t launch_stream_read(const void* src, size_t bytes, uint32_t* sink, in
 }
 
 cudaError_t launch_rmsnorm_bf16(const float* y, int M, int H, float eps, uint16_t* out, cudaStream_t st) {
-  rmsnorm_bf16_kernel<<<M, 256, 0, st>>>(y, H, eps, out);
-  return cudaGetLastError();
+  return launch_dependent(rmsnorm_bf16_kernel, dim3(M), dim3(256), 0, st, false, y, H, eps, out);
 }
 
 cudaError_t launch_embed_gather(const uint16_t* table, int64_t V, int H, const int32_t* ids, int ids_stride, int M,
                                 uint16_t* out, cudaStream_t st) {
-  embed_gather_kernel<<<M, 128, 0, st>>>(table, V, H, ids, ids_stride, out);
-  return cudaGetLastError();
+  return launch_dependent(embed_gather_kernel, dim3(M), dim3(128), 0, st, false, table, V, H, ids, ids_stride, out);
 }
 
 }  // namespace moe
