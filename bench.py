@@ -53,6 +53,7 @@ def parse():
     p.add_argument("--only", choices=["all", "head", "moe"], default="all",
                    help="profiling aid: time only one half of the step (small device footprint)")
     p.add_argument("--layers", type=int, default=N_LAYERS, help="layer copies that rotate (profiling aid)")
+    p.add_argument("--profile-m", type=int, choices=[1, 4], default=1, help="tokens per step with --only (profiling aid)")
     p.add_argument("--no-stream", action="store_true", help="skip the 16-layer decode-stream leg")
     p.add_argument("--stream-steps", type=int, default=200)
     return p.parse_args()
@@ -721,12 +722,12 @@ def main():
     sampler = ClockSampler(local)  # started early: it samples through every timed region below
     n_layers = 0 if args.only == "head" else args.layers
     wl = Workload(B, I, args.seed + rank, device, n_layers=n_layers, head=args.only != "moe")
-    m1 = time_steps(wl, 1, args.steps, args.warmup, dist, device)
+    m1 = time_steps(wl, 1 if args.only == "all" else args.profile_m, args.steps, args.warmup, dist, device)
     sampler.mark(*m1["wall"])
     clocks = sampler.stop()
     if args.only != "all":
         # profiling aid: no end-to-end, M=4 or CPU legs
-        print(json.dumps({"only": args.only, "steps": args.steps, "per_step_us": m1["per_step_us"],
+        print(json.dumps({"only": args.only, "M": args.profile_m, "steps": args.steps, "per_step_us": m1["per_step_us"],
                           "moe_us_mean": m1["moe_us_mean"], "head_us_mean": m1["head_us_mean"], "clocks": clocks}))
         return 0
     e2e_us, h2d, d2h = time_e2e(wl, 1, args.steps, args.warmup, dist, device)
