@@ -271,11 +271,14 @@ moe_status moe_query_path(char* buf, size_t n) {
   if (!buf || n == 0) return MOE_ERR_INVALID_ARG;
   const char* desc =
       "sm_100a; moe: one cooperative persistent kernel (router fp32 GEMV with epoch-tagged logits, "
-      "bitonic top-k softmax routing in every CTA, split-K over the intermediate: 16-row slices of MXFP4 "
-      "E2M1/E8M0-32 gate/up + SiLU + down per work item, cp.async ring, E2M1->E5M2 by bit moves into "
-      "mma.sync m16n8k32 e5m2 x e4m3 with per-block activation scales, one grid barrier, fixed-order combine); "
-      "lm-head: online-FP8 E4M3 per-row-scale GEMV over the fragment-tiled head (coalesced 16-byte loads into registers, mma.sync m16n8k32 e4m3) fused top-k "
-      "with temperature/top-p sampling; comparator: BF16 head GEMV";
+      "top-k softmax routing in every CTA, split-K over the intermediate: 16-row slices of MXFP4 "
+      "E2M1/E8M0-32 gate/up + SiLU + down per work item, one bulk copy per item into a 3-stage ring, "
+      "E2M1->E5M2 by bit moves into mma.sync m16n8k32 e5m2 x e4m3 with per-block activation scales, "
+      "one grid barrier, fixed-order combine); "
+      "lm-head: online-FP8 E4M3 per-row-scale GEMV over the fragment-tiled head (warp-specialised: bulk-copy "
+      "ring, two mma.sync m16n8k32 e4m3 consumer groups, counter-scheduled tail tiles) fused top-k "
+      "with temperature/top-p sampling; kernels chained by programmatic dependent launch; "
+      "comparator: BF16 head GEMV";
   std::snprintf(buf, n, "%s", desc);
   return std::strlen(desc) < n ? MOE_OK : MOE_ERR_INVALID_ARG;
 }
