@@ -116,26 +116,30 @@ typedef struct {
 /* An expert bank re-laid out for moe_decode (moe_pack_experts): the same
  * MXFP4 bytes, grouped by the kernel's work items.  An item (e, j) is 16 rows
  * of expert e's intermediate dimension: gate and up rows 16j .. 16j+15 and
- * down columns 16j .. 16j+15.
- *   units   [count][inter/16][25 * hidden bytes]: item (e, j)'s bytes, one
- *           contiguous run in the order of the kernel's MMA fragments:
- *     A (hidden/32 blocks x 512 B): for K block b and lane l = 4g + t
- *       (g = l >> 2, t = l & 3), 16 bytes = the 4-byte words t of block b of
- *       gate row 16j+g, up row 16j+g, gate row 16j+8+g and up row 16j+8+g
- *       (word t of a block holds elements 32b + 8t .. 32b + 8t + 7);
- *     B (hidden/32 x 32 B): for block b and g, the E8M0 scales of block b of
- *       those four rows, in the same order;
+ * down columns 16j .. 16j+15.  The item's 32 gate/up rows (gate 16j ..
+ * 16j+15, then up 16j .. 16j+15) enter the tensor core as a 128-row operand:
+ * row 32s + R is row R over K segment s (elements s*Ks .. s*Ks + Ks - 1, with
+ * Ks = 64 T and T = ceil(hidden / 256) K tiles per segment):
+ *   units   [count][inter/16][unit]: item (e, j)'s bytes, one contiguous run
+ *           of unit = 4096 T + 256 T + 8 * hidden bytes (25 * hidden when
+ *           hidden is a multiple of 256):
+ *     A (T tiles x 4096 B): gate/up data as the A operand of a
+ *       block-scaled tensor-core MMA (canonical K-major layout, no swizzle):
+ *       half c (2048 B) of tile t holds, at 16 r, the 16 bytes of operand
+ *       row r = 32s + R: elements s*Ks + 64t + 32c .. +31 of row R, packed
+ *       E2M1 with element 2i in the low nibble of byte i; zero past hidden;
+ *     B (T x 256 B): byte 256t + 8R + 2s + c = the E8M0 scale of block
+ *       2Ts + 2t + c of row R (0 past hidden);
  *     C (hidden/32 groups x 256 B): for 32-row group G and lane l = 4g + t,
  *       8 bytes = 2 bytes (columns 16j + 4t .. 16j + 4t + 3) of each of down
- *       rows 32G + g, 32G + 8 + g, 32G + 16 + g and 32G + 24 + g;
+ *       rows 32G + g, 32G + 8 + g, 32G + 16 + g and 32G + 24 + g, with the bits
+ *       of each byte's two E2M1 codes re-placed: element 2j's sign, e1, e0, m
+ *       go to bits 7, 3, 2, 1 and element 2j+1's to bits 0, 6, 5, 4;
  *   dscales [count][inter/32][hidden]: the down scales of each 32-column
  *           pair p (shared by items 2p and 2p+1); byte 32G + 4g + r is the
  *           scale of down row 32G + 8r + g, block p.
- * Within every data byte the bits of its two E2M1 codes are re-placed:
- * element 2j's sign, e1, e0, m go to bits 7, 3, 2, 1 and element 2j+1's to
- * bits 0, 6, 5, 4 (scale bytes are unchanged).  fmt must be
- * MOE_FMT_MXFP4_MOE_PACKED.  The pages have no counterpart for this layout;
- * it moves bits, never changes a value.                                      */
+ * fmt must be MOE_FMT_MXFP4_MOE_PACKED.  The pages have no counterpart for
+ * this layout; it moves bytes and bits, never changes a value.              */
 typedef struct {
     int32_t fmt;
     int32_t count;
@@ -225,7 +229,7 @@ MOE_API size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts
  *   topk_w      [M][top_k] fp32 or NULL:  renormalised softmax weights
  *   workspace   device buffer of at least moe_workspace_bytes(...) bytes,
  *               zeroed once (moe_workspace_reset) before its first use.
- * Supported: H and I multiples of 32, 32 <= H <= 4096, 32 <= I <= 65536,
+ * Supported: H and I multiples of 32, 32 <= H <= 3840, 32 <= I <= 65536,
  * E <= 1024, 1 <= top_k <= 8 and top_k <= E.  The call is one cooperative
  * launch (one CTA per SM, all resident).  Each distinct routed expert is
  * streamed once per call, however many of the M tokens chose it.  The

@@ -272,9 +272,9 @@ moe_status moe_query_path(char* buf, size_t n) {
   const char* desc =
       "sm_100a; moe: one cooperative persistent kernel (router fp32 GEMV with epoch-tagged logits, "
       "top-k softmax routing in every CTA, split-K over the intermediate: 16-row slices of MXFP4 "
-      "E2M1/E8M0-32 gate/up + SiLU + down per work item, one bulk copy per item into a 3-stage ring, "
-      "E2M1->E5M2 by bit moves into mma.sync m16n8k32 e5m2 x e4m3 with per-block activation scales, "
-      "one grid barrier, fixed-order combine); "
+      "E2M1/E8M0-32 gate/up + SiLU + down per work item, one bulk copy per item into a stage ring, "
+      "gate/up as tcgen05.mma kind::mxf4 block-scaled (TMEM accumulator, activations as 8 E2M1 parts), "
+      "down as mma.sync f16 on E2M1 placed as E5M2, one grid barrier, fixed-order combine); "
       "lm-head: online-FP8 E4M3 per-row-scale GEMV over the fragment-tiled head (warp-specialised: bulk-copy "
       "ring, two mma.sync m16n8k32 e4m3 consumer groups, counter-scheduled tail tiles) fused top-k "
       "with temperature/top-p sampling; kernels chained by programmatic dependent launch; "

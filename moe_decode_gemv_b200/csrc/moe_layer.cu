@@ -36,21 +36,26 @@
 //    them in a fixed order (no float atomics: the result is the same on
 //    every run).
 //
-// Arithmetic: mma.sync m16n8k32 E5M2 (weights) x E4M3 (activations) -> fp32.
-// The packed nibbles become E5M2 codes of the E2M1 values times 2^-14 by one
-// mask (even elements) or two shifts (odd ones).  Each 32-element block's MMA
-// result is scaled by the weights' E8M0 scale and the activation block's own
-// power of two before it joins an fp32 sum.
-//  * x: per token and 32-element block, scaled so that the block's largest
-//    magnitude lies in [2^7, 2^8), then carried by two E4M3 parts (exact for
-//    bf16 values down to 2^-10 of the block's largest) in two columns of the
-//    MMA: column n = part n & 1 of token n >> 1.
+// Arithmetic.
+//  * gate/up on the fifth-generation tensor cores: one block-scaled FP4 MMA
+//    (tcgen05.mma kind::mxf4, E8M0 scale per 32 elements, fp32 accumulator in
+//    TMEM) per 64-element K tile, issued by one thread.  A = the item's 32
+//    gate/up rows as stored (E2M1, with the bank's own E8M0 scales), cut
+//    into four K segments stacked as 128 operand rows, so that every row the
+//    tensor core reads is a weight row; B = the tokens, each as eight E2M1
+//    base-4 digits per 32-element block and K segment; only the diagonal
+//    (segment s of A with segment s of B) of the product is read.  The
+//    digits carry a bf16 value exactly when it is within 2^-8 of its block's
+//    largest, and to within 2^-16 of the largest below.  The tensor core
+//    applies both scales, so no instruction decodes a weight; an MMA takes
+//    about 75 cycles, a fifth of the time the item's bytes take to arrive.
 //  * h: per token and item (16 values), scaled by a power of two that puts
 //    the largest magnitude in [2^14, 2^15) and carried by two f16 parts (about
 //    22 significant bits) into mma.sync m16n8k16 f16 x f16 -> fp32, whose K of
-//    16 is exactly the item's slice.  The weights' E5M2 bytes are the top
-//    bytes of f16 values (one byte permute each pair); column n of B = part
-//    n & 1 of token n >> 1, so one MMA covers 16 output rows of all tokens.
+//    16 is exactly the item's slice.  The down weights' E5M2 bytes (E2M1
+//    codes placed by the bank's bit layout) are the top bytes of f16 values;
+//    column n of B = part n & 1 of token n >> 1, so one MMA covers 16 output
+//    rows of all tokens.
 #include <cuda_runtime.h>
 
 #include <cfloat>
@@ -59,29 +64,43 @@
 #include "device_cache.h"
 #include "moe.h"
 #include "pack.h"
+#include "tcgen05.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kMaxBlocksPerWarp = 8;  // H <= 8 * 16 * 32 = 4096
+constexpr int kMaxBlocksPerWarp = 8;  // down: 32-row groups per warp, H <= 8 * 16 * 32 = 4096
+constexpr int kMaxH = 3840;           // a multiple of 256: the K segments' padded blocks stay within kMaxBlocks
+constexpr int kMaxBlocks = kMaxH / 32;
+constexpr int kParts = 8;             // E2M1 digits per activation value
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemD = 0;        // the gate/up accumulator: 128 lanes x up to 128 columns
+constexpr uint32_t kTmemSfa = 128;    // the item's weight scales: 4 columns per K tile
+constexpr int16_t kZeroBlock = -32768;
 constexpr int kMaxStages = 4;
 constexpr int kMaxSlots = 4 * 8 + 1;
 constexpr int kRouterChunk = 8;        // float4 router loads in flight per lane
 constexpr int kMaxE = 1024;
 constexpr uint32_t kFull = 0xffffffffu;
 
+// Token columns of the gate/up MMA's B operand per K segment: 8 digits of
+// each of mp tokens, mp = M rounded up to 1, 2 or 4 (N = 32 mp).
+__host__ __device__ constexpr int padded_tokens(int M) { return M <= 1 ? 1 : (M == 2 ? 2 : 4); }
+
 struct Geo {
-  int H, I, nb, n_sl, n_pairs, a_bytes, b_bytes, unit_bytes, stage_bytes;
-  __host__ __device__ Geo(int H_, int I_) : H(H_), I(I_) {
+  int H, I, nb, n_sl, n_pairs, kt, a_bytes, b_bytes, unit_bytes, stage_bytes, xparts_bytes;
+  __host__ __device__ Geo(int H_, int I_, int M) : H(H_), I(I_) {
     nb = H / 32;
     n_sl = I / kSliceRows;
     n_pairs = I / 32;
+    kt = slice_ktiles(H);
     a_bytes = slice_a_bytes(H);
     b_bytes = slice_b_bytes(H);
     unit_bytes = slice_unit_bytes(H);
     stage_bytes = (unit_bytes + H + 127) / 128 * 128;  // the unit, then its pair's down scales
+    xparts_bytes = kt * 1024 * padded_tokens(M);       // the activation digits: 32 mp rows x 64 T elements, E2M1
   }
 };
 
@@ -90,8 +109,12 @@ constexpr int kCandCap = 256;  // routing candidates per token: at most top_k la
 struct Ctl {
   uint64_t full[kMaxStages];                 // one phase per item copied into the stage
   uint64_t xbar;                             // the tokens' copy into shared memory
+  uint64_t mma_bar;                          // one phase per item's gate/up MMAs
+  uint32_t tmem;                             // TMEM base address
   float router_part[kWarps][4];
-  int32_t sigma_x[4][kMaxBlocksPerWarp * kWarps];
+  int16_t ex[4][kMaxBlocks + 1];             // per token and block: floor(log2) of the largest magnitude, or kZeroBlock
+  int16_t tshift[kMaxBlocks + 1];            // per block: powers of two moved from the weights' scales to the digits'
+  float gu[4][4][32];                        // gate/up of one item: [K segment][token][row R]
   uint16_t cand[4][kCandCap];                // routing: candidate experts of each token
   int32_t ids[4][8];
   float topv[4][8];
@@ -103,15 +126,14 @@ struct Ctl {
   float hfw[4];
   int nslots;
   int poison;
+  int shifted;  // some block's t is not 0
 };
 constexpr int kCtlBytes = (int)((sizeof(Ctl) + 127) / 128 * 128);
-// The scratch area holds, one after the other: the tokens (bf16, while the
-// router and the activation fragments read them), the M x E router logits
-// (while routing), each item's gate/up partial sums (after).
+// The scratch area holds the tokens (bf16, while the router and the
+// activation parts read them), then the M x E router logits (while routing).
 __host__ __device__ constexpr int scratch_bytes(int H) {
-  const int xb = 4 * H * 2, lb = 4 * kMaxE * 4, rb = kWarps * 32 * 16;
-  const int m = xb > lb ? (xb > rb ? xb : rb) : (lb > rb ? lb : rb);
-  return (m + 127) / 128 * 128;
+  const int xb = 4 * H * 2, lb = 4 * kMaxE * 4;
+  return ((xb > lb ? xb : lb) + 127) / 128 * 128;
 }
 
 struct LayerArgs {
@@ -172,6 +194,37 @@ __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t
 __device__ __forceinline__ float scale_pow2(float v, int s) {
   return s > 126 ? v * exp2i(126) * exp2i(s - 126) : v * exp2i(s);
 }
+// v * 2^k for |k| <= 378: exact whenever the result is a normal number.
+__device__ __forceinline__ float mul_pow2(float v, int k) {
+  if (k > 126) {
+    v *= exp2i(126);
+    k -= 126;
+    if (k > 126) {
+      v *= exp2i(126);
+      k -= 126;
+    }
+  } else if (k < -126) {
+    v *= exp2i(-126);
+    k += 126;
+    if (k < -126) {
+      v *= exp2i(-126);
+      k += 126;
+    }
+  }
+  return v * exp2i(k);
+}
+// floor(log2(a)) of a positive finite float (subnormals included).
+__device__ __forceinline__ int floor_log2(float a) {
+  const uint32_t b = __float_as_uint(a);
+  const int e = (int)((b >> 23) & 0xffu);
+  return e ? e - 127 : (31 - __clz(b & 0x7fffffu)) - 149;
+}
+// The value of an E2M1 code (bit 3 the sign): 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const uint32_t m = c & 7u;
+  const float v = m >= 2u ? (float)(2u + (m & 1u)) * exp2i((int)(m >> 1) - 2) : 0.5f * (float)m;
+  return (c & 8u) ? -v : v;
+}
 
 // ---- routing: the best 8 of up to 1,024 logits across warps ----
 // (value, expert) pairs under `better`: larger value first, lower id on ties.
@@ -202,8 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   Ctl& C = *reinterpret_cast<Ctl*>(smem);
   uint8_t* scratch = smem + kCtlBytes;
-  const Geo geo(a.H, a.I);
-  uint8_t* stages = scratch + scratch_bytes(a.H);
+  const Geo geo(a.H, a.I, a.M);
+  uint8_t* xparts = scratch + scratch_bytes(a.H);   // the gate/up B operand: [K tile][half][32 mp rows][16 B]
+  uint8_t* stages = xparts + geo.xparts_bytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
   const int G = gridDim.x, c = blockIdx.x;
@@ -238,10 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) mbar_init(&C.full[s], 1);
     mbar_init(&C.xbar, 1);
+    mbar_init(&C.mma_bar, 1);
     fence_mbar_init();
     C.poison = 0;
+    C.shifted = 0;
     top_up(n_pre);  // the shared expert's items: weights, which no kernel writes
   }
+  if (warp == 0) tmem_alloc(&C.tmem, kTmemCols);  // one CTA per SM: all of the SM's TMEM
 
   // ---- router loads of this CTA's rows: the first chunk goes out now ----
   const int e_begin = (int)((int64_t)E * c / G), e_end = (int)((int64_t)E * (c + 1) / G);
@@ -269,7 +326,12 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   int r_row, r_f0, r_f1;
   router_slot(0, r_row, r_f0, r_f1);
   if (R > 0) router_load(r_row, r_f0 + lane, r_f1);
-  __syncthreads();  // the barriers are initialised
+  tc_fence_before_sync();
+  __syncthreads();  // the barriers are initialised, TMEM is allocated
+  tc_fence_after_sync();
+  const uint32_t tm = C.tmem;
+  const int T = geo.kt;
+  const uint32_t tm_sfb = kTmemSfa + 4u * (uint32_t)T;  // the activation parts' scales: 4 columns per K tile
   // Everything below may read what the previous kernel on the stream wrote
   // (the tokens, the workspace): wait for it.  The weight copies and loads
   // above are already on their way.
@@ -335,9 +397,21 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
     __syncthreads();
   }
 
-  // ---- x: per (token, block) power-of-two scale, then this lane's B fragments ----
-  for (int t = threadIdx.x; t < M * nb; t += kThreads) {
-    const int m = t / nb, b = t - m * nb;
+  // ---- x: eight E2M1 digits per token and 32-element block ----
+  // The gate/up MMA's B operand has N = 32 mp rows: row n = 8 mp s + 8 m + p
+  // holds digit p of token m over K segment s (elements 64 T s ..), K-major
+  // like the weights.  For a block whose largest magnitude lies in [2^E,
+  // 2^(E+1)), each value v is rounded to N = round(|v| 2^(15 - E)), an
+  // integer below 2^16 (exact when v is within 2^-8 of the block's largest,
+  // else off by at most 2^(E-16)), and written in base 4: digit p = bits
+  // 14 - 2p, 15 - 2p of N, stored as the E2M1 code of d / 2 (codes 0..3 are
+  // 0, 0.5, 1, 1.5) with v's sign, scale 2^(E - 2p).  The tensor core
+  // applies the scales, so the eight digit columns of a token sum to N
+  // 2^(E-15) x the weights.  The digits' E8M0 scales go to TMEM.
+  const int mp = padded_tokens(M);
+  // 1. E per (token, block)
+  for (int u = threadIdx.x; u < M * nb; u += kThreads) {
+    const int m = u / nb, b = u - m * nb;
     const uint4* p = reinterpret_cast<const uint4*>(xs + m * H + 32 * b);
     float am = 0.f;
 #pragma unroll
@@ -348,42 +422,109 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
       am = fmaxf(am, fmaxf(fmaxf(bf16_bits_to_f32(v.z & 0x7fffu), bf16_bits_to_f32((v.z >> 16) & 0x7fffu)),
                            fmaxf(bf16_bits_to_f32(v.w & 0x7fffu), bf16_bits_to_f32((v.w >> 16) & 0x7fffu))));
     }
-    C.sigma_x[m][b] = pow2_sigma(am);
+    C.ex[m][b] = am > 0.f ? (int16_t)floor_log2(am) : kZeroBlock;
   }
   __syncthreads();
-  // Lane (g, t) of warp w, block b = w + 16 jb: column g of B = part g & 1 of
-  // token g >> 1; its even elements 32b + 8t + 2i fill b0, the odd ones b1
-  // (the order of the weight nibbles).  fx undoes the scale of token t's block
-  // and the E5M2 weights' 2^-14 on the D side (columns 2t, 2t+1 = token t).
-  uint32_t bx[kB][2];
-  float fx[kB];
-  {
-    const int mB = g >> 1, part = g & 1;
-#pragma unroll
-    for (int jb = 0; jb < kB; ++jb) {
-      const int b = warp + kWarps * jb;
-      uint32_t b0 = 0u, b1 = 0u;
-      if (b < nb && mB < M) {
-        const int sg = C.sigma_x[mB][b];
-        const uint4 q = *reinterpret_cast<const uint4*>(xs + mB * H + 32 * b + 8 * tq);
-        auto xsc = [&](uint32_t bits) { return scale_pow2(bf16_bits_to_f32(bits), sg); };
-        uint32_t pe[2], po[2];
-        split_e4m3x4<2>(xsc(q.x & 0xffffu), xsc(q.y & 0xffffu), xsc(q.z & 0xffffu), xsc(q.w & 0xffffu), pe);
-        split_e4m3x4<2>(xsc(q.x >> 16), xsc(q.y >> 16), xsc(q.z >> 16), xsc(q.w >> 16), po);
-        b0 = part ? pe[1] : pe[0];
-        b1 = part ? po[1] : po[0];
+  // 2. per block, t: the product of a weight scale 2^(c - 127) and a digit
+  // scale 2^(E - 2p) is taken as 2^(c - t - 127) x 2^(E - 2p + t), with t
+  // chosen so that every token's digit codes E - 2p + t + 127 lie in [0,
+  // 254] (0 unless the block is below about 2^-113 or above 2^127).
+  for (int b = threadIdx.x; b < 8 * T; b += kThreads) {
+    int lo = -100000, hi = 100000;
+    for (int m = 0; m < M; ++m) {
+      const int eb = b < nb ? C.ex[m][b] : kZeroBlock;
+      if (eb != kZeroBlock) {
+        lo = max(lo, -127 - (eb - 2 * (kParts - 1)));
+        hi = min(hi, 127 - eb);
       }
-      bx[jb][0] = b0;
-      bx[jb][1] = b1;
-      fx[jb] = (b < nb && tq < M) ? exp2i(14 - C.sigma_x[tq][b]) : 0.f;
     }
+    int t = 0;
+    if (t < lo) t = lo;
+    if (t > hi) t = hi;  // the leading digits win if no shift fits all
+    C.tshift[b] = (int16_t)t;
+    if (t != 0) C.shifted = 1;
   }
+  // 3. the digits: one thread per (token, block, 8 elements, 4 digits),
+  // four 4-byte words; zero for padding
+  const int lmp = mp == 1 ? 0 : (mp == 2 ? 1 : 2);
+  for (int u = threadIdx.x; u < mp * 64 * T; u += kThreads) {
+    const int ph = u & 1, u8 = u >> 1;
+    const int m = u8 / (32 * T), rest = u8 - m * (32 * T), b = rest >> 2, q = rest & 3;
+    const int sg = b / (2 * T), lb = b - sg * (2 * T), t = lb >> 1, hf = lb & 1;
+    uint8_t* dst = xparts + (size_t)t * (1024 * mp) + hf * (512 * mp) + (sg * mp + m) * 128 + 64 * ph + 4 * q;
+    const int eb = (m < M && b < nb) ? C.ex[m][b] : kZeroBlock;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (eb != kZeroBlock) {
+      const uint4 xv = *reinterpret_cast<const uint4*>(xs + m * H + 32 * b + 8 * q);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+      uint32_t pr[4] = {0u, 0u, 0u, 0u}, sgn = 0u;  // pr[i] = N_i | N_(i+4) << 16
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t bits = (xw[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+        const uint32_t n = __float2uint_rn(mul_pow2(bf16_bits_to_f32(bits & 0x7fffu), 15 - eb));
+        pr[i & 3] |= n << (16 * (i >> 2));
+        sgn |= (bits >> 15) << (4 * i + 3);
+      }
+      const int sh0 = 14 - 8 * ph;  // digit 4 ph: bits sh0, sh0 + 1
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        uint32_t v = sgn;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v |= ((pr[i] >> (sh0 - 2 * p)) & 0x00030003u) << (4 * i);
+        w[p] = v;
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) *reinterpret_cast<uint32_t*>(dst + 16 * p) = w[p];
+  }
+  fence_proxy_async_smem();  // the tensor core reads these through the async proxy
+  __syncthreads();           // every block's t is written; the tokens are no longer read
+  const bool shifted = C.shifted != 0;
+  // 4. the digits' scales: K tile t, operand row n = 32 q + lane in column q
+  // of the tile's group, in every lane quarter; bytes 0, 1 = the two halves;
+  // 127 where the digit is zero.  All threads fill a table [T][4][32] in the
+  // scratch area, then warps 0..3 copy it into their lane quarters.
+  uint32_t* sfbt = reinterpret_cast<uint32_t*>(scratch);
+  for (int e = threadIdx.x; e < 128 * T; e += kThreads) {
+    const int t = e >> 7, q = (e >> 5) & 3, n = e & 127;
+    const int sg = n >> (3 + lmp), m = (n >> 3) & (mp - 1), p = n & 7;
+    uint32_t w = 0u;
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int b = 2 * T * sg + 2 * t + hf;
+      const int eb = (q < mp && m < M && b < nb) ? C.ex[m][b] : kZeroBlock;
+      int code = 127;
+      if (eb != kZeroBlock) code = min(max(eb - 2 * p + C.tshift[b] + 127, 0), 254);
+      w |= (uint32_t)code << (8 * hf);
+    }
+    sfbt[e] = w;
+  }
+  __syncthreads();
+  if (warp < 4) {
+    for (int t0 = 0; t0 < T; t0 += 8) {
+      uint32_t v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = t0 + (i >> 2) < T ? sfbt[(t0 * 4 + i) * 32 + lane] : 0u;
+      const uint32_t ta = tm + ((uint32_t)(32 * warp) << 16) + tm_sfb + 4u * t0;
+      if (T - t0 >= 8) {
+        tmem_st_x32(ta, v);
+      } else {
+#pragma unroll
+        for (int tt = 0; tt < 7; ++tt)
+          if (tt < T - t0) tmem_st_x4(ta + 4u * tt, v[4 * tt], v[4 * tt + 1], v[4 * tt + 2], v[4 * tt + 3]);
+      }
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before_sync();
   __syncthreads();  // the tokens' shared memory is free from here on
+  tc_fence_after_sync();
 
   // ---- one work item: gate/up over H, SiLU gate, down over its 16 columns ----
   float yacc[kB][4];
 #pragma unroll
   for (int jg = 0; jg < kB; ++jg) yacc[jg][0] = yacc[jg][1] = yacc[jg][2] = yacc[jg][3] = 0.f;
+  int n_done = 0;  // items computed: the phase of the MMA barrier
   auto compute = [&](int j) {
     const int s = j % NS;
     const int slot = (c + G * j) / n_sl;
@@ -391,56 +532,101 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
     const uint8_t* st = stages + (size_t)s * geo.stage_bytes;
     const uint32_t all = (1u << M) - 1u;
     const uint32_t mask = slot == 0 ? all : C.slot_mask[slot];
-    // gate/up: this warp's K blocks, two 16-row tiles (gate rows g, up rows g
-    // of the slice's first and second half)
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    // gate/up on the tensor core.  The item's weight scales go to TMEM
+    // (warps 0..3, each its lane quarter; operand row 32 s + R in lane R,
+    // column s of the K tile's group), shifted by the blocks' t; then one
+    // thread issues one block-scaled MMA per K tile: D[32 s + R][n] = gate/up
+    // row R over K segment s times B row n, summed over the segment's tiles.
+    // Only the 8 mp columns of segment s are wanted from lanes 32 s ..
+    {
+      // warp w writes lane quarter w % 4 for K tiles w / 4, w / 4 + 4, ...;
+      // both tiles' values are loaded before either store (a TMEM store
+      // between shared-memory loads costs hundreds of cycles)
+      const uint2* sb = reinterpret_cast<const uint2*>(st + geo.a_bytes);  // [T][32 rows][4 segments][2 halves]
+      const uint32_t tq = tm + ((uint32_t)(32 * (warp & 3)) << 16) + kTmemSfa;
+      for (int t0 = warp >> 2; t0 < T; t0 += 8) {
+        const bool two = t0 + 4 < T;
+        const uint2 c0 = sb[t0 * 32 + lane];
+        const uint2 c1 = two ? sb[(t0 + 4) * 32 + lane] : make_uint2(0u, 0u);
+        uint32_t v[8] = {c0.x & 0xffffu, c0.x >> 16, c0.y & 0xffffu, c0.y >> 16,
+                         c1.x & 0xffffu, c1.x >> 16, c1.y & 0xffffu, c1.y >> 16};
+        if (shifted) {
 #pragma unroll
-    for (int jb = 0; jb < kB; ++jb) {
-      const int b = warp + kWarps * jb;
-      if (b < nb) {
-        const uint4 q = *reinterpret_cast<const uint4*>(st + (b * 32 + lane) * 16);
-        const uint32_t sc = *reinterpret_cast<const uint32_t*>(st + geo.a_bytes + (b * 8 + g) * 4);
-        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_e5m2_e4m3(d0, packed_even_to_e5m2x4(q.x), packed_even_to_e5m2x4(q.y), packed_odd_to_e5m2x4(q.x),
-                      packed_odd_to_e5m2x4(q.y), bx[jb][0], bx[jb][1]);
-        mma_e5m2_e4m3(d1, packed_even_to_e5m2x4(q.z), packed_even_to_e5m2x4(q.w), packed_odd_to_e5m2x4(q.z),
-                      packed_odd_to_e5m2x4(q.w), bx[jb][0], bx[jb][1]);
-        const float f = fx[jb];
-        acc[0] = fmaf(d0[0] + d0[1], e8m0_to_f32_fast(sc & 0xffu) * f, acc[0]);          // gate row g, token t
-        acc[1] = fmaf(d0[2] + d0[3], e8m0_to_f32_fast((sc >> 8) & 0xffu) * f, acc[1]);   // up row g
-        acc[2] = fmaf(d1[0] + d1[1], e8m0_to_f32_fast((sc >> 16) & 0xffu) * f, acc[2]);  // gate row 8 + g
-        acc[3] = fmaf(d1[2] + d1[3], e8m0_to_f32_fast(sc >> 24) * f, acc[3]);            // up row 8 + g
+          for (int i = 0; i < 8; ++i) {
+            const int t = t0 + 4 * (i >> 2), sg = i & 3;
+            uint32_t w = 0u;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const int cc = (int)((v[i] >> (8 * hf)) & 0xffu);
+              const int cs = (cc == 255 || t >= T) ? cc : min(max(cc - C.tshift[2 * T * sg + 2 * t + hf], 0), 254);
+              w |= (uint32_t)cs << (8 * hf);
+            }
+            v[i] = w;
+          }
+        }
+        tmem_st_x4(tq + 4u * t0, v[0], v[1], v[2], v[3]);
+        if (two) tmem_st_x4(tq + 4u * (t0 + 4), v[4], v[5], v[6], v[7]);
       }
+      tmem_wait_st();
     }
-    float4* red = reinterpret_cast<float4*>(scratch);
-    red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    tc_fence_before_sync();
     __syncthreads();
-    // h for the slice's 16 rows and each token, in fp32; then its f16 parts
-    if (threadIdx.x < 64) {
-      const int m = threadIdx.x >> 4, r = threadIdx.x & 15;
-      const float2* rp = reinterpret_cast<const float2*>(red + (r & 7) * 4 + m) + (r >> 3);
-      float gs = 0.f, us = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float2 p = rp[w * 64];
-        gs += p.x;
-        us += p.y;
-      }
-      const bool live = m < M && ((mask >> m) & 1u);
-      const float h = live ? gs / (1.0f + expf(-gs)) * us : 0.f;
-      float am = fabsf(h);
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(kFull, am, o));
-      // sigma such that the largest |h| of the slice lies in [2^14, 2^15)
-      const int sig = min(pow2_sigma(am) + 7, 140);
-      const float v = scale_pow2(h, sig);
-      const __half hi = __float2half_rn(v);
-      const __half lo = __float2half_rn(v - __half2float(hi));
-      const int pos = ((r & 1) << 1) | ((r >> 1) & 1);  // element r = 4t + i sits at [t][0, 2, 1, 3 -> 0..3]
-      C.hp[m][0][r >> 2][pos] = __half_as_ushort(hi);
-      C.hp[m][1][r >> 2][pos] = __half_as_ushort(lo);
-      if (r == 0) C.hfw[m] = live ? (slot == 0 ? 1.0f : C.slot_w[slot][m]) * exp2i(14 - sig) : 0.f;
+    if (threadIdx.x == 0) {
+      tc_fence_after_sync();
+      const uint32_t a0 = smem_addr(st), b0 = smem_addr(xparts);
+      const uint32_t bt = 1024u * (uint32_t)mp, idesc = mxf4_idesc(32u * (uint32_t)mp);
+      for (int t = 0; t < T; ++t)
+        mma_mxf4(tm + kTmemD, umma_desc_kmajor(a0 + 4096u * t, 2048u, 128u),
+                 umma_desc_kmajor(b0 + bt * t, bt >> 1, 128u), idesc, tm + kTmemSfa + 4u * t,
+                 tm + tm_sfb + 4u * t, t > 0);
+      mma_commit(&C.mma_bar);
     }
+    // h from the accumulator: warp s < 4 adds the digit columns of segment s
+    // for each token (lane R = gate/up row R); warp m < M then sums the four
+    // segments of token m, h = silu(gate) * up, the slice's power of two and
+    // its two f16 parts
+    if (warp < 4) {
+      if (!poisoned() && !mbar_wait(&C.mma_bar, (uint32_t)(n_done & 1))) fail();
+      tc_fence_after_sync();
+      uint32_t d[32];
+      const uint32_t ta = tm + ((uint32_t)(32 * warp) << 16) + kTmemD + 8u * (uint32_t)(mp * warp);
+      if (mp == 1) tmem_ld_x8(ta, d);
+      else if (mp == 2) tmem_ld_x16(ta, d);
+      else tmem_ld_x32(ta, d);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        if (m < mp) {
+          float gv = 0.f;
+#pragma unroll
+          for (int p = 0; p < kParts; ++p) gv += __uint_as_float(d[8 * m + p]);
+          C.gu[warp][m][lane] = gv;
+        }
+      }
+      tc_fence_before_sync();
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // warps 0..3: the segments' sums are in shared memory
+      if (warp < M) {
+        const int m = warp, r = lane & 15;
+        const float gv = (C.gu[0][m][lane] + C.gu[1][m][lane]) + (C.gu[2][m][lane] + C.gu[3][m][lane]);
+        const float uv = __shfl_down_sync(kFull, gv, 16);
+        const bool live = lane < 16 && ((mask >> m) & 1u);
+        const float h = live ? gv / (1.0f + expf(-gv)) * uv : 0.f;
+        float am = fabsf(h);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(kFull, am, o));
+        // sigma such that the largest |h| of the slice lies in [2^14, 2^15)
+        const int sig = min(pow2_sigma(am) + 7, 140);
+        const float v = scale_pow2(h, sig);
+        const __half hi = __float2half_rn(v);
+        const __half lo = __float2half_rn(v - __half2float(hi));
+        const int pos = ((r & 1) << 1) | ((r >> 1) & 1);  // element r = 4t + i sits at [t][0, 2, 1, 3 -> 0..3]
+        if (lane < 16) {
+          C.hp[m][0][r >> 2][pos] = __half_as_ushort(hi);
+          C.hp[m][1][r >> 2][pos] = __half_as_ushort(lo);
+        }
+        if (lane == 0) C.hfw[m] = live ? (slot == 0 ? 1.0f : C.slot_w[slot][m]) * exp2i(14 - sig) : 0.f;
+      }
+    }
+    ++n_done;
     __syncthreads();
     // down: this warp's 32-row output groups, two MMAs (16 rows each) per group
     // for all tokens; lane (g, t) ends with rows 32G + 8r + g of token t
@@ -539,15 +725,23 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
         bound.v = __shfl_sync(kFull, b.v, __ffs(hit) - 1);
         bound.i = __shfl_sync(kFull, b.i, __ffs(hit) - 1);
       }
+      // compaction, eight ballots at a time (independent loads and votes,
+      // then the running count)
       int nc = 0;
-#pragma unroll 4
-      for (int e0 = 0; e0 < E; e0 += 32) {
-        const int e = e0 + lane;
-        const bool keep = e < E && !better(bound.v, bound.i, lm[e], e);
-        const uint32_t bal = __ballot_sync(kFull, keep);
-        const int pos = nc + __popc(bal & ((1u << lane) - 1u));
-        if (keep && pos < kCandCap) C.cand[m][pos] = (uint16_t)e;  // never more: k lanes' experts at most
-        nc += __popc(bal);
+      for (int e0 = 0; e0 < E; e0 += 256) {
+        uint32_t bal[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int e = e0 + 32 * u + lane;
+          bal[u] = __ballot_sync(kFull, e < E && !better(bound.v, bound.i, lm[e], e));
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int pos = nc + __popc(bal[u] & ((1u << lane) - 1u));
+          if (((bal[u] >> lane) & 1u) && pos < kCandCap)  // never more: k lanes' experts at most
+            C.cand[m][pos] = (uint16_t)(e0 + 32 * u + lane);
+          nc += __popc(bal[u]);
+        }
       }
       __syncwarp();
       nc = min(nc, kCandCap);
@@ -691,11 +885,14 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
       if (lane == 0) *reinterpret_cast<float4*>(&a.out[(size_t)m * H + row]) = s;
     }
   }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tm, kTmemCols);
 }
 
-int moe_stages(int H) {
-  const Geo geo(H, 32);
-  const int avail = kMaxDynamicSmem - kCtlBytes - scratch_bytes(H);
+int moe_stages(int H, int M) {
+  const Geo geo(H, 32, M);
+  const int avail = kMaxDynamicSmem - kCtlBytes - scratch_bytes(H) - geo.xparts_bytes;
   int n = avail / geo.stage_bytes;
   return n > kMaxStages ? kMaxStages : n;
 }
@@ -706,9 +903,10 @@ cudaError_t launch_layer_t(const LayerArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   if ((e = current_device_sms(&dev, &sms)) != cudaSuccess) return e;
-  const Geo geo(a.H, a.I);
+  const Geo geo(a.H, a.I, a.M);
   const int grid = sms < MoeWs::kMaxGrid ? sms : MoeWs::kMaxGrid;  // one CTA per SM, all resident
-  const size_t smem = (size_t)kCtlBytes + scratch_bytes(a.H) + (size_t)a.stages * geo.stage_bytes;
+  const size_t smem =
+      (size_t)kCtlBytes + scratch_bytes(a.H) + geo.xparts_bytes + (size_t)a.stages * geo.stage_bytes;
   e = launch_dependent(moe_layer_kernel<kB>, dim3(grid), dim3(kThreads), smem, st, true, a);
   return e;
 }
@@ -716,13 +914,13 @@ cudaError_t launch_layer_t(const LayerArgs& a, cudaStream_t st) {
 }  // namespace
 
 bool moe_layer_supported(int H, int I) {
-  return H >= 32 && H % 32 == 0 && H <= kMaxBlocksPerWarp * kWarps * 32 && I >= 32 && I % 32 == 0 &&
-         I <= 65536 && moe_stages(H) >= 1;
+  return H >= 32 && H % 32 == 0 && H <= kMaxH && I >= 32 && I % 32 == 0 &&
+         I <= 65536 && moe_stages(H, 4) >= 1;
 }
 
 cudaError_t launch_moe_layer(const MoeArgs& m, cudaStream_t st) {
   LayerArgs a{m.x, m.router_w, m.router_bias, m.bank, m.shared, m.M, m.top_k, m.E, m.H, m.I,
-              moe_stages(m.H), m.out, m.ids_out, m.w_out, m.ws};
+              moe_stages(m.H, m.M), m.out, m.ids_out, m.w_out, m.ws};
   const int need = (m.H / 32 + kWarps - 1) / kWarps;  // K blocks (= output groups) per warp
   if (need <= 1) return launch_layer_t<1>(a, st);
   if (need <= 2) return launch_layer_t<2>(a, st);

@@ -5,25 +5,33 @@
 // of the intermediate dimension: item (e, j) computes gate and up rows
 // 16j .. 16j+15 of expert e, h = silu(gate x) * (up x) for those rows, and
 // applies down columns 16j .. 16j+15 to h.  Each item's weight bytes are one
-// contiguous unit, already in the order of the kernel's MMA fragments:
+// contiguous unit, already in the order its matrix instructions read them.
+// The gate/up rows go to the tensor core as a 128-row operand: the item's 32
+// rows (gate 16j .. 16j+15, then up 16j .. 16j+15) times four K segments of
+// Ks = 64 T elements each, T = ceil(H / 256); row r = 32 s + R of the operand
+// is row R over elements s Ks .. s Ks + Ks - 1.
 //
-//   A  gate/up data, (H/32) blocks x 512 bytes: for K block b and lane
-//      l = 4g + t (g = l >> 2, t = l & 3), 16 bytes = the 4-byte words t of
-//      block b of gate row 16j+g, up row 16j+g, gate row 16j+8+g and up row
-//      16j+8+g (a word holds elements 32b + 8t .. 32b + 8t + 7);
-//   B  gate/up scales, (H/32) x 32 bytes: for block b and g, 4 bytes = the
-//      E8M0 scales of block b of those four rows, in the same order;
+//   A  gate/up data as the A operand of a block-scaled tensor-core MMA, in
+//      the canonical K-major layout without swizzle: T K tiles of 4096 bytes,
+//      each two halves of 2048 bytes; in half c of tile t, operand row r is
+//      the 16 bytes at 16 r (8-row core matrices 128 bytes apart), holding
+//      elements s Ks + 64t + 32c .. +31 of its gate/up row as packed E2M1
+//      (element 2i in the low nibble of byte i).  Elements past H are zero.
+//   B  gate/up scales, T x 256 bytes: for K tile t, row R, segment s and
+//      half c, byte 256t + 8R + 2s + c = the E8M0 scale of block 2T s + 2t + c
+//      of row R (0 past H).
 //   C  down data, (H/32) groups x 256 bytes: for 32-row group G and lane
 //      l = 4g + t, 8 bytes = 2 bytes (columns 16j + 4t .. 16j + 4t + 3) of each
-//      of down rows 32G + g, 32G + 8 + g, 32G + 16 + g, 32G + 24 + g.
+//      of down rows 32G + g, 32G + 8 + g, 32G + 16 + g, 32G + 24 + g, with
+//      the two E2M1 codes of each byte re-placed bit by bit (element 2j's
+//      sign|e1 e0 m at bits 7|3 2 1, element 2j+1's at 0|6 5 4) so that a
+//      mask gives the even elements of a word as E5M2 codes and two shifts
+//      the odd ones.
 //
 // The down scales are per 32 columns, so two items share them: they sit in a
 // second array, [E][I/32][H] bytes, where pair p's byte 32G + 4g + r is the
-// scale of down row 32G + 8r + g, block p.  Within every data byte
-// the two E2M1 codes are re-placed bit by bit (element 2j's sign|e1 e0 m at
-// bits 7|3 2 1, element 2j+1's at 0|6 5 4) so that a mask gives the even
-// elements of a word as E5M2 codes and two shifts the odd ones.  The layout
-// moves bytes and bits only; no value changes.
+// scale of down row 32G + 8r + g, block p.  The layout moves bytes and bits
+// only; no value changes.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -34,10 +42,14 @@ namespace moe {
 
 constexpr int kSliceRows = 16;  // intermediate rows per work item
 
-// Bytes of one item's unit (parts A, B, C): 25 H.
-__host__ __device__ constexpr int slice_unit_bytes(int H) { return (H / 32) * (512 + 32 + 256); }
-__host__ __device__ constexpr int slice_a_bytes(int H) { return (H / 32) * 512; }
-__host__ __device__ constexpr int slice_b_bytes(int H) { return (H / 32) * 32; }
+// K tiles of 64 elements per K segment (four segments cover H).
+__host__ __device__ constexpr int slice_ktiles(int H) { return (H + 255) / 256; }
+// Bytes of one item's parts A, B, C and of the whole unit (25 H when H is a
+// multiple of 256).
+__host__ __device__ constexpr int slice_a_bytes(int H) { return slice_ktiles(H) * 4096; }
+__host__ __device__ constexpr int slice_b_bytes(int H) { return slice_ktiles(H) * 256; }
+__host__ __device__ constexpr int slice_c_bytes(int H) { return (H / 32) * 256; }
+__host__ __device__ constexpr int slice_unit_bytes(int H) { return slice_a_bytes(H) + slice_b_bytes(H) + slice_c_bytes(H); }
 
 size_t packed_units_bytes(int64_t E, int H, int I);
 size_t packed_dscales_bytes(int64_t E, int H, int I);

@@ -23,7 +23,7 @@ __global__ void pack_units_kernel(const uint8_t* __restrict__ gate_d, const uint
                                   const uint8_t* __restrict__ down_d, int64_t E, int H, int I,
                                   uint8_t* __restrict__ out) {
   const int nb = H / 32, n_sl = I / kSliceRows;
-  const int ua = slice_a_bytes(H), ub = slice_b_bytes(H), unit = slice_unit_bytes(H);
+  const int ua = slice_a_bytes(H), ub = slice_b_bytes(H), unit = slice_unit_bytes(H), T = slice_ktiles(H);
   const int64_t total = E * n_sl * (int64_t)unit;
   const int64_t hb = H / 2, ib = I / 2;  // data bytes per gate/up row and per down row
   for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < total; o += (int64_t)gridDim.x * blockDim.x) {
@@ -33,18 +33,20 @@ __global__ void pack_units_kernel(const uint8_t* __restrict__ gate_d, const uint
     const int j = (int)(item - e * n_sl);
     uint32_t v;
     if (k < ua) {
-      // block b, lane l, word w of [gate g, up g, gate 8+g, up 8+g], byte bw
-      const int b = k / 512, l = (k % 512) / 16, w = (k % 16) / 4, bw = k % 4;
-      const int g = l >> 2, t = l & 3;
-      const int row = 16 * j + 8 * (w >> 1) + g;
-      const uint8_t* src = (w & 1) ? up_d : gate_d;
-      v = nibble_relayout(src[(e * I + row) * hb + 16 * b + 4 * t + bw]);
+      // tile t, half c, operand row r = 32 s + R, byte bi of its 16
+      const int t = k / 4096, c = (k % 4096) / 2048, r = (k % 2048) / 16, bi = k % 16;
+      const int s = r / 32, R = r % 32;  // R: 0..15 gate rows, 16..31 up rows
+      const int row = 16 * j + (R & 15);
+      const int k0 = s * 64 * T + 64 * t + 32 * c + 2 * bi;  // the byte's first element
+      const uint8_t* src = R < 16 ? gate_d : up_d;
+      v = k0 < H ? src[(e * I + row) * hb + k0 / 2] : 0u;
     } else if (k < ua + ub) {
       const int kk = k - ua;
-      const int b = kk / 32, g = (kk % 32) / 4, w = kk % 4;
-      const int row = 16 * j + 8 * (w >> 1) + g;
-      const uint8_t* src = (w & 1) ? up_s : gate_s;
-      v = src[(e * I + row) * nb + b];
+      const int t = kk / 256, R = (kk % 256) / 8, s = (kk % 8) / 2, c = kk % 2;
+      const int b = 2 * T * s + 2 * t + c;
+      const int row = 16 * j + (R & 15);
+      const uint8_t* src = R < 16 ? gate_s : up_s;
+      v = b < nb ? src[(e * I + row) * nb + b] : 0u;
     } else {
       // group G, lane l, row r of the four (32G + 8r + g), byte bw of its two
       const int kk = k - ua - ub;

@@ -56,7 +56,8 @@ def test_workspace_sizes(lib):
     assert lib.moe_workspace_bytes(1, 9, 512, 2560, 768) == 0          # top_k > 8
     assert lib.moe_workspace_bytes(1, 8, 512, 2561, 768) == 0          # H not a multiple of 32
     assert lib.moe_workspace_bytes(1, 8, 512, 2560, 80) == 0           # I not a multiple of 32
-    assert lib.moe_workspace_bytes(1, 8, 512, 4128, 768) == 0          # H above 4096
+    assert lib.moe_workspace_bytes(1, 8, 512, 3872, 768) == 0          # H above 3840 (TMEM columns)
+    assert lib.moe_workspace_bytes(1, 8, 512, 3840, 768) > 0
     assert lib.moe_workspace_bytes(1, 8, 1025, 2560, 768) == 0         # more than 1024 experts
     assert lib.moe_workspace_bytes(1, 8, 512, 96, 32) > 0              # the smallest odd sizes
     assert lib.lmhead_workspace_bytes(1, 29, 157184, 2560) > 0
