@@ -235,18 +235,21 @@ MOE_API size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts
  * streamed once per call, however many of the M tokens chose it.  The
  * output is the same on every call with the same inputs (a fixed summation
  * order on a given GPU).
- * Arithmetic: fp32 sums of exact products of the E2M1 weights with parts
- * of the activations.  x, per token and 32-element block scaled by a power
- * of two, is split into two E4M3 parts: exact for bf16 values down to 2^-10
- * of the block's largest magnitude, within 2^-17 of it below.  h, per token
- * and 16 values scaled likewise, is split into two f16 parts (about 22
- * significant bits).  Activations and h must stay below 2^120 in magnitude;
- * every smaller bf16 value, subnormals included, is carried as above.
- * E8M0 scales are decoded by one multiply into the fp32 exponent: code 0
- * contributes 0 instead of 2^-127 times its elements (below 2^-116 of any
- * product), and code 255 acts as +inf, so a non-finite block as
- * moe_quantize_mxfp4 writes it (scale 0xFF, zero elements) still turns the
- * rows that read it into NaN.                                                */
+ * Arithmetic: gate/up on the tensor core (block-scaled FP4 MMA, fp32
+ * accumulation): the E2M1 weights with their E8M0 scales times x written,
+ * per token and 32-element block, as eight E2M1 base-4 digits with power-of-
+ * two scales: exact for bf16 values within 2^-8 of the block's largest
+ * magnitude, rounded to within 2^-16 of it below.  Where a block's weight
+ * and activation scales together leave E8M0's range (activations below
+ * about 2^-113 or above 2^127), powers of two move between them, and a
+ * weight scale pushed out of range saturates.  h, per token and 16 values
+ * scaled by a power of two, is split into two f16 parts (about 22
+ * significant bits) for the down products.  Down E8M0 scales are decoded
+ * by one multiply into the fp32 exponent: code 0 contributes 0 instead of
+ * 2^-127 times its elements, and code 255 acts as +inf, so a non-finite
+ * block as moe_quantize_mxfp4 writes it (scale 0xFF, zero elements) still
+ * turns the rows that read it into NaN; a gate/up weight block with scale
+ * 0xFF makes its row NaN.                                                   */
 MOE_API moe_status moe_decode(const uint16_t* hidden_bf16, const float* router_w, const float* router_bias,
                       const moe_packed_bank* experts, const moe_packed_bank* shared,
                       int32_t M, int32_t top_k, float* out, int32_t* topk_ids, float* topk_w,
