@@ -757,8 +757,9 @@ def main():
                         "back_to_back_mean_us": m1["per_step_us"], "steps": args.steps,
                         "timing": "CUDA events at step boundaries on the launching stream; inputs larger than L2 "
                                   "(8 rotating layer copies + the 403 MB head per step)"},
-        "arithmetic": "fp32 accumulate; activations carried as two E4M3 parts per block (x) and two f16 parts "
-                      "per 16-value slice (h); weights MXFP4 (experts) and E4M3 + fp32 row scale (head)",
+        "arithmetic": "fp32 accumulate; MoE gate/up on tcgen05 block-scaled FP4 with x as eight E2M1 base-4 "
+                      "digits per 32-block, down on f16 MMA with h as two f16 parts per 16-value slice; head x as "
+                      "two E4M3 parts; weights MXFP4 (experts) and E4M3 + fp32 row scale (head)",
         "roofline": {"bound": "hbm", "kernel": "lmhead_fp8_kernel (FP8 LM head, M=1)", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": profiled_traffic(), "algorithmic_bytes_per_launch": head_bytes},

@@ -273,7 +273,8 @@ moe_status moe_query_path(char* buf, size_t n) {
       "sm_100a; moe: one cooperative persistent kernel (router fp32 GEMV with epoch-tagged logits, "
       "top-k softmax routing in every CTA, split-K over the intermediate: 16-row slices of MXFP4 "
       "E2M1/E8M0-32 gate/up + SiLU + down per work item, one bulk copy per item into a stage ring, "
-      "gate/up as tcgen05.mma kind::mxf4 block-scaled (TMEM accumulator, activations as 8 E2M1 parts), "
+      "gate/up as tcgen05.mma kind::mxf4 block-scaled on a 128-row operand of four K segments (TMEM "
+      "accumulator, activations as 8 E2M1 base-4 digits), "
       "down as mma.sync f16 on E2M1 placed as E5M2, one grid barrier, fixed-order combine); "
       "lm-head: online-FP8 E4M3 per-row-scale GEMV over the fragment-tiled head (warp-specialised: bulk-copy "
       "ring, two mma.sync m16n8k32 e4m3 consumer groups, counter-scheduled tail tiles) fused top-k "
