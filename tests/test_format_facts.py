@@ -12,6 +12,11 @@ independent decoder (ml_dtypes) -- not against the kernels' own code.
 * An E4M3 hi/lo split carries a bf16 value (the token scaled so that its
   largest magnitude is in [2^7, 2^8)) exactly when the scaled magnitude is
   at least 2^-2, and within 2^-10 below that.
+* The MoE gate/up's activation digits: for a block whose largest magnitude
+  lies in [2^E, 2^(E+1)), N = round(|v| 2^(15-E)) stays below 2^16, and its
+  eight base-4 digits d_p, each an E2M1 code 0..3 (value d/2) with the
+  value's sign at scale 2^(E-2p), sum to v exactly when v is within 2^-8 of
+  the block's largest and to within 2^(E-16) of it below.
 """
 import itertools
 
@@ -94,3 +99,30 @@ def test_bf16_is_carried_by_two_e4m3_parts():
     assert np.abs((hi + lo) - vals)[~big].max() <= 2.0 ** -10
     # the bound is tight: some value just below 2^-2 is not carried exactly
     assert (np.abs((hi + lo) - vals)[~big] > 0).any()
+
+
+def bf16_values():
+    """Every finite bf16 value, as float64."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    v = bits.view(ml_dtypes.bfloat16).astype(np.float64)
+    return v[np.isfinite(v)]
+
+
+@pytest.mark.parametrize("E", [-133, -127, -40, -1, 0, 7, 60, 127])
+def test_bf16_is_carried_by_eight_e2m1_digits(E):
+    v = bf16_values()
+    v = v[np.abs(v) < 2.0 ** (E + 1)]  # every value a block with largest magnitude in [2^E, 2^(E+1)) can hold
+    n = np.rint(np.abs(v) * 2.0 ** (15 - E))  # numpy rounds half to even, as the kernel's conversion does
+    assert n.max() < 2 ** 16
+    n = n.astype(np.int64)
+    digits = [(n >> (14 - 2 * p)) & 3 for p in range(8)]
+    # each digit is an E2M1 code (0, 0.5, 1, 1.5 for codes 0..3); decode it independently
+    total = np.zeros_like(v)
+    for p, d in enumerate(digits):
+        codes = d.astype(np.uint8) | np.where(v < 0, 8, 0).astype(np.uint8)
+        vals = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+        assert np.array_equal(np.abs(vals), d / 2.0)
+        total += vals * 2.0 ** (E - 2 * p)
+    big = np.abs(v) >= 2.0 ** (E - 8)
+    assert np.array_equal(total[big], v[big])
+    assert np.all(np.abs(total - v) <= 2.0 ** (E - 16))
