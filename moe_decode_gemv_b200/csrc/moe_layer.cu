@@ -130,10 +130,13 @@ struct Ctl {
 };
 constexpr int kCtlBytes = (int)((sizeof(Ctl) + 127) / 128 * 128);
 // The scratch area holds the tokens (bf16, while the router and the
-// activation parts read them), then the M x E router logits (while routing).
-__host__ __device__ constexpr int scratch_bytes(int H) {
-  const int xb = 4 * H * 2, lb = 4 * kMaxE * 4;
-  return ((xb > lb ? xb : lb) + 127) / 128 * 128;
+// activation digits read them), then the digits' scale table (T x 512 B),
+// then the M x E router logits (while routing): sized for this call, so that
+// a small M leaves room for another stage.
+__host__ __device__ constexpr int scratch_bytes(int H, int M, int E) {
+  const int xb = M * H * 2, tb = slice_ktiles(H) * 512, lb = M * E * 4;
+  const int b = xb > tb ? xb : tb;
+  return ((b > lb ? b : lb) + 127) / 128 * 128;
 }
 
 struct LayerArgs {
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   Ctl& C = *reinterpret_cast<Ctl*>(smem);
   uint8_t* scratch = smem + kCtlBytes;
   const Geo geo(a.H, a.I, a.M);
-  uint8_t* xparts = scratch + scratch_bytes(a.H);   // the gate/up B operand: [K tile][half][32 mp rows][16 B]
+  uint8_t* xparts = scratch + scratch_bytes(a.H, a.M, a.E);   // the gate/up B operand: [K tile][half][32 mp rows][16 B]
   uint8_t* stages = xparts + geo.xparts_bytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -890,9 +893,9 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   if (warp == 0) tmem_dealloc(tm, kTmemCols);
 }
 
-int moe_stages(int H, int M) {
+int moe_stages(int H, int M, int E) {
   const Geo geo(H, 32, M);
-  const int avail = kMaxDynamicSmem - kCtlBytes - scratch_bytes(H) - geo.xparts_bytes;
+  const int avail = kMaxDynamicSmem - kCtlBytes - scratch_bytes(H, M, E) - geo.xparts_bytes;
   int n = avail / geo.stage_bytes;
   return n > kMaxStages ? kMaxStages : n;
 }
@@ -906,7 +909,7 @@ cudaError_t launch_layer_t(const LayerArgs& a, cudaStream_t st) {
   const Geo geo(a.H, a.I, a.M);
   const int grid = sms < MoeWs::kMaxGrid ? sms : MoeWs::kMaxGrid;  // one CTA per SM, all resident
   const size_t smem =
-      (size_t)kCtlBytes + scratch_bytes(a.H) + geo.xparts_bytes + (size_t)a.stages * geo.stage_bytes;
+      (size_t)kCtlBytes + scratch_bytes(a.H, a.M, a.E) + geo.xparts_bytes + (size_t)a.stages * geo.stage_bytes;
   e = launch_dependent(moe_layer_kernel<kB>, dim3(grid), dim3(kThreads), smem, st, true, a);
   return e;
 }
@@ -915,12 +918,12 @@ cudaError_t launch_layer_t(const LayerArgs& a, cudaStream_t st) {
 
 bool moe_layer_supported(int H, int I) {
   return H >= 32 && H % 32 == 0 && H <= kMaxH && I >= 32 && I % 32 == 0 &&
-         I <= 65536 && moe_stages(H, 4) >= 1;
+         I <= 65536 && moe_stages(H, 4, kMaxE) >= 1;
 }
 
 cudaError_t launch_moe_layer(const MoeArgs& m, cudaStream_t st) {
   LayerArgs a{m.x, m.router_w, m.router_bias, m.bank, m.shared, m.M, m.top_k, m.E, m.H, m.I,
-              moe_stages(m.H, m.M), m.out, m.ids_out, m.w_out, m.ws};
+              moe_stages(m.H, m.M, m.E), m.out, m.ids_out, m.w_out, m.ws};
   const int need = (m.H / 32 + kWarps - 1) / kWarps;  // K blocks (= output groups) per warp
   if (need <= 1) return launch_layer_t<1>(a, st);
   if (need <= 2) return launch_layer_t<2>(a, st);
