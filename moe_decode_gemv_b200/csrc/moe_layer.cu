@@ -82,6 +82,8 @@ constexpr int16_t kZeroBlock = -32768;
 constexpr int kMaxStages = 4;
 constexpr int kMaxSlots = 4 * 8 + 1;
 constexpr int kRouterChunk = 8;        // float4 router loads in flight per lane
+constexpr int kRouteWarps = 8;         // warps 0..7 route while warps 8..15 build the activation digits
+constexpr int kGroupThreads = 32 * kRouteWarps;
 constexpr int kMaxE = 1024;
 constexpr uint32_t kFull = 0xffffffffu;
 
@@ -129,14 +131,14 @@ struct Ctl {
   int shifted;  // some block's t is not 0
 };
 constexpr int kCtlBytes = (int)((sizeof(Ctl) + 127) / 128 * 128);
-// The scratch area holds the tokens (bf16, while the router and the
-// activation digits read them), then the digits' scale table (T x 512 B),
-// then the M x E router logits (while routing): sized for this call, so that
-// a small M leaves room for another stage.
+// The scratch area holds, side by side, the tokens (bf16; the router and the
+// activation digits read them), the digits' scale table (T x 512 B) and the
+// M x E router logits (routing runs beside the digits): sized for this call,
+// so that a small M leaves room for another stage.
+__host__ __device__ constexpr int scratch_tokens_bytes(int H, int M) { return (M * H * 2 + 127) / 128 * 128; }
+__host__ __device__ constexpr int scratch_table_bytes(int H) { return slice_ktiles(H) * 512; }
 __host__ __device__ constexpr int scratch_bytes(int H, int M, int E) {
-  const int xb = M * H * 2, tb = slice_ktiles(H) * 512, lb = M * E * 4;
-  const int b = xb > tb ? xb : tb;
-  return ((b > lb ? b : lb) + 127) / 128 * 128;
+  return scratch_tokens_bytes(H, M) + scratch_table_bytes(H) + (M * E * 4 + 127) / 128 * 128;
 }
 
 struct LayerArgs {
@@ -150,6 +152,9 @@ struct LayerArgs {
   float* w_out;
   MoeWs ws;
 };
+
+// Barrier among `n` threads (whole warps) of the CTA, id 1..15.
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 // ---- memory helpers ----
 __device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
@@ -400,128 +405,288 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
     __syncthreads();
   }
 
-  // ---- x: eight E2M1 digits per token and 32-element block ----
-  // The gate/up MMA's B operand has N = 32 mp rows: row n = 8 mp s + 8 m + p
-  // holds digit p of token m over K segment s (elements 64 T s ..), K-major
-  // like the weights.  For a block whose largest magnitude lies in [2^E,
-  // 2^(E+1)), each value v is rounded to N = round(|v| 2^(15 - E)), an
-  // integer below 2^16 (exact when v is within 2^-8 of the block's largest,
-  // else off by at most 2^(E-16)), and written in base 4: digit p = bits
-  // 14 - 2p, 15 - 2p of N, stored as the E2M1 code of d / 2 (codes 0..3 are
-  // 0, 0.5, 1, 1.5) with v's sign, scale 2^(E - 2p).  The tensor core
-  // applies the scales, so the eight digit columns of a token sum to N
-  // 2^(E-15) x the weights.  The digits' E8M0 scales go to TMEM.
+  // ---- routing (warps 0..7): every CTA takes the same top-k of each token ----
+  auto route = [&]() {
+    float* lg = reinterpret_cast<float*>(scratch + scratch_tokens_bytes(H, M) + scratch_table_bytes(H));  // [M][E]
+    {
+      // this thread's words (at most 16: M * E <= 4096), eight loads at a
+      // time; only stale ones are read again
+      for (int i0 = threadIdx.x; i0 < M * E; i0 += 8 * kGroupThreads) {
+        uint64_t v[8];
+        uint32_t stale = 0u;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kGroupThreads;
+          if (i < M * E) {
+            v[u] = ld_relaxed_u64(&ws.logits[i]);
+            if ((uint32_t)(v[u] >> 32) != tag) stale |= 1u << u;
+          }
+        }
+        const uint64_t start = global_ns();
+        while (stale && !poisoned()) {
+          if (global_ns() - start > kWaitLimitNs) {
+            fail();
+            break;
+          }
+          __nanosleep(32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            if (stale >> u & 1u) {
+              v[u] = ld_relaxed_u64(&ws.logits[i0 + u * kGroupThreads]);
+              if ((uint32_t)(v[u] >> 32) == tag) stale &= ~(1u << u);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kGroupThreads;
+          if (i < M * E) {
+            const float x = __uint_as_float((uint32_t)v[u]);
+            lg[i] = x > -FLT_MAX ? x : -FLT_MAX;  // NaN and -inf rank as -FLT_MAX
+          }
+        }
+      }
+    }
+    named_sync(2, kGroupThreads);
+    // One warp per token: lane l holds experts l, l + 32, ...  The k-th best
+    // of the 32 lane maxima bounds the k-th best logit from below (those are k
+    // real logits), so only logits not worse than it are candidates; they are
+    // ranked by counting (ids are distinct, so ranks are).
+    if (warp < M) {
+      const int m = warp;
+      const float* lm = lg + m * E;
+      VI b = pad_entry(0);
+#pragma unroll 8
+      for (int e = lane; e < E; e += 32)
+        if (better(lm[e], e, b.v, b.i)) b = VI{lm[e], e};
+      int rank = 0;
+#pragma unroll
+      for (int o = 0; o < 32; ++o) {
+        const float ov = __shfl_sync(kFull, b.v, o);
+        const int32_t oi = __shfl_sync(kFull, b.i, o);
+        rank += better(ov, oi, b.v, b.i);
+      }
+      const uint32_t hit = __ballot_sync(kFull, rank == a.top_k - 1 && b.i < E);
+      VI bound = pad_entry(0);  // none: fewer than k lanes hold an expert, every expert is a candidate
+      if (hit) {
+        bound.v = __shfl_sync(kFull, b.v, __ffs(hit) - 1);
+        bound.i = __shfl_sync(kFull, b.i, __ffs(hit) - 1);
+      }
+      // compaction, eight ballots at a time (independent loads and votes,
+      // then the running count)
+      int nc = 0;
+      for (int e0 = 0; e0 < E; e0 += 256) {
+        uint32_t bal[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int e = e0 + 32 * u + lane;
+          bal[u] = __ballot_sync(kFull, e < E && !better(bound.v, bound.i, lm[e], e));
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int pos = nc + __popc(bal[u] & ((1u << lane) - 1u));
+          if (((bal[u] >> lane) & 1u) && pos < kCandCap)  // never more: k lanes' experts at most
+            C.cand[m][pos] = (uint16_t)(e0 + 32 * u + lane);
+          nc += __popc(bal[u]);
+        }
+      }
+      __syncwarp();
+      nc = min(nc, kCandCap);
+      for (int q = lane; q < nc; q += 32) {
+        const int e = C.cand[m][q];
+        const float v = lm[e];
+        int r = 0;
+#pragma unroll 8
+        for (int o = 0; o < nc; ++o) {
+          const int f = C.cand[m][o];
+          r += better(lm[f], f, v, e);
+        }
+        if (r < a.top_k) {
+          C.ids[m][r] = e;
+          C.topv[m][r] = v;
+        }
+      }
+      __syncwarp();
+      // softmax over the selected k, renormalised
+      const float v0 = C.topv[m][0];
+      const float ex = lane < a.top_k ? expf(C.topv[m][lane] - v0) : 0.f;
+      float z = ex;
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
+      if (lane < a.top_k) C.wts[m][lane] = ex / z;
+    }
+    named_sync(2, kGroupThreads);
+    if (warp == 0) {
+      // Slot table: slot 0 is the shared expert, then one slot per distinct
+      // routed expert in order of first appearance over (token, rank).
+      // Lane l holds choice l = m * top_k + r (M * top_k <= 32).
+      const int k = a.top_k, n_in = M * k;
+      const bool act = lane < n_in;
+      const int mm = act ? lane / k : 0, r = act ? lane - mm * k : 0;
+      int32_t ex = act ? C.ids[mm][r] : -1 - lane;  // idle lanes get ids of their own
+      if (act && (ex < 0 || ex >= E)) {  // cannot happen (every rank below k is filled); never index out of range
+        report(hdr, MOE_ERR_DEVICE_CHECK);
+        ex = 0;
+      }
+      const uint32_t same = __match_any_sync(kFull, ex);
+      const int leader = __ffs(same) - 1;
+      const uint32_t leaders = __ballot_sync(kFull, act && leader == lane);
+      const int slot = 1 + __popc(leaders & ((1u << leader) - 1u));
+      if (act && leader == lane) {
+        C.slot_expert[slot] = ex;
+        C.slot_mask[slot] = 0u;
+        for (int t = 0; t < 4; ++t) C.slot_w[slot][t] = 0.f;
+      }
+      if (lane == 0) {
+        C.slot_expert[0] = -1;
+        C.slot_mask[0] = (1u << M) - 1u;
+        for (int t = 0; t < 4; ++t) C.slot_w[0][t] = 1.0f;
+      }
+      __syncwarp();
+      if (act) {
+        atomicOr(&C.slot_mask[slot], 1u << mm);
+        C.slot_w[slot][mm] = C.wts[mm][r];  // a token picks an expert at most once
+      }
+      __syncwarp();
+      if (lane == 0) C.nslots = 1 + __popc(leaders);
+    }
+    named_sync(2, kGroupThreads);
+    if (c == 0) {
+      for (int i = threadIdx.x; i < M * a.top_k; i += kGroupThreads) {
+        if (a.ids_out) a.ids_out[i] = C.ids[i / a.top_k][i % a.top_k];
+        if (a.w_out) a.w_out[i] = C.wts[i / a.top_k][i % a.top_k];
+      }
+    }
+  };
+
   const int mp = padded_tokens(M);
-  // 1. E per (token, block)
-  for (int u = threadIdx.x; u < M * nb; u += kThreads) {
-    const int m = u / nb, b = u - m * nb;
-    const uint4* p = reinterpret_cast<const uint4*>(xs + m * H + 32 * b);
-    float am = 0.f;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 v = p[q];
-      am = fmaxf(am, fmaxf(fmaxf(bf16_bits_to_f32(v.x & 0x7fffu), bf16_bits_to_f32((v.x >> 16) & 0x7fffu)),
-                           fmaxf(bf16_bits_to_f32(v.y & 0x7fffu), bf16_bits_to_f32((v.y >> 16) & 0x7fffu))));
-      am = fmaxf(am, fmaxf(fmaxf(bf16_bits_to_f32(v.z & 0x7fffu), bf16_bits_to_f32((v.z >> 16) & 0x7fffu)),
-                           fmaxf(bf16_bits_to_f32(v.w & 0x7fffu), bf16_bits_to_f32((v.w >> 16) & 0x7fffu))));
-    }
-    C.ex[m][b] = am > 0.f ? (int16_t)floor_log2(am) : kZeroBlock;
-  }
-  __syncthreads();
-  // 2. per block, t: the product of a weight scale 2^(c - 127) and a digit
-  // scale 2^(E - 2p) is taken as 2^(c - t - 127) x 2^(E - 2p + t), with t
-  // chosen so that every token's digit codes E - 2p + t + 127 lie in [0,
-  // 254] (0 unless the block is below about 2^-113 or above 2^127).
-  for (int b = threadIdx.x; b < 8 * T; b += kThreads) {
-    int lo = -100000, hi = 100000;
-    for (int m = 0; m < M; ++m) {
-      const int eb = b < nb ? C.ex[m][b] : kZeroBlock;
-      if (eb != kZeroBlock) {
-        lo = max(lo, -127 - (eb - 2 * (kParts - 1)));
-        hi = min(hi, 127 - eb);
-      }
-    }
-    int t = 0;
-    if (t < lo) t = lo;
-    if (t > hi) t = hi;  // the leading digits win if no shift fits all
-    C.tshift[b] = (int16_t)t;
-    if (t != 0) C.shifted = 1;
-  }
-  // 3. the digits: one thread per (token, block, 8 elements, 4 digits),
-  // four 4-byte words; zero for padding
   const int lmp = mp == 1 ? 0 : (mp == 2 ? 1 : 2);
-  for (int u = threadIdx.x; u < mp * 64 * T; u += kThreads) {
-    const int ph = u & 1, u8 = u >> 1;
-    const int m = u8 / (32 * T), rest = u8 - m * (32 * T), b = rest >> 2, q = rest & 3;
-    const int sg = b / (2 * T), lb = b - sg * (2 * T), t = lb >> 1, hf = lb & 1;
-    uint8_t* dst = xparts + (size_t)t * (1024 * mp) + hf * (512 * mp) + (sg * mp + m) * 128 + 64 * ph + 4 * q;
-    const int eb = (m < M && b < nb) ? C.ex[m][b] : kZeroBlock;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (eb != kZeroBlock) {
-      const uint4 xv = *reinterpret_cast<const uint4*>(xs + m * H + 32 * b + 8 * q);
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-      uint32_t pr[4] = {0u, 0u, 0u, 0u}, sgn = 0u;  // pr[i] = N_i | N_(i+4) << 16
+  if (warp < kRouteWarps) {
+    route();
+  } else {
+    const int xt = threadIdx.x - kGroupThreads;  // warps 8..15
+    // ---- x: eight E2M1 digits per token and 32-element block ----
+    // The gate/up MMA's B operand has N = 32 mp rows: row n = 8 mp s + 8 m + p
+    // holds digit p of token m over K segment s (elements 64 T s ..), K-major
+    // like the weights.  For a block whose largest magnitude lies in [2^E,
+    // 2^(E+1)), each value v is rounded to N = round(|v| 2^(15 - E)), an
+    // integer below 2^16 (exact when v is within 2^-8 of the block's largest,
+    // else off by at most 2^(E-16)), and written in base 4: digit p = bits
+    // 14 - 2p, 15 - 2p of N, stored as the E2M1 code of d / 2 (codes 0..3 are
+    // 0, 0.5, 1, 1.5) with v's sign, scale 2^(E - 2p).  The tensor core
+    // applies the scales, so the eight digit columns of a token sum to N
+    // 2^(E-15) x the weights.  The digits' E8M0 scales go to TMEM.
+    // 1. E per (token, block)
+    for (int u = xt; u < M * nb; u += kGroupThreads) {
+      const int m = u / nb, b = u - m * nb;
+      const uint4* p = reinterpret_cast<const uint4*>(xs + m * H + 32 * b);
+      float am = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t bits = (xw[i >> 1] >> (16 * (i & 1))) & 0xffffu;
-        const uint32_t n = __float2uint_rn(mul_pow2(bf16_bits_to_f32(bits & 0x7fffu), 15 - eb));
-        pr[i & 3] |= n << (16 * (i >> 2));
-        sgn |= (bits >> 15) << (4 * i + 3);
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = p[q];
+        am = fmaxf(am, fmaxf(fmaxf(bf16_bits_to_f32(v.x & 0x7fffu), bf16_bits_to_f32((v.x >> 16) & 0x7fffu)),
+                             fmaxf(bf16_bits_to_f32(v.y & 0x7fffu), bf16_bits_to_f32((v.y >> 16) & 0x7fffu))));
+        am = fmaxf(am, fmaxf(fmaxf(bf16_bits_to_f32(v.z & 0x7fffu), bf16_bits_to_f32((v.z >> 16) & 0x7fffu)),
+                             fmaxf(bf16_bits_to_f32(v.w & 0x7fffu), bf16_bits_to_f32((v.w >> 16) & 0x7fffu))));
       }
-      const int sh0 = 14 - 8 * ph;  // digit 4 ph: bits sh0, sh0 + 1
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        uint32_t v = sgn;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v |= ((pr[i] >> (sh0 - 2 * p)) & 0x00030003u) << (4 * i);
-        w[p] = v;
+      C.ex[m][b] = am > 0.f ? (int16_t)floor_log2(am) : kZeroBlock;
+    }
+    named_sync(3, kGroupThreads);
+    // 2. per block, t: the product of a weight scale 2^(c - 127) and a digit
+    // scale 2^(E - 2p) is taken as 2^(c - t - 127) x 2^(E - 2p + t), with t
+    // chosen so that every token's digit codes E - 2p + t + 127 lie in [0,
+    // 254] (0 unless the block is below about 2^-113 or above 2^127).
+    for (int b = xt; b < 8 * T; b += kGroupThreads) {
+      int lo = -100000, hi = 100000;
+      for (int m = 0; m < M; ++m) {
+        const int eb = b < nb ? C.ex[m][b] : kZeroBlock;
+        if (eb != kZeroBlock) {
+          lo = max(lo, -127 - (eb - 2 * (kParts - 1)));
+          hi = min(hi, 127 - eb);
+        }
       }
+      int t = 0;
+      if (t < lo) t = lo;
+      if (t > hi) t = hi;  // the leading digits win if no shift fits all
+      C.tshift[b] = (int16_t)t;
+      if (t != 0) C.shifted = 1;
     }
+    // 3. the digits: one thread per (token, block, 8 elements, 4 digits),
+    // four 4-byte words; zero for padding
+    for (int u = xt; u < mp * 64 * T; u += kGroupThreads) {
+      const int ph = u & 1, u8 = u >> 1;
+      const int m = u8 / (32 * T), rest = u8 - m * (32 * T), b = rest >> 2, q = rest & 3;
+      const int sg = b / (2 * T), lb = b - sg * (2 * T), t = lb >> 1, hf = lb & 1;
+      uint8_t* dst = xparts + (size_t)t * (1024 * mp) + hf * (512 * mp) + (sg * mp + m) * 128 + 64 * ph + 4 * q;
+      const int eb = (m < M && b < nb) ? C.ex[m][b] : kZeroBlock;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (eb != kZeroBlock) {
+        const uint4 xv = *reinterpret_cast<const uint4*>(xs + m * H + 32 * b + 8 * q);
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        uint32_t pr[4] = {0u, 0u, 0u, 0u}, sgn = 0u;  // pr[i] = N_i | N_(i+4) << 16
 #pragma unroll
-    for (int p = 0; p < 4; ++p) *reinterpret_cast<uint32_t*>(dst + 16 * p) = w[p];
-  }
-  fence_proxy_async_smem();  // the tensor core reads these through the async proxy
-  __syncthreads();           // every block's t is written; the tokens are no longer read
-  const bool shifted = C.shifted != 0;
-  // 4. the digits' scales: K tile t, operand row n = 32 q + lane in column q
-  // of the tile's group, in every lane quarter; bytes 0, 1 = the two halves;
-  // 127 where the digit is zero.  All threads fill a table [T][4][32] in the
-  // scratch area, then warps 0..3 copy it into their lane quarters.
-  uint32_t* sfbt = reinterpret_cast<uint32_t*>(scratch);
-  for (int e = threadIdx.x; e < 128 * T; e += kThreads) {
-    const int t = e >> 7, q = (e >> 5) & 3, n = e & 127;
-    const int sg = n >> (3 + lmp), m = (n >> 3) & (mp - 1), p = n & 7;
-    uint32_t w = 0u;
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t bits = (xw[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+          const uint32_t n = __float2uint_rn(mul_pow2(bf16_bits_to_f32(bits & 0x7fffu), 15 - eb));
+          pr[i & 3] |= n << (16 * (i >> 2));
+          sgn |= (bits >> 15) << (4 * i + 3);
+        }
+        const int sh0 = 14 - 8 * ph;  // digit 4 ph: bits sh0, sh0 + 1
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const int b = 2 * T * sg + 2 * t + hf;
-      const int eb = (q < mp && m < M && b < nb) ? C.ex[m][b] : kZeroBlock;
-      int code = 127;
-      if (eb != kZeroBlock) code = min(max(eb - 2 * p + C.tshift[b] + 127, 0), 254);
-      w |= (uint32_t)code << (8 * hf);
-    }
-    sfbt[e] = w;
-  }
-  __syncthreads();
-  if (warp < 4) {
-    for (int t0 = 0; t0 < T; t0 += 8) {
-      uint32_t v[32];
+        for (int p = 0; p < 4; ++p) {
+          uint32_t v = sgn;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = t0 + (i >> 2) < T ? sfbt[(t0 * 4 + i) * 32 + lane] : 0u;
-      const uint32_t ta = tm + ((uint32_t)(32 * warp) << 16) + tm_sfb + 4u * t0;
-      if (T - t0 >= 8) {
-        tmem_st_x32(ta, v);
-      } else {
-#pragma unroll
-        for (int tt = 0; tt < 7; ++tt)
-          if (tt < T - t0) tmem_st_x4(ta + 4u * tt, v[4 * tt], v[4 * tt + 1], v[4 * tt + 2], v[4 * tt + 3]);
+          for (int i = 0; i < 4; ++i) v |= ((pr[i] >> (sh0 - 2 * p)) & 0x00030003u) << (4 * i);
+          w[p] = v;
+        }
       }
+#pragma unroll
+      for (int p = 0; p < 4; ++p) *reinterpret_cast<uint32_t*>(dst + 16 * p) = w[p];
     }
-    tmem_wait_st();
+    fence_proxy_async_smem();  // the tensor core reads these through the async proxy
+    named_sync(3, kGroupThreads);  // every block's t is written
+    // 4. the digits' scales: K tile t, operand row n = 32 q + lane in column q
+    // of the tile's group, in every lane quarter; bytes 0, 1 = the two halves;
+    // 127 where the digit is zero.  These warps fill a table [T][4][32] in the
+    // scratch area, then warps 8..11 copy it into lane quarters 0..3.
+    uint32_t* sfbt = reinterpret_cast<uint32_t*>(scratch + scratch_tokens_bytes(H, M));
+    for (int e = xt; e < 128 * T; e += kGroupThreads) {
+      const int t = e >> 7, q = (e >> 5) & 3, n = e & 127;
+      const int sg = n >> (3 + lmp), m = (n >> 3) & (mp - 1), p = n & 7;
+      uint32_t w = 0u;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int b = 2 * T * sg + 2 * t + hf;
+        const int eb = (q < mp && m < M && b < nb) ? C.ex[m][b] : kZeroBlock;
+        int code = 127;
+        if (eb != kZeroBlock) code = min(max(eb - 2 * p + C.tshift[b] + 127, 0), 254);
+        w |= (uint32_t)code << (8 * hf);
+      }
+      sfbt[e] = w;
+    }
+    named_sync(3, kGroupThreads);
+    if (warp < kRouteWarps + 4) {
+      for (int t0 = 0; t0 < T; t0 += 8) {
+        uint32_t v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = t0 + (i >> 2) < T ? sfbt[(t0 * 4 + i) * 32 + lane] : 0u;
+        const uint32_t ta = tm + ((uint32_t)(32 * (warp & 3)) << 16) + tm_sfb + 4u * t0;
+        if (T - t0 >= 8) {
+          tmem_st_x32(ta, v);
+        } else {
+#pragma unroll
+          for (int tt = 0; tt < 7; ++tt)
+            if (tt < T - t0) tmem_st_x4(ta + 4u * tt, v[4 * tt], v[4 * tt + 1], v[4 * tt + 2], v[4 * tt + 3]);
+        }
+      }
+      tmem_wait_st();
+    }
+
   }
   tc_fence_before_sync();
-  __syncthreads();  // the tokens' shared memory is free from here on
+  __syncthreads();  // routed, and the digits are built; the tokens' shared memory is free from here on
   tc_fence_after_sync();
+  const bool shifted = C.shifted != 0;
 
   // ---- one work item: gate/up over H, SiLU gate, down over its 16 columns ----
   float yacc[kB][4];
@@ -662,169 +827,11 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
     __syncthreads();  // the stage, the partial sums and h are free for the next item
   };
 
-  // ---- routing: every CTA takes the same top-k of each token ----
-  auto route = [&]() {
-    float* lg = reinterpret_cast<float*>(scratch);  // [M][E]
-    {
-      // this thread's words (at most 8: M * E <= 4096), all read at once;
-      // only stale ones are read again
-      constexpr int kPer = 4 * kMaxE / kThreads;
-      uint64_t v[kPer];
-      uint32_t stale = 0u;
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int i = threadIdx.x + u * kThreads;
-        if (i < M * E) {
-          v[u] = ld_relaxed_u64(&ws.logits[i]);
-          if ((uint32_t)(v[u] >> 32) != tag) stale |= 1u << u;
-        }
-      }
-      const uint64_t start = global_ns();
-      while (stale && !poisoned()) {
-        if (global_ns() - start > kWaitLimitNs) {
-          fail();
-          break;
-        }
-        __nanosleep(32);
-#pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-          if (stale >> u & 1u) {
-            v[u] = ld_relaxed_u64(&ws.logits[threadIdx.x + u * kThreads]);
-            if ((uint32_t)(v[u] >> 32) == tag) stale &= ~(1u << u);
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int i = threadIdx.x + u * kThreads;
-        if (i < M * E) {
-          const float x = __uint_as_float((uint32_t)v[u]);
-          lg[i] = x > -FLT_MAX ? x : -FLT_MAX;  // NaN and -inf rank as -FLT_MAX
-        }
-      }
-    }
-    __syncthreads();
-    // One warp per token: lane l holds experts l, l + 32, ...  The k-th best
-    // of the 32 lane maxima bounds the k-th best logit from below (those are k
-    // real logits), so only logits not worse than it are candidates; they are
-    // ranked by counting (ids are distinct, so ranks are).
-    if (warp < M) {
-      const int m = warp;
-      const float* lm = lg + m * E;
-      VI b = pad_entry(0);
-#pragma unroll 8
-      for (int e = lane; e < E; e += 32)
-        if (better(lm[e], e, b.v, b.i)) b = VI{lm[e], e};
-      int rank = 0;
-#pragma unroll
-      for (int o = 0; o < 32; ++o) {
-        const float ov = __shfl_sync(kFull, b.v, o);
-        const int32_t oi = __shfl_sync(kFull, b.i, o);
-        rank += better(ov, oi, b.v, b.i);
-      }
-      const uint32_t hit = __ballot_sync(kFull, rank == a.top_k - 1 && b.i < E);
-      VI bound = pad_entry(0);  // none: fewer than k lanes hold an expert, every expert is a candidate
-      if (hit) {
-        bound.v = __shfl_sync(kFull, b.v, __ffs(hit) - 1);
-        bound.i = __shfl_sync(kFull, b.i, __ffs(hit) - 1);
-      }
-      // compaction, eight ballots at a time (independent loads and votes,
-      // then the running count)
-      int nc = 0;
-      for (int e0 = 0; e0 < E; e0 += 256) {
-        uint32_t bal[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int e = e0 + 32 * u + lane;
-          bal[u] = __ballot_sync(kFull, e < E && !better(bound.v, bound.i, lm[e], e));
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int pos = nc + __popc(bal[u] & ((1u << lane) - 1u));
-          if (((bal[u] >> lane) & 1u) && pos < kCandCap)  // never more: k lanes' experts at most
-            C.cand[m][pos] = (uint16_t)(e0 + 32 * u + lane);
-          nc += __popc(bal[u]);
-        }
-      }
-      __syncwarp();
-      nc = min(nc, kCandCap);
-      for (int q = lane; q < nc; q += 32) {
-        const int e = C.cand[m][q];
-        const float v = lm[e];
-        int r = 0;
-#pragma unroll 8
-        for (int o = 0; o < nc; ++o) {
-          const int f = C.cand[m][o];
-          r += better(lm[f], f, v, e);
-        }
-        if (r < a.top_k) {
-          C.ids[m][r] = e;
-          C.topv[m][r] = v;
-        }
-      }
-      __syncwarp();
-      // softmax over the selected k, renormalised
-      const float v0 = C.topv[m][0];
-      const float ex = lane < a.top_k ? expf(C.topv[m][lane] - v0) : 0.f;
-      float z = ex;
-#pragma unroll
-      for (int o = 4; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
-      if (lane < a.top_k) C.wts[m][lane] = ex / z;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // Slot table: slot 0 is the shared expert, then one slot per distinct
-      // routed expert in order of first appearance over (token, rank).
-      // Lane l holds choice l = m * top_k + r (M * top_k <= 32).
-      const int k = a.top_k, n_in = M * k;
-      const bool act = lane < n_in;
-      const int mm = act ? lane / k : 0, r = act ? lane - mm * k : 0;
-      int32_t ex = act ? C.ids[mm][r] : -1 - lane;  // idle lanes get ids of their own
-      if (act && (ex < 0 || ex >= E)) {  // cannot happen (every rank below k is filled); never index out of range
-        report(hdr, MOE_ERR_DEVICE_CHECK);
-        ex = 0;
-      }
-      const uint32_t same = __match_any_sync(kFull, ex);
-      const int leader = __ffs(same) - 1;
-      const uint32_t leaders = __ballot_sync(kFull, act && leader == lane);
-      const int slot = 1 + __popc(leaders & ((1u << leader) - 1u));
-      if (act && leader == lane) {
-        C.slot_expert[slot] = ex;
-        C.slot_mask[slot] = 0u;
-        for (int t = 0; t < 4; ++t) C.slot_w[slot][t] = 0.f;
-      }
-      if (lane == 0) {
-        C.slot_expert[0] = -1;
-        C.slot_mask[0] = (1u << M) - 1u;
-        for (int t = 0; t < 4; ++t) C.slot_w[0][t] = 1.0f;
-      }
-      __syncwarp();
-      if (act) {
-        atomicOr(&C.slot_mask[slot], 1u << mm);
-        C.slot_w[slot][mm] = C.wts[mm][r];  // a token picks an expert at most once
-      }
-      __syncwarp();
-      if (lane == 0) C.nslots = 1 + __popc(leaders);
-    }
-    __syncthreads();
-    if (c == 0) {
-      for (int i = threadIdx.x; i < M * a.top_k; i += kThreads) {
-        if (a.ids_out) a.ids_out[i] = C.ids[i / a.top_k][i % a.top_k];
-        if (a.w_out) a.w_out[i] = C.wts[i / a.top_k][i % a.top_k];
-      }
-    }
-  };
-
-  // ---- the items: the shared expert's first, routing when they are done ----
-  int n_my = n_pre;
-  for (int j = 0;; ++j) {
-    if (j == n_pre) {
-      route();
-      const int n_items = C.nslots * n_sl;
-      n_my = c < n_items ? (n_items - c + G - 1) / G : 0;
-      top_up(n_my);
-    }
-    if (j >= n_my) break;
+  // ---- the items: the shared expert's first (its copies went out at the start) ----
+  const int n_all = C.nslots * n_sl;
+  const int n_my = c < n_all ? (n_all - c + G - 1) / G : 0;
+  top_up(n_my);
+  for (int j = 0; j < n_my; ++j) {
     compute(j);
     consumed = j + 1;
     top_up(n_my);
