@@ -311,8 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   // ---- router loads of this CTA's rows: the first chunk goes out now ----
   const int e_begin = (int)((int64_t)E * c / G), e_end = (int)((int64_t)E * (c + 1) / G);
   const int R = e_end - e_begin;
-  const int RR = R < kRouteWarps ? R : kRouteWarps;  // rows per round (warps 0..7 run the router)
-  const int wpr = RR > 0 ? kRouteWarps / RR : 1;      // warps per row
+  const int RR = R < kWarps ? R : kWarps;    // rows per round
+  const int wpr = RR > 0 ? kWarps / RR : 1;  // warps per row
   const int F = H / 4;                       // float4 per router row
   auto router_slot = [&](int base, int& row, int& f0, int& f1) {  // this warp's share of a round
     const int lr = warp / wpr, part = warp - lr * wpr;
@@ -362,50 +362,48 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   };
   if (!mbar_wait(&C.xbar, 0)) fail();
 
-  // ---- router GEMV (warps 0..7): finish the first chunk, then any further chunks/rounds ----
-  auto router = [&]() {
-    float racc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int base = 0; base < R; base += RR) {
-      router_slot(base, r_row, r_f0, r_f1);
-      for (int f = r_f0 + lane; f < r_f1; f += 32 * kRouterChunk) {
-        if (!(base == 0 && f == r_f0 + lane)) router_load(r_row, f, r_f1);
-        if (r_row >= 0) {
+  // ---- router GEMV: finish the first chunk, then any further chunks/rounds ----
+  float racc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int base = 0; base < R; base += RR) {
+    router_slot(base, r_row, r_f0, r_f1);
+    for (int f = r_f0 + lane; f < r_f1; f += 32 * kRouterChunk) {
+      if (!(base == 0 && f == r_f0 + lane)) router_load(r_row, f, r_f1);
+      if (r_row >= 0) {
 #pragma unroll
-          for (int i = 0; i < kRouterChunk; ++i) {
-            const int ff = f + 32 * i;
-            if (ff < r_f1) {
+        for (int i = 0; i < kRouterChunk; ++i) {
+          const int ff = f + 32 * i;
+          if (ff < r_f1) {
 #pragma unroll
-              for (int m = 0; m < 4; ++m) {
-                if (m < M) {
-                  const uint2 xv = *reinterpret_cast<const uint2*>(xs + m * H + 4 * ff);
-                  racc[m] += wv[i].x * bf16_bits_to_f32(xv.x & 0xffffu) + wv[i].y * bf16_bits_to_f32(xv.x >> 16) +
-                             wv[i].z * bf16_bits_to_f32(xv.y & 0xffffu) + wv[i].w * bf16_bits_to_f32(xv.y >> 16);
-                }
+            for (int m = 0; m < 4; ++m) {
+              if (m < M) {
+                const uint2 xv = *reinterpret_cast<const uint2*>(xs + m * H + 4 * ff);
+                racc[m] += wv[i].x * bf16_bits_to_f32(xv.x & 0xffffu) + wv[i].y * bf16_bits_to_f32(xv.x >> 16) +
+                           wv[i].z * bf16_bits_to_f32(xv.y & 0xffffu) + wv[i].w * bf16_bits_to_f32(xv.y >> 16);
               }
             }
           }
         }
       }
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float v = warp_sum(racc[m]);
-        if (lane == 0) C.router_part[warp][m] = v;
-        racc[m] = 0.f;
-      }
-      named_sync(2, kGroupThreads);
-      if (threadIdx.x < RR * 4) {
-        const int lr = threadIdx.x >> 2, m = threadIdx.x & 3;
-        const int e = e_begin + base + lr;
-        if (m < M && base + lr < R) {
-          float l = 0.f;
-          for (int p = 0; p < wpr; ++p) l += C.router_part[lr * wpr + p][m];
-          if (a.router_bias) l += a.router_bias[e];
-          st_relaxed_u64(&ws.logits[(size_t)m * E + e], ((uint64_t)tag << 32) | __float_as_uint(l));
-        }
-      }
-      named_sync(2, kGroupThreads);
     }
-  };
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float v = warp_sum(racc[m]);
+      if (lane == 0) C.router_part[warp][m] = v;
+      racc[m] = 0.f;
+    }
+    __syncthreads();
+    if (threadIdx.x < RR * 4) {
+      const int lr = threadIdx.x >> 2, m = threadIdx.x & 3;
+      const int e = e_begin + base + lr;
+      if (m < M && base + lr < R) {
+        float l = 0.f;
+        for (int p = 0; p < wpr; ++p) l += C.router_part[lr * wpr + p][m];
+        if (a.router_bias) l += a.router_bias[e];
+        st_relaxed_u64(&ws.logits[(size_t)m * E + e], ((uint64_t)tag << 32) | __float_as_uint(l));
+      }
+    }
+    __syncthreads();
+  }
 
   // ---- routing (warps 0..7): every CTA takes the same top-k of each token ----
   auto route = [&]() {
@@ -564,7 +562,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   const int mp = padded_tokens(M);
   const int lmp = mp == 1 ? 0 : (mp == 2 ? 1 : 2);
   if (warp < kRouteWarps) {
-    router();
     route();
   } else {
     const int xt = threadIdx.x - kGroupThreads;  // warps 8..15
