@@ -261,13 +261,20 @@ def _q(v, f):
     return v[min(len(v) - 1, int(f * len(v)))]
 
 
+def block_steps(steps):
+    """Steps between two timing events in the distribution pass: 20 when
+    there are at least 200 steps (so at least 10 blocks), else a tenth."""
+    return 20 if steps >= 200 else max(1, steps // 10)
+
+
 def time_steps(wl, M, steps, warmup, dist, device, skewed=False):
     """Device time of `steps` steps, in three passes over the same steps on
-    the launching stream: (1) CUDA events at step boundaries only, for the
-    per-step distribution (the MoE -> head hand-over inside a step keeps its
-    programmatic launch); (2) two events around all steps, for the mean of
-    back-to-back steps; (3) an extra event between the MoE layer and the head
-    of every step, for the split between them (us)."""
+    the launching stream: (1) CUDA events every `block` steps only, for the
+    distribution of the per-step time over blocks (inside a block every
+    kernel keeps its programmatic launch, across steps too); (2) two events
+    around all steps, for the mean of back-to-back steps; (3) an extra event
+    between the MoE layer and the head of every step, for the split between
+    them (us)."""
     torch = wl.torch
     for i in range(warmup):
         wl.step(i, M, skewed=skewed)
@@ -275,16 +282,19 @@ def time_steps(wl, M, steps, warmup, dist, device, skewed=False):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    # (1) per-step distribution
-    bounds = [ev() for _ in range(steps + 1)]
+    # (1) per-step time over blocks of steps
+    block = block_steps(steps)
+    nblk = max(1, steps // block)
+    bounds = [ev() for _ in range(nblk + 1)]
     t0 = time.time()
     bounds[0].record()
-    for i in range(steps):
-        wl.step(warmup + i, M, skewed=skewed)
-        bounds[i + 1].record()
+    for b in range(nblk):
+        for i in range(block):
+            wl.step(warmup + b * block + i, M, skewed=skewed)
+        bounds[b + 1].record()
     torch.cuda.synchronize()
     t1 = time.time()
-    step = [bounds[i].elapsed_time(bounds[i + 1]) * 1e3 for i in range(steps)]
+    step = [bounds[b].elapsed_time(bounds[b + 1]) * 1e3 / block for b in range(nblk)]
     # (2) back-to-back
     e0, e1 = ev(), ev()
     e0.record()
@@ -301,7 +311,7 @@ def time_steps(wl, M, steps, warmup, dist, device, skewed=False):
     moe = [e[0].elapsed_time(e[1]) * 1e3 for e in evs]
     head = [e[1].elapsed_time(e[2]) * 1e3 for e in evs]
     med = max_over_ranks(statistics.median(step), dist, device)
-    return {"total_us": total_ms * 1e3, "per_step_us": total_ms * 1e3 / steps,
+    return {"total_us": total_ms * 1e3, "per_step_us": total_ms * 1e3 / steps, "block_steps": block,
             "step_us_median": med, "step_us_p10": _q(step, 0.1), "step_us_p90": _q(step, 0.9),
             "moe_us_mean": statistics.fmean(moe), "moe_us_median": statistics.median(moe),
             "moe_us_p10": _q(moe, 0.1), "moe_us_p90": _q(moe, 0.9),
@@ -755,8 +765,10 @@ def main():
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(),
         "value_stats": {"median_us": m1["step_us_median"], "p10_us": m1["step_us_p10"], "p90_us": m1["step_us_p90"],
                         "back_to_back_mean_us": m1["per_step_us"], "steps": args.steps,
-                        "timing": "CUDA events at step boundaries on the launching stream; inputs larger than L2 "
-                                  "(8 rotating layer copies + the 403 MB head per step)"},
+                        "block_steps": m1["block_steps"],
+                        "timing": "CUDA events on the launching stream every block_steps steps; value = the median "
+                                  "over blocks of the block time / block_steps; inputs larger than L2 (8 rotating "
+                                  "layer copies + the 403 MB head per step)"},
         "arithmetic": "fp32 accumulate; MoE gate/up on tcgen05 block-scaled FP4 with x as eight E2M1 base-4 "
                       "digits per 32-block, down on f16 MMA with h as two f16 parts per 16-value slice; head x as "
                       "two E4M3 parts; weights MXFP4 (experts) and E4M3 + fp32 row scale (head)",

@@ -99,3 +99,12 @@ def test_workload_config_names_the_workload():
     assert cfg["top_k"] == 8 and cfg["vocab"] == 157184 and cfg["head_top_k"] == 29 and cfg["M"] == 1
     assert "larger than L2" in cfg["l2"]
     assert bench.UNIT == "us/step"
+
+
+def test_block_steps_gives_at_least_ten_blocks():
+    bench = _bench()
+    assert bench.block_steps(2000) == 20
+    assert bench.block_steps(200) == 20
+    assert bench.block_steps(199) == 19
+    assert bench.block_steps(30) == 3
+    assert bench.block_steps(3) == 1
