@@ -741,12 +741,21 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
     __syncthreads();
     if (threadIdx.x == 0) {
       tc_fence_after_sync();
-      const uint32_t a0 = smem_addr(st), b0 = smem_addr(xparts);
       const uint32_t bt = 1024u * (uint32_t)mp, idesc = mxf4_idesc(32u * (uint32_t)mp);
-      for (int t = 0; t < T; ++t)
-        mma_mxf4(tm + kTmemD, umma_desc_kmajor(a0 + 4096u * t, 2048u, 128u),
-                 umma_desc_kmajor(b0 + bt * t, bt >> 1, 128u), idesc, tm + kTmemSfa + 4u * t,
-                 tm + tm_sfb + 4u * t, t > 0);
+      // tile t's descriptors are tile 0's plus t times the tile size in
+      // 16-byte units (the start-address field; no carry: shared memory is
+      // below 256 KB)
+      uint64_t ad = umma_desc_kmajor(smem_addr(st), 2048u, 128u);
+      uint64_t bd = umma_desc_kmajor(smem_addr(xparts), bt >> 1, 128u);
+      uint32_t sfa = tm + kTmemSfa, sfb = tm + tm_sfb;
+      mma_mxf4(tm + kTmemD, ad, bd, idesc, sfa, sfb, false);
+      for (int t = 1; t < T; ++t) {
+        ad += 4096u >> 4;
+        bd += bt >> 4;
+        sfa += 4u;
+        sfb += 4u;
+        mma_mxf4(tm + kTmemD, ad, bd, idesc, sfa, sfb, true);
+      }
       mma_commit(&C.mma_bar);
     }
     // h from the accumulator: warp s < 4 adds the digit columns of segment s
