@@ -507,6 +507,17 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
         }
       }
       __syncwarp();
+      if (M == 1) {
+        // one token: its k experts are the routed slots in rank order, so the
+        // CTA's routed items can go out now, before the softmax and the table
+        if (lane < a.top_k) C.slot_expert[1 + lane] = C.ids[0][lane];
+        if (lane == 0) C.nslots = 1 + a.top_k;
+        __syncwarp();
+        if (threadIdx.x == 0) {
+          const int n_items = C.nslots * n_sl;
+          top_up(c < n_items ? (n_items - c + G - 1) / G : 0);
+        }
+      }
       // softmax over the selected k, renormalised
       const float v0 = C.topv[m][0];
       const float ex = lane < a.top_k ? expf(C.topv[m][lane] - v0) : 0.f;
@@ -786,7 +797,9 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
         const float gv = (C.gu[0][m][lane] + C.gu[1][m][lane]) + (C.gu[2][m][lane] + C.gu[3][m][lane]);
         const float uv = __shfl_down_sync(kFull, gv, 16);
         const bool live = lane < 16 && ((mask >> m) & 1u);
-        const float h = live ? gv / (1.0f + expf(-gv)) * uv : 0.f;
+        // silu with the fast exponential and division (relative error near 2^-21; a very negative
+        // gate gives 0 where silu is below 2^-125 in magnitude)
+        const float h = live ? __fdividef(gv, 1.0f + __expf(-gv)) * uv : 0.f;
         float am = fabsf(h);
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(kFull, am, o));
