@@ -202,25 +202,6 @@ __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t
 __device__ __forceinline__ float scale_pow2(float v, int s) {
   return s > 126 ? v * exp2i(126) * exp2i(s - 126) : v * exp2i(s);
 }
-// v * 2^k for |k| <= 378: exact whenever the result is a normal number.
-__device__ __forceinline__ float mul_pow2(float v, int k) {
-  if (k > 126) {
-    v *= exp2i(126);
-    k -= 126;
-    if (k > 126) {
-      v *= exp2i(126);
-      k -= 126;
-    }
-  } else if (k < -126) {
-    v *= exp2i(-126);
-    k += 126;
-    if (k < -126) {
-      v *= exp2i(-126);
-      k += 126;
-    }
-  }
-  return v * exp2i(k);
-}
 // floor(log2(a)) of a positive finite float (subnormals included).
 __device__ __forceinline__ int floor_log2(float a) {
   const uint32_t b = __float_as_uint(a);
@@ -635,10 +616,14 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
         const uint4 xv = *reinterpret_cast<const uint4*>(xs + m * H + 32 * b + 8 * q);
         const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
         uint32_t pr[4] = {0u, 0u, 0u, 0u}, sgn = 0u;  // pr[i] = N_i | N_(i+4) << 16
+        // 2^(15 - E) as one or two exact factors (15 - E <= 148), found once
+        // per unit: a range test per element costs a branch per element
+        const int kk = 15 - eb;
+        const float f1 = kk > 126 ? exp2i(126) : 1.0f, f2 = exp2i(kk > 126 ? kk - 126 : kk);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint32_t bits = (xw[i >> 1] >> (16 * (i & 1))) & 0xffffu;
-          const uint32_t n = __float2uint_rn(mul_pow2(bf16_bits_to_f32(bits & 0x7fffu), 15 - eb));
+          const uint32_t n = __float2uint_rn(bf16_bits_to_f32(bits & 0x7fffu) * f1 * f2);
           pr[i & 3] |= n << (16 * (i >> 2));
           sgn |= (bits >> 15) << (4 * i + 3);
         }
