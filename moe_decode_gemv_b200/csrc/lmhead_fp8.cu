@@ -660,7 +660,14 @@ cudaError_t launch_fp8_t(const uint16_t* x, const uint8_t* qt, const float* s, i
 bool lmhead_fp8_plan(int H, int M, int top_k, int64_t V, int grid, int* stages, size_t* smem) {
   if (grid < 1 || grid > kLmheadMaxGrid) return false;
   if (H < 64 || H % 64 != 0 || H > kMaxHF || M < 1 || M > 4 || top_k < 1 || top_k > 64) return false;
-  for (int st = kMaxStagesF; st >= 2; --st) {
+  // An even number of stages: the two consumer groups take alternate
+  // iterations and iteration i uses stage i % stages, so each stage then
+  // belongs to one group, and a group never waits on a stage's barrier two
+  // phases ahead of it.  With an odd count a stage alternates between the
+  // groups, and a group running ahead could take the other group's earlier
+  // phase of the barrier for its own (the parities match) and read the
+  // other group's tile.
+  for (int st = kMaxStagesF & ~1; st >= 2; st -= 2) {
     const HeadGeo g = head_geo(V, H, M, grid, st, top_k);
     if (g.smem <= (size_t)kMaxDynamicSmem) {
       *stages = st;
