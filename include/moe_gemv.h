@@ -230,8 +230,9 @@ MOE_API size_t moe_workspace_bytes(int32_t M, int32_t top_k, int32_t num_experts
  *   workspace   device buffer of at least moe_workspace_bytes(...) bytes,
  *               zeroed once (moe_workspace_reset) before its first use.
  * Supported: H and I multiples of 32, 32 <= H <= 3840, 32 <= I <= 65536,
- * E <= 1024, 1 <= top_k <= 8 and top_k <= E.  The call is one cooperative
- * launch (one CTA per SM, all resident).  Each distinct routed expert is
+ * E <= 1024, 1 <= top_k <= 8 and top_k <= E.  The call is one launch of
+ * one CTA per SM, all resident (a kernel of another process that holds SMs
+ * for over a second makes it return MOE_ERR_TIMEOUT).  Each distinct routed expert is
  * streamed once per call, however many of the M tokens chose it.  The
  * output is the same on every call with the same inputs (a fixed summation
  * order on a given GPU).

@@ -270,7 +270,7 @@ moe_status moe_workspace_status(void* workspace, void* stream) {
 moe_status moe_query_path(char* buf, size_t n) {
   if (!buf || n == 0) return MOE_ERR_INVALID_ARG;
   const char* desc =
-      "sm_100a; moe: one cooperative persistent kernel (router fp32 GEMV with epoch-tagged logits, "
+      "sm_100a; moe: one persistent kernel, one CTA per SM (router fp32 GEMV with epoch-tagged logits, "
       "top-k softmax routing in every CTA, split-K over the intermediate: 16-row slices of MXFP4 "
       "E2M1/E8M0-32 gate/up + SiLU + down per work item, one bulk copy per item into a stage ring, "
       "gate/up as tcgen05.mma kind::mxf4 block-scaled on a 128-row operand of four K segments (TMEM "

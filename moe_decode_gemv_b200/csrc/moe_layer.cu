@@ -1,6 +1,6 @@
 // moe_layer.cu -- the whole MoE layer (router GEMV, top-k softmax routing,
 // MXFP4 gate/up GEMV + SiLU gate, down GEMV, shared expert, weighted
-// combine) as one cooperative persistent kernel, for M <= 4 tokens.
+// combine) as one persistent kernel, for M <= 4 tokens.
 //
 // The pages: each token goes to 8 of 512 routed experts plus a shared expert
 // that always runs (saipien.org essay, "Why one user waits on weights"); the
@@ -10,7 +10,7 @@
 // layer is bound by weight reads, so the kernel keeps as many weight bytes in
 // flight as it can and synchronises the grid once.
 //
-//  * One CTA per SM (cooperative launch: all CTAs resident), 16 warps.
+//  * One CTA per SM (all CTAs resident; see launch_layer_t), 16 warps.
 //  * Work items split every expert along its intermediate dimension: item
 //    (slot, j) computes gate and up rows 16j .. 16j+15, h = silu(gate) * up
 //    for those rows, and applies the matching 16 columns of the down matrix
@@ -226,7 +226,7 @@ struct VI {
 // larger padding ids, so padded lists stay sorted.
 __device__ __forceinline__ VI pad_entry(int pos) { return VI{-FLT_MAX, 0x7fffff00 + pos}; }
 
-// Grid barrier on one word (all CTAs are resident: cooperative launch).  The
+// Grid barrier on one word (all CTAs are resident; see launch_layer_t).  The
 // first CTA adds 2^31 - (G - 1), the others 1, so the top bit flips exactly
 // when all G have arrived and the low bits return to where they were: the
 // same word serves every call.  Arrival publishes the caller's earlier writes
@@ -924,12 +924,15 @@ cudaError_t launch_layer_t(const LayerArgs& a, cudaStream_t st) {
   const int grid = sms < MoeWs::kMaxGrid ? sms : MoeWs::kMaxGrid;  // one CTA per SM, all resident
   const size_t smem =
       (size_t)kCtlBytes + scratch_bytes(a.H, a.M, a.E) + geo.xparts_bytes + (size_t)a.stages * geo.stage_bytes;
-  // A cooperative launch: every CTA resident before any starts.  A regular
-  // launch let the next layer start 1.1 us after the LM head's last CTA
-  // instead of 5.4 us, but the GPU test suite then failed in a later LM-head
-  // test (an unspecified launch failure, reproducible, and only with
-  // asynchronous launches), so the cooperative launch stays.
-  e = launch_dependent(moe_layer_kernel<kB>, dim3(grid), dim3(kThreads), smem, st, true, a);
+  // A regular launch, not a cooperative one: a cooperative launch waits for the
+  // whole previous kernel to finish (about 5 us after the LM head's last CTA),
+  // while this one's CTAs take SMs as the previous kernel's CTAs leave.  All
+  // G CTAs (one per SM, the shared memory allows no second) still become
+  // resident: nothing launched after this kernel starts before every CTA
+  // has run griddepcontrol.launch_dependents, and kernels before it finish
+  // on their own.  Should another process hold SMs, the grid barrier's wait
+  // is bounded and the call reports MOE_ERR_TIMEOUT instead of hanging.
+  e = launch_dependent(moe_layer_kernel<kB>, dim3(grid), dim3(kThreads), smem, st, false, a);
   return e;
 }
 
