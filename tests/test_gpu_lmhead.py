@@ -139,6 +139,30 @@ def test_repeat_calls_identical(B, tiny):
 
 
 @pytest.mark.parametrize("M", [1, 4])
+def test_ling_head_back_to_back_calls_identical(B, ling, M):
+    """The full head, 24 calls queued back to back on one stream (each call's
+    CTAs start as the previous call's leave): every call's logits and top-k
+    bit-identical to the first.  A ring whose stages alternated between the
+    two consumer groups once let a group compute the other group's tile and
+    leave rows of the logits unwritten; this catches that class of race."""
+    w, head, q, s = ling
+    x = I.hidden_states(5, M, I.LING_HEAD.hidden, tag="lmhead").cuda()
+    ws = B.new_workspace(B.lmhead_workspace_bytes(M, 29, I.LING_HEAD.vocab, I.LING_HEAD.hidden))
+    outs = [(torch.empty((M, 29), dtype=torch.int32, device="cuda"), torch.empty((M, 29), dtype=torch.float32, device="cuda"),
+             torch.full((M, I.LING_HEAD.vocab), float("nan"), dtype=torch.float32, device="cuda")) for _ in range(24)]
+    for ids, vals, logits in outs:
+        B.lmhead_decode(x, head, 29, ids, vals, logits, workspace=ws)
+    torch.cuda.synchronize()
+    assert B.moe_workspace_status(ws) == B.Status.OK
+    ids0, vals0, lg0 = (t.cpu().numpy() for t in outs[0])
+    assert np.isfinite(lg0).all()
+    for c, (ids, vals, logits) in enumerate(outs[1:], 1):
+        assert np.array_equal(ids.cpu().numpy(), ids0), f"call {c}: ids differ"
+        assert np.array_equal(vals.cpu().numpy(), vals0), f"call {c}: values differ"
+        assert np.array_equal(logits.cpu().numpy(), lg0), f"call {c}: logits differ"
+
+
+@pytest.mark.parametrize("M", [1, 4])
 def test_ling_head_outlier_tokens(B, O, ling, M):
     """A token with one element at 1e3 among 1e-3 values (and, at M = 4, a
     plain token, a negative outlier and a scaled token beside it)."""

@@ -149,6 +149,29 @@ def test_ling_layer(B, O, ling, M):
             assert len(set(ids.reshape(-1).tolist())) <= 32
 
 
+@pytest.mark.parametrize("M", [1, 4])
+def test_ling_layer_back_to_back_calls_identical(B, ling, M):
+    """24 calls of the Ling layer queued back to back on one stream, sharing
+    one workspace (each call's CTAs start as the previous call's leave): every
+    call's output, ids and weights bit-identical to the first."""
+    k, H = ling.shape.top_k, ling.shape.hidden
+    x = I.hidden_states(6, M, H, tag="back2back").cuda()
+    ws = B.new_workspace(B.moe_workspace_bytes(M, k, ling.shape.experts, H, ling.shape.inter))
+    outs = [(torch.full((M, H), float("nan"), dtype=torch.float32, device="cuda"),
+             torch.empty((M, k), dtype=torch.int32, device="cuda"), torch.empty((M, k), dtype=torch.float32, device="cuda"))
+            for _ in range(24)]
+    for y, ids, w in outs:
+        B.moe_decode(x, ling.router_w_dev, ling.router_bias_dev, ling.packed, ling.packed_shared, k, y, ids, w,
+                     workspace=ws)
+    torch.cuda.synchronize()
+    assert B.moe_workspace_status(ws) == B.Status.OK
+    first = [t.cpu().numpy() for t in outs[0]]
+    assert np.isfinite(first[0]).all()
+    for c, o in enumerate(outs[1:], 1):
+        for a, b in zip(o, first):
+            assert np.array_equal(a.cpu().numpy(), b), f"call {c} differs"
+
+
 def test_ling_layer_skewed_m4(B, O, ling_skewed):
     """Skewed router (per-expert logit bias N(0, 2^2)): tokens share experts."""
     x = I.hidden_states(0, 4, I.LING_MOE.hidden, tag="skew")
