@@ -285,7 +285,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
     fence_mbar_init();
     C.poison = 0;
     C.shifted = 0;
-    top_up(n_pre);  // the shared expert's items: weights, which no kernel writes
   }
   if (warp == 0) tmem_alloc(&C.tmem, kTmemCols);  // one CTA per SM: all of the SM's TMEM
 
@@ -318,6 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   tc_fence_before_sync();
   __syncthreads();  // the barriers are initialised, TMEM is allocated
   tc_fence_after_sync();
+  // The shared expert's items (weights, which no kernel writes) go out after
+  // the router rows: those are on the path to routing, these are needed
+  // only after it.
+  top_up(n_pre);
   const uint32_t tm = C.tmem;
   const int T = geo.kt;
   const uint32_t tm_sfb = kTmemSfa + 4u * (uint32_t)T;  // the activation parts' scales: 4 columns per K tile
