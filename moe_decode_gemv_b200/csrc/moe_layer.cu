@@ -20,16 +20,18 @@
 //    brought into a ring of shared-memory stages by bulk copies (no
 //    multicast) that complete on an mbarrier per stage.  Item q goes to CTA
 //    q mod G; the shared expert's items come first, so the CTAs that own them
-//    start streaming and computing before routing is known.
+//    stream those bytes while routing runs.
 //  * Router: the tokens are copied into shared memory at once; each CTA
 //    scores its share of the router rows (fp32 weights, bf16 activations,
 //    fp32 sums) and publishes each logit as one 64-bit word (epoch tag << 32
-//    | value), so that readers need no barrier: every CTA polls the words
-//    until all carry this call's tag, then takes the same top-k and builds
-//    the same slot table (slot 0 = shared expert, then each distinct routed
-//    expert once).  Top-k, one warp per token: the k-th best of the 32 lane
-//    maxima bounds the k-th best logit from below, and the few logits not
-//    worse than that bound are ranked by counting.
+//    | value), so that readers need no barrier.  Then warps 0..7 poll the
+//    words until all carry this call's tag, take the same top-k as every
+//    other CTA and build the same slot table (slot 0 = shared expert, then
+//    each distinct routed expert once), while warps 8..15 turn the tokens
+//    into the gate/up MMA's operand.  Top-k, one warp per token: the k-th
+//    best of the 32 lane maxima bounds the k-th best logit from below, and
+//    the few logits not worse than that bound are ranked by counting; at
+//    M = 1 the routed items are issued as soon as they are ranked.
 //  * Each lane owns a fixed set of output rows and accumulates its CTA's
 //    weighted contributions in registers across items.  After the last item
 //    the CTAs write these partial outputs, meet at one grid barrier, and sum
