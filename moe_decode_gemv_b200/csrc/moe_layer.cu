@@ -185,11 +185,11 @@ __device__ __forceinline__ float4 ld_router(const float* p, uint64_t policy) {
   return r;
 }
 
-// ---- power-of-two scaling of activation blocks ----
-// sigma such that amax * 2^sigma lies in [2^7, 2^8) (the top of E4M3's normal
-// range, max 448), clamped to [-113, 140] so that 2^(14 - sigma) is a normal
-// fp32 number; 140 covers every bf16 value (the smallest is 2^-133).  0 for
-// amax = 0 (or NaN).
+// ---- power-of-two scaling of h ----
+// sigma such that amax * 2^sigma lies in [2^7, 2^8), clamped to [-113, 140]
+// so that 2^(14 - sigma) is a normal fp32 number; 140 covers every bf16
+// value (the smallest is 2^-133).  0 for amax = 0 (or NaN).  h's slice uses
+// sigma + 7, which puts its largest magnitude in [2^14, 2^15).
 __device__ __forceinline__ int pow2_sigma(float amax) {
   if (!(amax > 0.f)) return 0;
   const uint32_t b = __float_as_uint(amax);
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_layer_kernel(LayerArgs a) {
   top_up(n_pre);
   const uint32_t tm = C.tmem;
   const int T = geo.kt;
-  const uint32_t tm_sfb = kTmemSfa + 4u * (uint32_t)T;  // the activation parts' scales: 4 columns per K tile
+  const uint32_t tm_sfb = kTmemSfa + 4u * (uint32_t)T;  // the activation digits' scales: 4 columns per K tile
   // Everything below may read what the previous kernel on the stream wrote
   // (the tokens, the workspace): wait for it.  The weight copies and loads
   // above are already on their way.
