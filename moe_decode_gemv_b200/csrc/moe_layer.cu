@@ -210,12 +210,6 @@ __device__ __forceinline__ int floor_log2(float a) {
   const int e = (int)((b >> 23) & 0xffu);
   return e ? e - 127 : (31 - __clz(b & 0x7fffffu)) - 149;
 }
-// The value of an E2M1 code (bit 3 the sign): 0, 0.5, 1, 1.5, 2, 3, 4, 6.
-__device__ __forceinline__ float e2m1_value(uint32_t c) {
-  const uint32_t m = c & 7u;
-  const float v = m >= 2u ? (float)(2u + (m & 1u)) * exp2i((int)(m >> 1) - 2) : 0.5f * (float)m;
-  return (c & 8u) ? -v : v;
-}
 
 // ---- routing: the best 8 of up to 1,024 logits across warps ----
 // (value, expert) pairs under `better`: larger value first, lower id on ties.
