@@ -217,6 +217,18 @@ def pin_mxfp4_quantize(O) -> None:
     assert scales[1, 0] == 127 and got_codes[1, 0] == 7      # 7.0 saturates to 6.0 * 2^0
     assert scales[2, 0] == 127 - 6 and got_codes[2, 5] == 15  # -0.1 -> -6 * 2^-6
 
+    # a non-finite input survives quantisation as NaN: under OCP MX a NaN
+    # scale makes every element of its block NaN when decoded (here by the
+    # library's E8M0 decoder); the row's other blocks stay finite
+    nf = (torch.randn(3, 64, generator=g) * 0.02).to(torch.bfloat16)
+    nf[0, 3] = float("inf")
+    nf[1, 40] = float("-inf")
+    nf[2, 7] = float("nan")
+    d2, s2 = O.mxfp4_quantize(_bf16_bits(nf))
+    deq2 = lib_mxfp4_dequant(d2, s2).reshape(3, 2, 32)
+    bad = np.array([[True, False], [False, True], [True, False]])
+    assert np.isnan(deq2[bad]).all() and np.isfinite(deq2[~bad]).all()
+
 
 def pin_mxfp4_roundtrip(O) -> None:
     g = torch.Generator().manual_seed(12)
@@ -396,14 +408,17 @@ def pin_topk(O) -> None:
 
 def pin_rmsnorm(O) -> None:
     rng = np.random.default_rng(71)
-    y = rng.normal(0, 5, 256)
-    got = lib_bf16(O.rmsnorm_bf16(y, 1e-6))
-    r = torch.nn.functional.rms_norm(torch.from_numpy(y), (256,), eps=1e-6).numpy()
-    # each output is one of the two bf16 neighbours of the exact value, the nearer one
-    for a, b in zip(got.tolist(), r.tolist()):
-        lo, hi = _bf16_neighbours(abs(b))
-        lo, hi = (lo, hi) if b >= 0 else (-hi, -lo)
-        assert a in (lo, hi) and abs(a - b) <= abs((hi if a == lo else lo) - b) + 1e-300, (a, b)
+    # unit-scale values, and values small enough that eps (inside the square
+    # root) changes the result by several bf16 steps
+    for sd, eps in ((5.0, 1e-6), (1e-3, 1e-6)):
+        y = rng.normal(0, sd, 256)
+        got = lib_bf16(O.rmsnorm_bf16(y, eps))
+        r = torch.nn.functional.rms_norm(torch.from_numpy(y), (256,), eps=eps).numpy()
+        # each output is one of the two bf16 neighbours of the exact value, the nearer one
+        for a, b in zip(got.tolist(), r.tolist()):
+            lo, hi = _bf16_neighbours(abs(b))
+            lo, hi = (lo, hi) if b >= 0 else (-hi, -lo)
+            assert a in (lo, hi) and abs(a - b) <= abs((hi if a == lo else lo) - b) + 1e-300, (a, b)
 
 
 def pin_sample_topk(O) -> None:

@@ -49,6 +49,33 @@ MUTATIONS = {
     "sample_nucleus_inclusive": ("while (n < k && before < top_p * total) {", "while (n < k && before <= top_p * total) {"),
     "sample_draw_unnormalised": ("const double r = u * kept;", "const double r = u * total;"),
     "mtp_accept_skips_mismatch": ("while (a < D && draft[a] == verify[a]) {", "while (a < D && draft[a] != verify[a] + 1) {"),
+    # a second batch: indexing, sign and special-value slips
+    "e2m1_sign_bit": ("unsigned s = (code >> 3) & 1u, e = (code >> 1) & 3u", "unsigned s = (code >> 2) & 1u, e = (code >> 1) & 3u"),
+    "e8m0_nan_as_inf": ("        return NAN;\n    return ldexp(1.0, (int)code - 127);",
+                        "        return INFINITY;\n    return ldexp(1.0, (int)code - 127);"),
+    "e4m3_subnormal_scale": ("ldexp((double)m, -9) : ldexp", "ldexp((double)m, -10) : ldexp"),
+    "e4m3_binade_carry": ("            t = 8.0;\n            E += 1;", "            t = 8.0;"),
+    "bf16_sign_dropped": ("return signbit(v) ? (uint16_t)(b | 0x8000u) : b;", "return b;"),
+    "mx_block_scale_index": ("g_e8m0[scales[r * (K / 32) + j / 32]]", "g_e8m0[scales[r * (K / 32)]]"),
+    "mx_nonfinite_block_scale": ("scales[r * nb + b] = 0xFFu;", "scales[r * nb + b] = 0x00u;"),
+    "mx_zero_block_scale": ("                xexp = -127;\n            } else {", "                xexp = 0;\n            } else {"),
+    "fp8_amax_signed": ("float a = fabsf((float)orc_bf16_to_double(row[j]));", "float a = (float)orc_bf16_to_double(row[j]);"),
+    "fp8_zero_row_scale": ("(amax == 0.0f) ? 1.0f : amax / 448.0f", "(amax == 0.0f) ? 0.0f : amax / 448.0f"),
+    "topk_ascending": ("if (best < 0 || v[j] > v[best])", "if (best < 0 || v[j] < v[best])"),
+    "router_token0": ("acc += orc_bf16_to_double(x_bf16[(int64_t)m * H + j]) * (double)Wr[(int64_t)e * H + j];",
+                      "acc += orc_bf16_to_double(x_bf16[j]) * (double)Wr[(int64_t)e * H + j];"),
+    "router_not_renormalised": ("        for (int i = 0; i < k; ++i)\n            z += exp(sel[i] - sel[0]);",
+                                "        for (int i = 0; i < E; ++i)\n            z += exp(lg[i] - sel[0]);"),
+    "down_uses_gate_scales": ("orc_mxfp4_element(I, down_d, down_s, i, r)", "orc_mxfp4_element(I, down_d, gate_s, i, r)"),
+    "layer_token0": ("const uint16_t* xm = x_bf16 + (int64_t)m * H;", "const uint16_t* xm = x_bf16;"),
+    "shared_weighted": ("        for (int j = 0; j < H; ++j)\n            ym[j] += out[j];",
+                        "        for (int j = 0; j < H; ++j)\n            ym[j] += w[(int64_t)m * k] * out[j];"),
+    "lmhead_token0": ("            xd[j] = orc_bf16_to_double(x_bf16[(int64_t)m * H + j]);\n        for (int64_t v = 0; v < V; ++v) {\n            const uint8_t* row",
+                      "            xd[j] = orc_bf16_to_double(x_bf16[j]);\n        for (int64_t v = 0; v < V; ++v) {\n            const uint8_t* row"),
+    "lmhead_bf16_token0": ("            xd[j] = orc_bf16_to_double(x_bf16[(int64_t)m * H + j]);\n        for (int64_t v = 0; v < V; ++v) {\n            double acc",
+                           "            xd[j] = orc_bf16_to_double(x_bf16[j]);\n        for (int64_t v = 0; v < V; ++v) {\n            double acc"),
+    "rmsnorm_eps_outside": ("sqrt(ss / (double)H + eps)", "sqrt(ss / (double)H) + eps"),
+    "mtp_emits_draft_after_accept": ("        emitted[a] = draft[a];\n        ++a;", "        emitted[a] = verify[a + 1 < D ? a + 1 : a];\n        ++a;"),
 }
 
 
