@@ -268,9 +268,9 @@ MOE_API size_t lmhead_workspace_bytes(int32_t M, int32_t top_k, int64_t vocab, i
  *   workspace: at least lmhead_workspace_bytes(...), zeroed once before use.
  * Supported: hidden a multiple of 64 and at most 5120, vocab < 2^31, and a
  * vocabulary whose logits fit in shared memory across the GPU's SMs while the
- * head streams (each CTA keeps its rows' M logits: on a 148-SM B200 about
- * 1.2 M rows at M = 4 and H = 2560); larger returns
- * MOE_ERR_UNSUPPORTED_SHAPE.                                                */
+ * head streams (each CTA keeps its rows' M logits and candidates: on a
+ * 148-SM B200 with H = 2560, about 1.8 M rows at M = 1 and 430 K rows at
+ * M = 4); larger returns MOE_ERR_UNSUPPORTED_SHAPE.                          */
 MOE_API moe_status lmhead_decode(const uint16_t* hidden_bf16, const moe_fp8_head* head,
                          int32_t M, int32_t top_k, int32_t* topk_ids, float* topk_vals,
                          float* logits, void* workspace, size_t workspace_bytes, void* stream);
