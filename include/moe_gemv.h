@@ -373,9 +373,11 @@ MOE_API moe_status moe_workspace_reset(void* workspace, size_t workspace_bytes, 
 MOE_API moe_status moe_workspace_status(void* workspace, void* stream);
 
 /* Write a NUL-terminated description of the compiled kernels and formats
- * ("sm_100a ...") into buf.  The pages advise confirming at startup that each
- * optimisation is live (ncijnetwork.com summary, "The integration trap");
- * this is the string to log.                                                 */
+ * ("sm_100a ...") into buf of n bytes.  The pages advise confirming at startup
+ * that each optimisation is live (ncijnetwork.com summary, "The integration
+ * trap"); this is the string to log.  A buffer too small for the whole text
+ * (1 KB always suffices) gets its first n - 1 characters, NUL-terminated, and
+ * the call returns MOE_ERR_INVALID_ARG.                                      */
 MOE_API moe_status moe_query_path(char* buf, size_t n);
 
 /* Self-test of the bounded device waits; the pages have no counterpart.

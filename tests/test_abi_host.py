@@ -56,7 +56,7 @@ def test_workspace_sizes(lib):
     assert lib.moe_workspace_bytes(1, 9, 512, 2560, 768) == 0          # top_k > 8
     assert lib.moe_workspace_bytes(1, 8, 512, 2561, 768) == 0          # H not a multiple of 32
     assert lib.moe_workspace_bytes(1, 8, 512, 2560, 80) == 0           # I not a multiple of 32
-    assert lib.moe_workspace_bytes(1, 8, 512, 3872, 768) == 0          # H above 3840 (TMEM columns)
+    assert lib.moe_workspace_bytes(1, 8, 512, 3872, 768) == 0          # H above 3840 (shared memory)
     assert lib.moe_workspace_bytes(1, 8, 512, 3840, 768) > 0
     assert lib.moe_workspace_bytes(1, 8, 1025, 2560, 768) == 0         # more than 1024 experts
     assert lib.moe_workspace_bytes(1, 8, 512, 96, 32) > 0              # the smallest odd sizes
@@ -195,3 +195,73 @@ def test_sampling_and_accept_reject_bad_arguments(lib):
     assert L.moe_mtp_accept(A, A, 65, A, A, None) == S.INVALID_ARG
     assert L.moe_mtp_accept(A, None, 3, A, A, None) == S.INVALID_ARG
     assert L.moe_mtp_accept(A, A + 1, 3, A, A, None) == S.MISALIGNED
+
+
+def test_moe_decode_rejects_out_of_range_shapes_and_pointers(lib):
+    S, L = lib.Status, lib.library
+    ok_bank, ok_shared = _packed(lib), _packed(lib, E=1)
+    assert _decode(lib, _packed(lib, E=4), ok_shared, top_k=8) == S.UNSUPPORTED_SHAPE           # top_k > E
+    assert _decode(lib, _packed(lib, E=1025), ok_shared) == S.UNSUPPORTED_SHAPE                 # E > 1024
+    assert _decode(lib, _packed(lib, H=3872), _packed(lib, E=1, H=3872)) == S.UNSUPPORTED_SHAPE  # H > 3840
+    assert _decode(lib, _packed(lib, I=65568), _packed(lib, E=1, I=65568)) == S.UNSUPPORTED_SHAPE
+    assert _decode(lib, ok_bank, ok_shared, ws=0) == S.INVALID_ARG
+    assert _decode(lib, ok_bank, ok_shared, ws=U) == S.MISALIGNED
+
+    def call(router_w=A, bias=None, out=A, ids=None, w=None):
+        return L.moe_decode(A, router_w, bias, ctypes.byref(ok_bank), ctypes.byref(ok_shared), 1, 2, out, ids, w,
+                            A, 1 << 24, None)
+
+    assert call(router_w=None) == S.INVALID_ARG
+    assert call(out=None) == S.INVALID_ARG
+    assert call(router_w=U) == S.MISALIGNED
+    assert call(bias=U) == S.MISALIGNED
+    assert call(out=U) == S.MISALIGNED
+    assert call(ids=U) == S.MISALIGNED
+    assert call(w=U) == S.MISALIGNED
+    # a NULL experts or shared bank is an argument error, not a crash
+    assert L.moe_decode(A, A, None, None, ctypes.byref(ok_shared), 1, 2, A, None, None, A, 1 << 24,
+                        None) == S.INVALID_ARG
+    assert L.moe_decode(A, A, None, ctypes.byref(ok_bank), None, 1, 2, A, None, None, A, 1 << 24,
+                        None) == S.INVALID_ARG
+
+
+def test_stream_glue_and_housekeeping_reject_bad_arguments(lib):
+    S, L = lib.Status, lib.library
+    # RMSNorm between layers: y [M][H] fp32 -> bf16, H a multiple of 8, eps >= 0
+    assert L.moe_rmsnorm_bf16(None, 1, 256, 1e-6, A, None) == S.INVALID_ARG
+    assert L.moe_rmsnorm_bf16(A, 0, 256, 1e-6, A, None) == S.INVALID_ARG
+    assert L.moe_rmsnorm_bf16(A, 1, 100, 1e-6, A, None) == S.INVALID_ARG
+    assert L.moe_rmsnorm_bf16(A, 1, 256, -1.0, A, None) == S.INVALID_ARG
+    assert L.moe_rmsnorm_bf16(A, 1, 256, float("nan"), A, None) == S.INVALID_ARG
+    assert L.moe_rmsnorm_bf16(U, 1, 256, 1e-6, A, None) == S.MISALIGNED
+    assert L.moe_rmsnorm_bf16(A, 1, 256, 1e-6, U, None) == S.MISALIGNED
+    # embedding gather for the next step's input
+    assert L.moe_embed_gather(A, 0, 256, A, 1, 1, A, None) == S.INVALID_ARG
+    assert L.moe_embed_gather(A, 1000, 12, A, 1, 1, A, None) == S.INVALID_ARG
+    assert L.moe_embed_gather(A, 1000, 256, None, 1, 1, A, None) == S.INVALID_ARG
+    assert L.moe_embed_gather(A, 1000, 256, A, 0, 1, A, None) == S.INVALID_ARG
+    assert L.moe_embed_gather(A, 1000, 256, A, 1, 0, A, None) == S.INVALID_ARG
+    assert L.moe_embed_gather(U, 1000, 256, A, 1, 1, A, None) == S.MISALIGNED
+    assert L.moe_embed_gather(A, 1000, 256, A + 2, 1, 1, A, None) == S.MISALIGNED
+    # the read-ceiling probe: whole 16-byte words from an aligned source
+    assert L.moe_stream_read(A, 8, A, None) == S.INVALID_ARG
+    assert L.moe_stream_read(A, 24, A, None) == S.INVALID_ARG
+    assert L.moe_stream_read(None, 1 << 20, A, None) == S.INVALID_ARG
+    assert L.moe_stream_read(U, 1 << 20, A, None) == S.MISALIGNED
+    assert L.moe_stream_read(A, 1 << 20, A + 2, None) == S.MISALIGNED
+    # workspaces and the bounded-wait self-test
+    assert L.moe_workspace_reset(None, 1 << 20, None) == S.INVALID_ARG
+    assert L.moe_workspace_reset(A, 8, None) == S.INVALID_ARG
+    assert L.moe_workspace_status(None, None) == S.INVALID_ARG
+    assert L.moe_selftest_wait_timeout(None, 64, 100, None) == S.WORKSPACE
+    assert L.moe_selftest_wait_timeout(A, 8, 100, None) == S.WORKSPACE
+    assert L.moe_selftest_wait_timeout(U, 64, 100, None) == S.MISALIGNED
+    assert L.moe_selftest_wait_timeout(A, 64, 0, None) == S.INVALID_ARG
+    assert L.moe_selftest_wait_timeout(A, 64, 1000001, None) == S.INVALID_ARG
+    buf = ctypes.create_string_buffer(8)
+    assert L.moe_query_path(None, 8) == S.INVALID_ARG
+    assert L.moe_query_path(buf, 0) == S.INVALID_ARG
+    # too small: the text's beginning, NUL-terminated, and an argument error
+    assert L.moe_query_path(buf, 8) == S.INVALID_ARG and buf.value == b"sm_100a"
+    big = ctypes.create_string_buffer(1024)
+    assert L.moe_query_path(big, 1024) == S.OK and big.value.startswith(b"sm_100a;")
