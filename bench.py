@@ -678,11 +678,38 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def source_code_only(text: str) -> str:
+    """C/CUDA source without its comments, whitespace runs collapsed: what
+    the compiler sees, so that editing a comment keeps a profile valid."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":                       # a string or character literal, copied whole
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):       # a line comment
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):       # a block comment
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the LM-head kernel's code (comments and layout excluded)."""
     h = hashlib.sha256()
     for name in ("lmhead_fp8.cu", "common.cuh"):
-        with open(os.path.join(ROOT, "moe_decode_gemv_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "moe_decode_gemv_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(source_code_only(f.read()).encode())
+            h.update(b"\0")
     return h.hexdigest()[:16]
 
 

@@ -15,7 +15,9 @@
 //    different rates finish together.  A producer warp streams the tiles into
 //    a ring of shared-memory stages, one bulk copy (no multicast) per tile
 //    plus one for its 16 row scales, completing on an mbarrier per stage; the
-//    ring keeps four or five tiles (~160-200 KB) in flight per SM.
+//    ring keeps four tiles (~160 KB) in flight per SM, two when a call's other
+//    shared-memory needs leave no room for four (always an even count: see
+//    lmhead_fp8_plan).
 //  * Two groups of ten consumer warps take alternate tiles, so that each
 //    group has two tiles' time for one: warp w of a group takes 64-byte
 //    slices w, w + 10, ... of its tiles, loads its A fragments from the stage

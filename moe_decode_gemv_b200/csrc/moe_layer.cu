@@ -49,8 +49,9 @@
 //    (segment s of A with segment s of B) of the product is read.  The
 //    digits carry a bf16 value exactly when it is within 2^-8 of its block's
 //    largest, and to within 2^-16 of the largest below.  The tensor core
-//    applies both scales, so no instruction decodes a weight; an MMA takes
-//    about 75 cycles, a fifth of the time the item's bytes take to arrive.
+//    applies both scales, so no instruction decodes a weight.  An MMA takes
+//    about 75 cycles: an item's ten (H = 2,560) take about a quarter of the
+//    time its 64 KB take to arrive at one SM's share of HBM bandwidth.
 //  * h: per token and item (16 values), scaled by a power of two that puts
 //    the largest magnitude in [2^14, 2^15) and carried by two f16 parts (about
 //    22 significant bits) into mma.sync m16n8k16 f16 x f16 -> fp32, whose K of

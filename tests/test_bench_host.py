@@ -87,9 +87,18 @@ def test_traffic_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch)
             (src / name).write_bytes(f.read())
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.profiled_traffic() == 409988352.0
-    # any change to the kernel source voids the stored counters
-    (src / "common.cuh").write_bytes((src / "common.cuh").read_bytes() + b"\n")
+    # a comment or a blank line is not a change of the kernel
+    (src / "common.cuh").write_bytes((src / "common.cuh").read_bytes() + b"\n// a note, 'quoted'\n/* more */\n")
+    assert bench.profiled_traffic() == 409988352.0
+    # any change to the code voids the stored counters
+    (src / "common.cuh").write_bytes((src / "common.cuh").read_bytes() + b"\nnamespace { int unused_x; }\n")
     assert bench.profiled_traffic() is None
+
+
+def test_source_code_only_strips_comments_not_literals():
+    bench = _bench()
+    t = 'int a = 1;  // x\n/* y\n z */ const char* s = "a // b /* c */";\nchar q = \'"\'; char r = \'\\\'\';'
+    assert bench.source_code_only(t) == 'int a = 1; const char* s = "a // b /* c */"; char q = \'"\'; char r = \'\\\'\';'
 
 
 def test_workload_config_names_the_workload():
