@@ -1,5 +1,5 @@
-// lmhead_kernels.cu -- the BF16 comparator head: the same GEMV + per-row
-// scale-free top-k as the FP8 head (lmhead_fp8.cu) over the unquantised BF16
+// lmhead_kernels.cu -- the BF16 comparator head: the same GEMV + top-k as the
+// FP8 head (lmhead_fp8.cu), without a row scale, over the unquantised BF16
 // [V][H] head, which the FP8 head halves in bytes.  One pass over the head
 // for all M tokens, fused with an optional logits write and a top-k.
 //
@@ -17,8 +17,8 @@
 //  * Eight consumer warps split K, each computing 16 rows x 8 token columns
 //    with mma.sync m16n8k16 (bf16 x bf16 -> fp32); the B fragments hold the
 //    tokens and stay in registers for the whole kernel.
-//  * An epilogue warp sums the consumers' partials, writes logits when asked
-//    and keeps each value in shared memory; after the stream one warp per
+//  * Two epilogue warps, on alternate tiles, sum the consumers' partials,
+//    write logits when asked and keep each value in shared memory; after the stream one warp per
 //    token takes the CTA's top-k, and the last CTA to finish merges all
 //    CTAs' lists (ties to the lower id).
 #include <cuda_runtime.h>

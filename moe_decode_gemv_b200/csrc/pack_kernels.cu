@@ -1,7 +1,8 @@
 // pack_kernels.cu -- load-time re-layout of MXFP4 expert banks for moe_decode
 // into the sliced layout of pack.h: one contiguous unit per work item, with
-// the bytes in the order the kernel's MMA fragments take them, plus the down
-// scales per 32-column pair.  Load time only; the kernels gather bytes one
+// the bytes in the order the kernel's MMAs read them (the tensor core's
+// K-major gate/up operand and its scales, then the down fragments), plus the
+// down scales per 32-column pair.  Load time only; the kernels gather bytes one
 // at a time and favour plainness over speed.
 #include <cuda_runtime.h>
 
