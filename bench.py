@@ -669,13 +669,27 @@ def reference_arm(args):
 # roofline bookkeeping
 # ---------------------------------------------------------------------------
 
+FALLBACK_HBM_GBS = 6650.0  # an earlier copy-bandwidth measurement on this kind of B200
+
+
 def measured_peaks():
+    """The HBM copy bandwidth the roofline divides by: the measured figure
+    from MEASURED_PEAKS.json (`hbm_gbs`, a number or an object with a
+    `value`), else the fallback, with the reason in the kind string."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
+    if not os.path.exists(p):
+        return FALLBACK_HBM_GBS, "fallback"
+    try:
         with open(p) as f:
-            d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+            v = json.load(f)["hbm_gbs"]
+        if isinstance(v, dict):
+            v = v["value"]
+        v = float(v)
+        if not (v > 0 and v < 1e5):
+            raise ValueError(f"hbm_gbs = {v}")
+        return v, "measured"
+    except (OSError, ValueError, KeyError, TypeError) as exc:
+        return FALLBACK_HBM_GBS, f"fallback (MEASURED_PEAKS.json unreadable: {type(exc).__name__})"
 
 
 def source_code_only(text: str) -> str:

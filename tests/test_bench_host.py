@@ -117,3 +117,18 @@ def test_block_steps_gives_at_least_ten_blocks():
     assert bench.block_steps(199) == 19
     assert bench.block_steps(30) == 3
     assert bench.block_steps(3) == 1
+
+
+def test_measured_peak_is_read_or_falls_back(tmp_path, monkeypatch):
+    bench = _bench()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_peaks() == (bench.FALLBACK_HBM_GBS, "fallback")
+    f = tmp_path / "MEASURED_PEAKS.json"
+    f.write_text('{"hbm_gbs": 6558.4, "bf16_tflops": 1590}')
+    assert bench.measured_peaks() == (6558.4, "measured")
+    f.write_text('{"hbm_gbs": {"value": 6600, "unit": "GB/s"}}')
+    assert bench.measured_peaks() == (6600.0, "measured")
+    for bad in ('{"bf16_tflops": 1590}', '{"hbm_gbs": null}', '{"hbm_gbs": -1}', "not json"):
+        f.write_text(bad)
+        peak, kind = bench.measured_peaks()
+        assert peak == bench.FALLBACK_HBM_GBS and kind.startswith("fallback (")
