@@ -846,7 +846,10 @@ def main():
         except Exception as exc:  # the headline numbers above stand without this leg
             line["stream_16_layers"] = {"error": f"{type(exc).__name__}: {str(exc).splitlines()[0][:200]}"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.seed)
+        try:
+            line["cpu_baseline"] = cpu_baseline(args.seed)
+        except Exception as exc:  # the GPU numbers above stand without the host leg
+            line["cpu_baseline"] = {"kind": "oracle", "error": f"{type(exc).__name__}: {str(exc).splitlines()[0][:200]}"}
     if dist is not None:
         dist.barrier()
     if rank == 0:
