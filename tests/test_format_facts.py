@@ -17,6 +17,11 @@ independent decoder (ml_dtypes) -- not against the kernels' own code.
   eight base-4 digits d_p, each an E2M1 code 0..3 (value d/2) with the
   value's sign at scale 2^(E-2p), sum to v exactly when v is within 2^-8 of
   the block's largest and to within 2^(E-16) of it below.
+* The MoE down step's h: an fp32 slice scaled by a power of two so that its
+  largest magnitude lies in [2^14, 2^15), then hi = f16(v) and
+  lo = f16(v - hi) (round to nearest even; v - hi is exact in fp32), gives
+  |v - (hi + lo)| <= 2^-8, i.e. 2^-22 of the slice's largest, with no f16
+  overflow; and an E2M1 value (as f16) times hi or lo is exact in fp32.
 """
 import itertools
 
@@ -126,3 +131,30 @@ def test_bf16_is_carried_by_eight_e2m1_digits(E):
     big = np.abs(v) >= 2.0 ** (E - 8)
     assert np.array_equal(total[big], v[big])
     assert np.all(np.abs(total - v) <= 2.0 ** (E - 16))
+
+
+def test_h_is_carried_by_two_f16_parts():
+    rng = np.random.default_rng(5)
+    # scaled slices: the largest magnitude in [2^14, 2^15), the rest spread
+    # over 40 binades below it (f16 subnormals included), signs mixed
+    top = rng.uniform(2.0 ** 14, 2.0 ** 15, 20000).astype(np.float32)
+    rest = (np.float32(2.0) ** rng.uniform(-26, 15, 200000).astype(np.float32)).astype(np.float32)
+    edge = np.array([2.0 ** 14, np.nextafter(np.float32(2.0 ** 15), np.float32(0)), 2.0 ** -24, 2.0 ** -25,
+                     3 * 2.0 ** -26, 2.0 ** -14, np.nextafter(np.float32(2.0 ** -14), np.float32(0)), 0.0],
+                    dtype=np.float32)
+    v = np.concatenate([top, rest, edge])
+    v = np.where(rng.random(v.size) < 0.5, -v, v).astype(np.float32)
+    hi = v.astype(np.float16)
+    r = (v - hi.astype(np.float32)).astype(np.float32)
+    # the residual is exact: it equals the fp64 difference
+    assert np.array_equal(r.astype(np.float64), v.astype(np.float64) - hi.astype(np.float64))
+    lo = r.astype(np.float16)
+    assert np.isfinite(hi).all() and np.isfinite(lo).all()
+    err = np.abs(v.astype(np.float64) - hi.astype(np.float64) - lo.astype(np.float64))
+    assert err.max() <= 2.0 ** -8
+    # the down MMA's products: E2M1 magnitudes {0.5 .. 6} times any f16 part
+    # need at most 11 + 2 significant bits, which fp32 holds exactly
+    e2m1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    parts = np.concatenate([hi, lo]).astype(np.float64)
+    prod = e2m1[:, None] * parts[None, :]
+    assert np.array_equal(prod.astype(np.float32).astype(np.float64), prod)
